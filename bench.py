@@ -1,0 +1,452 @@
+"""Benchmark: compressed-KV decode attention on B200 (one JSON line on rank 0).
+
+Workload (default ``llama8b``): Llama-3.1-8B-shaped decode, batch 1, 32 query /
+8 KV heads, head_dim 128, 32768 cached tokens per layer in 16-token pages, keys
+3-bit + QJL (m = 128), values 2-bit, 32 layers. One step = one generated token:
+for each of the 32 layers, quantize-append the new token's K/V (8 heads) and
+run decode attention for the 32 query heads over the whole cache. The 32 layer
+caches (about 0.86 GB) exceed the 126 MB L2, so every step streams from HBM.
+
+``value``   decode tokens/s with inputs resident in HBM (CUDA-graph replay of
+            K steps, CUDA events on the launching stream, max over ranks).
+``e2e``     the same steps through the C ABI with host buffers: per step the
+            new K/V and queries are copied from pinned host memory and the
+            attention outputs copied back, inside the timed region.
+``roofline`` decode attention (tq_decode_attention: query transform + split-K
+            decode) against the measured HBM copy bandwidth: algorithmic bytes =
+            compressed bytes of every cached token-head read (102 B each).
+``cpu_baseline`` the float64 oracle on the host, on a bounded sample.
+
+Multi-GPU: one process per GPU (torchrun); each rank serves its own sequence
+(weak scaling, no collective on the data path); value = all ranks' tokens /
+slowest rank's time.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV decode attention tokens/s & HBM GB/s vs roofline; quantize GB/s"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("tq_kernels.cu", "tq_host.cpp", "tq_internal.h"):
+        h.update(open(os.path.join(ROOT, "decode_attention_seeded_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind):
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches these sources."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get(kind)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while the GPU works."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _handle(self, device_index):
+        import torch
+        nv = self.nv
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            return nv.nvmlDeviceGetHandleByUUID(uuid.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(device_index)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- GPU workload
+class DecodeBench:
+    def __init__(self, wl, steps, warmup, device, rank):
+        import torch
+        from decode_attention_seeded_b200 import binding, synth
+        self.torch, self.binding, self.synth = torch, binding, synth
+        self.wl, self.dev = wl, device
+        self.steps, self.warmup = steps, warmup
+        gen0 = synth.Generator(wl, layer=0)
+        self.seeds = gen0.method_seeds()
+        self.ctx = binding.Context(wl.key_bits, wl.value_bits, self.seeds, device=device.index)
+        self.n_layers = wl.n_layers
+        self.T0 = wl.context
+        self.total_steps = warmup + steps
+        self.max_len = self.T0 + self.total_steps
+        self.pages = (self.max_len + 15) // 16
+        n_kv, nq, B = wl.n_kv_heads, wl.n_q_heads, wl.batch
+        assert B == 1
+        self.page_bytes = self.ctx.page_bytes(n_kv)
+        self.caches, self.btabs, self.slots = [], [], []
+        g = torch.Generator(device=device)
+        for layer in range(self.n_layers):
+            gen = synth.Generator(wl, layer=layer)
+            bt, n_pages = gen.page_pool(np.array([self.pages]))
+            cache = torch.empty(n_pages * self.page_bytes, dtype=torch.uint8, device=device)
+            btt = torch.from_numpy(bt).to(device)
+            g.manual_seed(wl.seed * 1000 + layer + 7919 * rank)
+            for which, name in (("k", "k"), ("v", "v")):
+                sc = torch.from_numpy(gen.scales[which]).float().to(device)
+                x = (torch.randn((self.T0 + self.total_steps, n_kv, 128), generator=g, device=device) * sc)
+                x = x.to(torch.bfloat16)
+                setattr(self, "_" + name, x)
+            self.ctx.quantize_prefill(self._k[:self.T0], self._v[:self.T0], btt[0], 0, cache, n_pages)
+            sl = synth.slots_for(bt[0], self.T0, self.total_steps)
+            self.slots.append(torch.from_numpy(sl).to(device))
+            if layer == 0:
+                self.newk = torch.empty((self.n_layers, self.total_steps, n_kv, 128), dtype=torch.bfloat16,
+                                        device=device)
+                self.newv = torch.empty_like(self.newk)
+            self.newk[layer] = self._k[self.T0:]
+            self.newv[layer] = self._v[self.T0:]
+            del self._k, self._v
+            self.caches.append((cache, n_pages))
+            self.btabs.append(btt)
+        torch.cuda.synchronize(device)
+        self.q = (torch.randn((self.total_steps, self.n_layers, B, nq, 128), generator=g, device=device)
+                  .to(torch.bfloat16))
+        self.lens = torch.arange(self.T0 + 1, self.T0 + self.total_steps + 1, dtype=torch.int32,
+                                 device=device).reshape(-1, 1)
+        self.out = torch.zeros((self.n_layers, B, nq, 128), dtype=torch.float32, device=device)
+        self.ws_bytes = self.ctx.decode_workspace_bytes(B, nq, n_kv, self.max_len)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        # host-side buffers for the end-to-end arm
+        self.h_newk = torch.empty((self.total_steps, self.n_layers, n_kv, 128), dtype=torch.bfloat16,
+                                  pin_memory=True)
+        self.h_newv = torch.empty_like(self.h_newk, pin_memory=True)
+        self.h_q = torch.empty((self.total_steps, self.n_layers, B, nq, 128), dtype=torch.bfloat16,
+                               pin_memory=True)
+        self.h_newk.copy_(self.newk.transpose(0, 1).cpu())
+        self.h_newv.copy_(self.newv.transpose(0, 1).cpu())
+        self.h_q.copy_(self.q.cpu())
+        self.h_out = torch.empty((self.total_steps, self.n_layers, B, nq, 128), dtype=torch.float32,
+                                 pin_memory=True)
+        self.d_stepk = torch.empty((self.n_layers, n_kv, 128), dtype=torch.bfloat16, device=device)
+        self.d_stepv = torch.empty_like(self.d_stepk)
+        self.d_stepq = torch.empty((self.n_layers, B, nq, 128), dtype=torch.bfloat16, device=device)
+
+    # one decode step (all layers) with inputs already on the device
+    def step(self, s):
+        wl = self.wl
+        for layer in range(self.n_layers):
+            cache, n_pages = self.caches[layer]
+            self.ctx.quantize_append(self.newk[layer, s:s + 1], self.newv[layer, s:s + 1],
+                                     self.slots[layer][s:s + 1], cache, n_pages)
+            self.ctx.decode_attention(self.q[s, layer], cache, n_pages, self.btabs[layer], self.lens[s],
+                                      wl.n_kv_heads, self.max_len, self.out[layer], self.ws)
+
+    # the same step through host buffers
+    def step_e2e(self, s):
+        wl = self.wl
+        self.d_stepk.copy_(self.h_newk[s], non_blocking=True)
+        self.d_stepv.copy_(self.h_newv[s], non_blocking=True)
+        self.d_stepq.copy_(self.h_q[s], non_blocking=True)
+        for layer in range(self.n_layers):
+            cache, n_pages = self.caches[layer]
+            self.ctx.quantize_append(self.d_stepk[layer:layer + 1], self.d_stepv[layer:layer + 1],
+                                     self.slots[layer][s:s + 1], cache, n_pages)
+            self.ctx.decode_attention(self.d_stepq[layer], cache, n_pages, self.btabs[layer], self.lens[s],
+                                      wl.n_kv_heads, self.max_len, self.out[layer], self.ws)
+        self.h_out[s].copy_(self.out, non_blocking=True)
+
+    def e2e_bytes(self):
+        e = 2
+        wl = self.wl
+        h2d = self.n_layers * (2 * wl.n_kv_heads * 128 * e + wl.batch * wl.n_q_heads * 128 * e)
+        d2h = self.n_layers * wl.batch * wl.n_q_heads * 128 * 4
+        return h2d, d2h
+
+    def capture(self, fn, steps):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=self.dev)
+        s.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for i in steps:
+                    fn(i)
+        torch.cuda.current_stream(self.dev).wait_stream(s)
+        return g
+
+    def decode_only_graph(self, reps):
+        """reps x (32 layers of tq_decode_attention) at the final context length."""
+        wl = self.wl
+        last = self.total_steps - 1
+
+        def body(_):
+            for layer in range(self.n_layers):
+                cache, n_pages = self.caches[layer]
+                self.ctx.decode_attention(self.q[last, layer], cache, n_pages, self.btabs[layer], self.lens[last],
+                                          wl.n_kv_heads, self.max_len, self.out[layer], self.ws)
+        return self.capture(body, range(reps))
+
+
+def timed(torch, dev, fn):
+    st = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(st)
+    fn()
+    b.record(st)
+    b.synchronize()
+    return a.elapsed_time(b) / 1e3
+
+
+# -------------------------------------------------------------- CPU baseline
+def oracle_sample(wl, budget_s=12.0, gpu_cache=None):
+    """Time the float64 oracle on a bounded sample of one decode step.
+
+    Sample: for one layer, quantize one new token for every KV head and decode
+    the query heads of one KV head over the full context, from packed cache
+    bytes; repeated for successive KV heads until the budget is used. The per
+    step time is extrapolated to all KV heads and layers.
+    """
+    import threadpoolctl
+    from oracle import decode as odec, layout as lay, quantize as oq, codebook as ocb, rng as orng
+    from decode_attention_seeded_b200 import synth
+    gen = synth.Generator(wl, layer=0)
+    seeds = gen.method_seeds()
+    kb, vb = ocb.codebook(wl.key_bits), ocb.codebook(wl.value_bits)
+    tab = dict(signs_k=orng.sign_vector(seeds[0], 128), signs_v=orng.sign_vector(seeds[1], 128),
+               sketch=orng.gaussian_sketch(seeds[2], 128, 128), centroids_k=kb.centroids,
+               centroids_v=vb.centroids, bk=wl.key_bits, bv=wl.value_bits)
+    T = wl.context
+    g = wl.group
+    rng = np.random.default_rng(0)
+    if gpu_cache is None:
+        # packed bytes of a synthetic cache (random bits: the oracle's cost does not depend on them)
+        npg = (T + 15) // 16
+        blocks = rng.integers(0, 256, size=(npg, lay.block_bytes(wl.key_bits, wl.value_bits)), dtype=np.uint8)
+        no = lay.section_offsets(wl.key_bits, wl.value_bits)["norm"]
+        blocks[:, no:no + 96] = np.frombuffer(
+            np.abs(rng.standard_normal((npg, 48))).astype(np.float16).tobytes(), dtype=np.uint8).reshape(npg, 96)
+    else:
+        blocks = gpu_cache
+    bt = np.arange(blocks.shape[0])
+    heads_done = 0
+    t0 = time.perf_counter()
+    with threadpoolctl.threadpool_limits(1):
+        while True:
+            x = rng.standard_normal((1, 128))
+            oq.quantize(x, tab["signs_k"], kb.centroids, kb.thresholds, tab["sketch"])
+            oq.quantize(x, tab["signs_v"], vb.centroids, vb.thresholds)
+            kc, sb, vc, nk, gm, nv = odec.gather_sequence(blocks[:, None, :], bt, T, 0, wl.key_bits, wl.value_bits)
+            for hh in range(g):
+                qt, p = odec.transform_query(rng.standard_normal(128), tab["signs_k"], tab["sketch"])
+                lg = odec.logits(qt, p, kc, nk, gm, sb, kb.centroids, 1 / np.sqrt(128), 128)
+                odec.attend(lg, vc, nv, vb.centroids, tab["signs_v"])
+            heads_done += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s or heads_done >= wl.n_kv_heads * wl.n_layers:
+                break
+    per_head = el / heads_done
+    per_step = per_head * wl.n_kv_heads * wl.n_layers
+    return {"value": wl.batch / per_step, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{heads_done} (layer, KV head) decode groups of {g} query heads over {T} tokens "
+                      f"plus one token quantize each, float64 NumPy, 1 thread; extrapolated x"
+                      f"{wl.n_kv_heads * wl.n_layers} to a full step", "seconds": round(el, 2)}
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from decode_attention_seeded_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.layers:
+        import dataclasses
+        wl = dataclasses.replace(wl, n_layers=args.layers)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cpu = oracle_sample(wl, budget_s=min(args.oracle_budget, 20.0))
+        v = cpu["value"]
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.n_q_heads,
+                           "kv_heads": wl.n_kv_heads, "context": wl.context, "layers": wl.n_layers,
+                           "key_bits": wl.key_bits, "value_bits": wl.value_bits},
+                "cpu_baseline": {k: cpu[k] for k in ("kind", "cores", "sample")} | {"value": v, "unit": "tokens/s"},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    bench = DecodeBench(wl, args.steps, args.warmup, dev, rank)
+    W, K = args.warmup, args.steps
+    g_warm = bench.capture(bench.step, range(W))
+    g_main = bench.capture(bench.step, range(W, W + K))
+    g_warm.replay()
+    torch.cuda.synchronize(dev)
+    assert bench.ctx.device_error() == 0
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    barrier()
+    with ClockSampler(local) as clk:
+        t_main = timed(torch, dev, g_main.replay)
+    barrier()
+    t_main = max_over_ranks(t_main)
+    clocks = clk.summary()
+
+    # end-to-end arm: same K steps from host buffers (state rewinds: same slots rewritten)
+    g_e2e = bench.capture(bench.step_e2e, range(W, W + K))
+    g_e2e_w = bench.capture(bench.step_e2e, range(W))
+    g_e2e_w.replay()
+    barrier()
+    t_e2e = max_over_ranks(timed(torch, dev, g_e2e.replay))
+    barrier()
+
+    # roofline: decode attention alone, back-to-back over the 32 layer caches
+    reps = 4
+    g_dec = bench.decode_only_graph(reps)
+    g_dec.replay()
+    barrier()
+    t_dec = max_over_ranks(timed(torch, dev, g_dec.replay))
+    n_dec = reps * bench.n_layers
+    dec_s = t_dec / n_dec
+    assert bench.ctx.device_error() == 0
+
+    peak, peak_kind = load_peaks()
+    bpt = bench.ctx.block_bytes // 16                     # bytes per token-head (102 for 3/2 bits)
+    ctx_len = bench.max_len
+    alg_bytes = bpt * ctx_len * wl.n_kv_heads * wl.batch
+    achieved = alg_bytes / dec_s / 1e9
+    traffic = recorded_traffic("bytes_per_launch")
+
+    tokens = K * wl.batch * world
+    value = tokens / t_main
+    h2d, d2h = bench.e2e_bytes()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": t_main / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8/fp16 tensor-core, fp32 accumulate (3-bit keys + QJL, 2-bit values)",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
+                   "head_dim": 128, "context": wl.context, "layers": wl.n_layers, "key_bits": wl.key_bits,
+                   "value_bits": wl.value_bits, "qjl_rows": 128, "page_tokens": 16,
+                   "l2": f"inputs larger than L2: {bench.n_layers} layer caches, "
+                         f"{bench.n_layers * bench.caches[0][1] * bench.page_bytes / 1e9:.2f} GB per step",
+                   "parallelism": f"replica x{world} (one sequence per GPU)"},
+        "e2e": {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                     "kernel": "tq_decode_attention (qtransform + split-K decode)",
+                     "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
+        "gpu_launches": K * bench.n_layers * 3,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(wl, budget_s=args.oracle_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,55 @@
+// Internal interface between the host library (tq_host.cpp) and the CUDA
+// kernels (tq_kernels.cu). Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace tq {
+
+constexpr int kHeadDim = 128;
+constexpr int kQjlRows = 128;
+constexpr int kPage = 16;
+
+// Everything a kernel needs to know about the codebooks and seeded tables.
+// Passed by value as a kernel parameter (lives in the constant bank).
+struct Tables {
+  int key_bits = 0, value_bits = 0;
+  int block_bytes = 0;          // bytes of one (page, KV head) block
+  int k_exp = 0;                // key centroids * 2^k_exp are exact int16 values
+  float thr_k[16];              // 2^b - 1 thresholds (rest unused)
+  float thr_v[16];
+  float cen_k[16];              // fp16 centroids widened to fp32
+  float cen_v[16];
+  uint32_t kq_hi[4];            // key centroid int16 split hi*256 + lo, hi bytes (16 entries)
+  uint32_t kq_lo[4];            //   ... lo bytes (signed, in [-128, 127])
+  uint32_t v_lo[4];             // value centroid fp16 low bytes (16 entries)
+  uint32_t v_hi[4];             //   ... high bytes
+  const float* signs_k = nullptr;     // device [128], +-1
+  const float* signs_v = nullptr;     // device [128], +-1
+  const uint16_t* sketch_t = nullptr; // device fp16 bits of S^T, [128 (d)][128 (m)]
+  unsigned* err = nullptr;            // device error word
+};
+
+// Workspace carve-up for one decode call; all offsets in bytes, 256-aligned.
+struct DecodePlan {
+  int batch, n_q, n_kv, group, n_hg;  // n_hg = ceil(group / 8) head groups of 8
+  int max_pages, pages_per_chunk, chunks;
+  size_t off_qfrag, off_qconst, off_partial, off_counter, total;
+};
+
+DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int block_bytes);
+
+cudaError_t launch_quantize_append(const Tables& t, const void* k, const void* v, int dtype,
+                                   int n_tokens, int n_kv, const int64_t* slots, void* cache,
+                                   int64_t n_pages, cudaStream_t s);
+cudaError_t launch_quantize_prefill(const Tables& t, const void* k, const void* v, int dtype,
+                                    int n_tokens, int n_kv, const int32_t* block_table,
+                                    int start_pos, void* cache, int64_t n_pages, cudaStream_t s);
+cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype,
+                          const void* cache, int64_t n_pages, const int32_t* block_tables,
+                          int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len,
+                          float scale, float* out, void* workspace, cudaStream_t s);
+
+}  // namespace tq

@@ -1,0 +1,172 @@
+/*
+ * tq.h -- C ABI of the B200 (sm_100a) compressed-KV cache library (libtq.so).
+ *
+ * TurboQuant-style KV-cache compression and decode attention, as described on
+ * the pages "TurboQuant : 6x moins de cache, jusqu'a 8x plus rapide"
+ * (leviatan.io: "Principe de quantification sans calibration", "Benchmarks de
+ * memoire") and the wis-web.com llama.cpp-fork post (paragraphs on PolarQuant
+ * and on QJL): each K/V vector is rotated by a seeded random Walsh-Hadamard
+ * transform, its L2 norm is kept, every rotated coordinate is coded with a fixed
+ * b-bit Lloyd-Max codebook of the known post-rotation law (no per-block scales),
+ * and keys add one QJL sign bit per row of a seeded Gaussian sketch plus the
+ * residual norm. Decode attention reads the packed cache directly.
+ *
+ * Conventions for every call:
+ *   - Pointers marked (device) are CUDA device pointers; (host) are host memory.
+ *     The caller owns every buffer it passes; the library owns only the context
+ *     and the small device tables it allocates in tq_create / tq_init_*.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream). Nothing throws across the ABI.
+ *   - Arguments the host can check are checked before any launch; a bad one
+ *     returns TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED and enqueues nothing.
+ *   - Faults detected on the device (a page id or slot out of range, a wait
+ *     that ran out) are not traps: the kernel skips the access, records a code
+ *     in the context's device error word and finishes. tq_get_device_error
+ *     reads (and clears) it.
+ *   - Fixed geometry in this version: head_dim d = 128, QJL rows m = 128,
+ *     16 tokens per page, key/value code widths 2, 3 or 4 bits.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,      /* null pointer, bad size, inconsistent shapes      */
+  TQ_ERR_UNSUPPORTED = 2,      /* geometry or bit width this build does not serve  */
+  TQ_ERR_WORKSPACE = 3,        /* workspace too small or misaligned                 */
+  TQ_ERR_CUDA = 4,             /* a CUDA runtime call failed                         */
+  TQ_ERR_DEVICE = 5,           /* device error word was set (see TQ_DEV_* bits)      */
+  TQ_ERR_NOT_INITIALIZED = 6   /* tq_init_rotation / tq_init_codebooks not called    */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* Bits of the device error word. */
+#define TQ_DEV_BAD_SLOT     0x1u   /* quantize: slot id outside the page pool           */
+#define TQ_DEV_BAD_PAGE     0x2u   /* decode: block-table entry outside the page pool    */
+#define TQ_DEV_TIMEOUT      0x4u   /* a bounded wait on a TMA transfer ran out          */
+#define TQ_DEV_BAD_LENGTH   0x8u   /* decode: seq_len above max_seq_len or negative     */
+
+typedef struct tq_ctx tq_ctx;   /* opaque; owned by the library */
+typedef void* tq_stream;        /* cudaStream_t */
+
+/* Library version (major*10000 + minor*100 + patch) and status text. */
+int tq_version(void);
+const char* tq_status_string(tq_status s);
+
+/*
+ * Create a context on CUDA device `device`. head_dim, qjl_rows and page_size
+ * must be 128, 128 and 16. Allocates a few tens of KB of device tables and the
+ * device error word. *out receives the context (NULL on error).
+ */
+tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int device);
+void tq_destroy(tq_ctx* ctx);
+
+/*
+ * Seeded rotation and sketch (pages: PolarQuant paragraph -- random
+ * Walsh-Hadamard rotation; QJL paragraph -- random projection signs).
+ * D_K, D_V in {+1,-1}^d: entry i is -1 iff the top bit of SplitMix64 output i
+ * of seed_k / seed_v is set. S (m x d): entry r*d+c is the cosine branch of
+ * Box-Muller on SplitMix64 outputs 2(r*d+c), 2(r*d+c)+1 of seed_s, rounded to
+ * fp16. Computed on the host, copied to the device on `stream`.
+ */
+tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64_t seed_s,
+                           tq_stream stream);
+
+/*
+ * Lloyd-Max codebooks (pages: the coordinate law after the rotation is known in
+ * advance, so no quantisation constants are stored; turbo2/3/4 = 2/3/4 bits).
+ * Law: one coordinate of a uniform point on the unit sphere, density
+ * proportional to (1-t^2)^((d-3)/2). Centroids are rounded to fp16; thresholds
+ * are midpoints of adjacent stored centroids. key_bits, value_bits in {2,3,4}.
+ */
+tq_status tq_init_codebooks(tq_ctx* ctx, int key_bits, int value_bits, tq_stream stream);
+
+/* Bytes of one (page, KV head) block and of one physical page (all KV heads):
+ * block = 16 * (16*key_bits + 16 + 4 + 16*value_bits + 2). 0 if not initialised. */
+size_t tq_block_bytes(const tq_ctx* ctx);
+size_t tq_page_bytes(const tq_ctx* ctx, int n_kv_heads);
+
+/*
+ * Quantize and append tokens into the paged cache.
+ *   k, v          (device) [n_tokens, n_kv_heads, 128] contiguous, dtype fp32 / bf16 / fp16.
+ *   slot_mapping  (device) int64 [n_tokens]: physical_page * 16 + offset of each token.
+ *                 Slots must be distinct within one call; any order is allowed.
+ *   cache         (device) n_cache_pages physical pages of tq_page_bytes() bytes each,
+ *                 page-major then KV-head-major; 16-byte aligned.
+ * For each (token, head): n = |x|, y = R x / n, codes = cell(y); keys also
+ * u = y - c[code], gamma = n |u|, sign bits [S u >= 0]; stored per the block layout.
+ * Slot ids outside [0, 16*n_cache_pages) set TQ_DEV_BAD_SLOT and are skipped.
+ */
+tq_status tq_quantize_append(tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
+                             int n_tokens, int n_kv_heads, const int64_t* slot_mapping,
+                             void* cache, int64_t n_cache_pages, tq_stream stream);
+
+/*
+ * Quantize a contiguous run of one sequence's tokens (a prefill or a chunk of
+ * one): logical positions [start_pos, start_pos + n_tokens) go to the pages
+ * named by block_table (device int32 [>= ceil((start_pos+n_tokens)/16)]).
+ * Same arithmetic as tq_quantize_append; whole pages are written with full-width
+ * stores, partial pages are merged with what they already hold.
+ */
+tq_status tq_quantize_prefill(tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
+                              int n_tokens, int n_kv_heads, const int32_t* block_table,
+                              int start_pos, void* cache, int64_t n_cache_pages, tq_stream stream);
+
+/*
+ * Workspace for tq_decode_attention (caller-allocated device memory, 256-byte
+ * aligned). It holds the transformed queries, split-K partials and one counter
+ * per (sequence, KV head); its contents need no initialisation.
+ */
+size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int n_q_heads, int n_kv_heads,
+                                 int max_seq_len);
+
+/*
+ * Decode attention over the compressed paged GQA cache.
+ *   q             (device) [batch, n_q_heads, 128], dtype fp32 / bf16 / fp16.
+ *   cache         (device) as written by tq_quantize_*.
+ *   block_tables  (device) int32 [batch, max_pages_per_seq]: physical page of each logical page.
+ *   seq_lens      (device) int32 [batch]: cached tokens per sequence, 0 <= len <= max_seq_len.
+ *   max_seq_len   host-side upper bound of seq_lens (sizes the split-K grid).
+ *   scale         softmax scale; 0 selects 1/sqrt(128).
+ *   out           (device) float32 [batch, n_q_heads, 128].
+ * Query head h reads KV head h / (n_q_heads / n_kv_heads). Per token t:
+ *   l_t = scale * ( |k_t| <R_K q, c[code_t]> + |r_t| sqrt(pi/2)/m <S R_K q, sign(S r_t)> ),
+ * softmax over t, a = sum_t w_t |v_t| c_v[code_v,t], out = R_V^T a. A sequence of
+ * length 0 yields zeros. Block-table entries outside the pool set TQ_DEV_BAD_PAGE
+ * (that page is skipped).
+ */
+tq_status tq_decode_attention(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
+                              int64_t n_cache_pages, const int32_t* block_tables,
+                              int max_pages_per_seq, const int32_t* seq_lens, int batch,
+                              int n_q_heads, int n_kv_heads, int max_seq_len, float scale,
+                              float* out, void* workspace, size_t workspace_bytes,
+                              tq_stream stream);
+
+/* Synchronise `stream`, then read and clear the device error word (TQ_DEV_* bits). */
+tq_status tq_get_device_error(tq_ctx* ctx, uint32_t* code, tq_stream stream);
+
+/* ---- Host-only table generators (no device needed; what tq_init_* upload) ---- */
+
+/* D in {+1,-1}^d for `seed` (see tq_init_rotation). out: (host) int8 [d]. */
+tq_status tq_host_sign_vector(uint64_t seed, int d, int8_t* out);
+
+/* S (m x d) for `seed` as fp16 bit patterns, row-major. out: (host) uint16 [m*d]. */
+tq_status tq_host_gaussian_sketch(uint64_t seed, int m, int d, uint16_t* out);
+
+/* b-bit codebook for head_dim d: centroids (host, fp16 bits [2^b], ascending) and
+ * thresholds (host, float [2^b - 1]). */
+tq_status tq_host_codebook(int bits, int d, uint16_t* centroids, float* thresholds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */
