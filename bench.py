@@ -3,8 +3,9 @@
 Workload (default ``llama8b``): Llama-3.1-8B-shaped decode, batch 1, 32 query /
 8 KV heads, head_dim 128, 32768 cached tokens per layer in 16-token pages, keys
 3-bit + QJL (m = 128), values 2-bit, 32 layers. One step = one generated token:
-for each of the 32 layers, quantize-append the new token's K/V (8 heads) and
-run decode attention for the 32 query heads over the whole cache. The 32 layer
+for each of the 32 layers, one tq_decode_step call quantizes and appends the new
+token's K/V (8 heads) and runs decode attention for the 32 query heads over the
+whole cache (two kernel launches: step preparation, then split-K attention). The 32 layer
 caches (about 0.86 GB) exceed the 126 MB L2, so every step streams from HBM.
 
 ``value``   decode tokens/s with inputs resident in HBM (CUDA-graph replay of
@@ -199,10 +200,9 @@ class DecodeBench:
         wl = self.wl
         for layer in range(self.n_layers):
             cache, n_pages = self.caches[layer]
-            self.ctx.quantize_append(self.newk[layer, s:s + 1], self.newv[layer, s:s + 1],
-                                     self.slots[layer][s:s + 1], cache, n_pages)
-            self.ctx.decode_attention(self.q[s, layer], cache, n_pages, self.btabs[layer], self.lens[s],
-                                      wl.n_kv_heads, self.max_len, self.out[layer], self.ws)
+            self.ctx.decode_step(self.newk[layer, s:s + 1], self.newv[layer, s:s + 1], self.q[s, layer], cache,
+                                 n_pages, self.btabs[layer], self.lens[s], wl.n_kv_heads, self.max_len,
+                                 self.out[layer], self.ws)
 
     # the same step through host buffers
     def step_e2e(self, s):
@@ -212,10 +212,9 @@ class DecodeBench:
         self.d_stepq.copy_(self.h_q[s], non_blocking=True)
         for layer in range(self.n_layers):
             cache, n_pages = self.caches[layer]
-            self.ctx.quantize_append(self.d_stepk[layer:layer + 1], self.d_stepv[layer:layer + 1],
-                                     self.slots[layer][s:s + 1], cache, n_pages)
-            self.ctx.decode_attention(self.d_stepq[layer], cache, n_pages, self.btabs[layer], self.lens[s],
-                                      wl.n_kv_heads, self.max_len, self.out[layer], self.ws)
+            self.ctx.decode_step(self.d_stepk[layer:layer + 1], self.d_stepv[layer:layer + 1], self.d_stepq[layer],
+                                 cache, n_pages, self.btabs[layer], self.lens[s], wl.n_kv_heads, self.max_len,
+                                 self.out[layer], self.ws)
         self.h_out[s].copy_(self.out, non_blocking=True)
 
     def e2e_bytes(self):
@@ -437,7 +436,7 @@ def main():
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                      "kernel": "tq_decode_attention (qtransform + split-K decode)",
                      "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
-        "gpu_launches": K * bench.n_layers * 3,
+        "gpu_launches": K * bench.n_layers * 2,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

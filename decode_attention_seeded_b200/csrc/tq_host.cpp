@@ -198,7 +198,7 @@ struct tq_ctx {
   int device = 0;
   bool rot_ready = false, cb_ready = false;
   float* d_signs = nullptr;        // [2][128]: D_K then D_V
-  uint16_t* d_sketch_t = nullptr;  // [128][128] fp16 bits of S^T
+  uint16_t* d_sketch_t = nullptr;  // [128][128] fp16 bits of S^T, then S (row-major)
   unsigned* d_err = nullptr;
   tq::Tables tables;
 };
@@ -286,22 +286,22 @@ DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int block_by
   p.n_hg = (p.group + 3) / 4;                    // groups of 4 query heads
   p.max_pages = std::max(1, (max_seq_len + kPage - 1) / kPage);
   const int pairs = batch * n_kv;
-  const int target_ctas = 148 * 3;
+  const int target_ctas = 148 * 2;               // two resident CTAs of 8 warps per SM
   int chunks = std::max(1, (target_ctas + pairs - 1) / pairs);
   int ppc = (p.max_pages + chunks - 1) / chunks;
-  ppc = std::max(ppc, 8);                         // keep each CTA's four warps busy
+  ppc = std::max(ppc, 16);                        // at least two pages per warp
   p.pages_per_chunk = ppc;
   p.chunks = (p.max_pages + ppc - 1) / ppc;
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   size_t off = 0;
   p.off_qfrag = off;
-  off = al(off + static_cast<size_t>(pairs) * p.n_hg * 2 * 2048);
+  off = al(off + static_cast<size_t>(pairs) * p.n_hg * 1024 * sizeof(uint32_t));
   p.off_qconst = off;
   off = al(off + static_cast<size_t>(pairs) * p.n_hg * 4 * 4 * sizeof(float));
   p.off_partial = off;
   off = al(off + static_cast<size_t>(pairs) * p.chunks * p.n_hg * 4 * 132 * sizeof(float));
   p.off_counter = off;
-  off = al(off + static_cast<size_t>(pairs) * sizeof(unsigned));
+  off = al(off + static_cast<size_t>(pairs) * sizeof(unsigned long long));
   p.total = off;
   return p;
 }
@@ -365,7 +365,7 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   tq_ctx* c = new tq_ctx;
   c->device = device;
   cudaError_t e = cudaMalloc(&c->d_signs, 2 * tq::kHeadDim * sizeof(float));
-  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
+  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 2 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
   if (e == cudaSuccess) e = cudaMalloc(&c->d_err, sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(unsigned));
   if (e != cudaSuccess) {
@@ -375,6 +375,7 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   c->tables.signs_k = c->d_signs;
   c->tables.signs_v = c->d_signs + tq::kHeadDim;
   c->tables.sketch_t = c->d_sketch_t;
+  c->tables.sketch = c->d_sketch_t + tq::kQjlRows * tq::kHeadDim;
   c->tables.err = c->d_err;
   *out = c;
   return TQ_OK;
@@ -397,7 +398,7 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
   if (tq_status st = check_device(ctx)) return st;
   const int d = tq::kHeadDim, m = tq::kQjlRows;
   std::vector<int8_t> sk(d), sv(d);
-  std::vector<uint16_t> s(m * d), st(m * d);
+  std::vector<uint16_t> s(m * d), st(2 * m * d);
   tq_host_sign_vector(seed_k, d, sk.data());
   tq_host_sign_vector(seed_v, d, sv.data());
   tq_host_gaussian_sketch(seed_s, m, d, s.data());
@@ -407,7 +408,10 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
     signs[d + i] = sv[i];
   }
   for (int r = 0; r < m; ++r)
-    for (int c = 0; c < d; ++c) st[c * m + r] = s[r * d + c];
+    for (int c = 0; c < d; ++c) {
+      st[c * m + r] = s[r * d + c];            // S^T
+      st[m * d + r * d + c] = s[r * d + c];    // S
+    }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // Synchronous copies from pageable memory: this is the cold set-up path.
   cudaError_t e = cudaMemcpyAsync(ctx->d_signs, signs.data(), 2 * d * sizeof(float),
@@ -491,12 +495,11 @@ size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int n_q_heads, in
   return tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len, 0).total;
 }
 
-tq_status tq_decode_attention(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
-                              int64_t n_cache_pages, const int32_t* block_tables,
-                              int max_pages_per_seq, const int32_t* seq_lens, int batch,
-                              int n_q_heads, int n_kv_heads, int max_seq_len, float scale,
-                              float* out, void* workspace, size_t workspace_bytes,
-                              tq_stream stream) {
+static tq_status check_decode_args(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
+                                   int64_t n_cache_pages, const int32_t* block_tables, int max_pages_per_seq,
+                                   const int32_t* seq_lens, int batch, int n_q_heads, int n_kv_heads,
+                                   int max_seq_len, float scale, const float* out, const void* workspace,
+                                   size_t workspace_bytes, tq::DecodePlan* plan) {
   if (!ctx) return TQ_ERR_INVALID_ARG;
   if (!ctx->rot_ready || !ctx->cb_ready) return TQ_ERR_NOT_INITIALIZED;
   if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads ||
@@ -510,15 +513,47 @@ tq_status tq_decode_attention(tq_ctx* ctx, const void* q, tq_dtype q_dtype, cons
   const size_t es = q_dtype == TQ_F32 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(q) % (4 * es)) return TQ_ERR_INVALID_ARG;
   if (!(scale >= 0.0f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
-  tq::DecodePlan plan = tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len,
-                                      ctx->tables.block_bytes);
-  if (workspace_bytes < plan.total || reinterpret_cast<uintptr_t>(workspace) % 256)
-    return TQ_ERR_WORKSPACE;
-  if (tq_status st = check_device(ctx)) return st;
+  *plan = tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len, ctx->tables.block_bytes);
+  if (workspace_bytes < plan->total || reinterpret_cast<uintptr_t>(workspace) % 256) return TQ_ERR_WORKSPACE;
+  return check_device(ctx);
+}
+
+tq_status tq_decode_attention(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
+                              int64_t n_cache_pages, const int32_t* block_tables,
+                              int max_pages_per_seq, const int32_t* seq_lens, int batch,
+                              int n_q_heads, int n_kv_heads, int max_seq_len, float scale,
+                              float* out, void* workspace, size_t workspace_bytes,
+                              tq_stream stream) {
+  tq::DecodePlan plan;
+  if (tq_status st = check_decode_args(ctx, q, q_dtype, cache, n_cache_pages, block_tables, max_pages_per_seq,
+                                       seq_lens, batch, n_q_heads, n_kv_heads, max_seq_len, scale, out,
+                                       workspace, workspace_bytes, &plan))
+    return st;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
   return from_cuda(tq::launch_decode(ctx->tables, plan, q, q_dtype, cache, n_cache_pages,
                                      block_tables, max_pages_per_seq, seq_lens, max_seq_len,
                                      scale, out, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+                         const void* q, tq_dtype q_dtype, void* cache, int64_t n_cache_pages,
+                         const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
+                         int batch, int n_q_heads, int n_kv_heads, int max_seq_len, float scale, float* out,
+                         void* workspace, size_t workspace_bytes, tq_stream stream) {
+  tq::DecodePlan plan;
+  if (tq_status st = check_decode_args(ctx, q, q_dtype, cache, n_cache_pages, block_tables, max_pages_per_seq,
+                                       seq_lens, batch, n_q_heads, n_kv_heads, max_seq_len, scale, out,
+                                       workspace, workspace_bytes, &plan))
+    return st;
+  if (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16 && kv_dtype != TQ_F16) return TQ_ERR_UNSUPPORTED;
+  if (!k_new || !v_new) return TQ_ERR_INVALID_ARG;
+  const size_t es = kv_dtype == TQ_F32 ? 4 : 2;
+  if (reinterpret_cast<uintptr_t>(k_new) % (4 * es) || reinterpret_cast<uintptr_t>(v_new) % (4 * es))
+    return TQ_ERR_INVALID_ARG;
+  if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
+  return from_cuda(tq::launch_decode_step(ctx->tables, plan, k_new, v_new, kv_dtype, q, q_dtype, cache,
+                                          n_cache_pages, block_tables, max_pages_per_seq, seq_lens, max_seq_len,
+                                          scale, out, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 tq_status tq_get_device_error(tq_ctx* ctx, uint32_t* code, tq_stream stream) {

@@ -29,12 +29,13 @@ struct Tables {
   const float* signs_k = nullptr;     // device [128], +-1
   const float* signs_v = nullptr;     // device [128], +-1
   const uint16_t* sketch_t = nullptr; // device fp16 bits of S^T, [128 (d)][128 (m)]
+  const uint16_t* sketch = nullptr;   // device fp16 bits of S, [128 (m)][128 (d)]
   unsigned* err = nullptr;            // device error word
 };
 
 // Workspace carve-up for one decode call; all offsets in bytes, 256-aligned.
 struct DecodePlan {
-  int batch, n_q, n_kv, group, n_hg;  // n_hg = ceil(group / 8) head groups of 8
+  int batch, n_q, n_kv, group, n_hg;  // n_hg = ceil(group / 4) groups of 4 query heads
   int max_pages, pages_per_chunk, chunks;
   size_t off_qfrag, off_qconst, off_partial, off_counter, total;
 };
@@ -51,5 +52,10 @@ cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q
                           const void* cache, int64_t n_pages, const int32_t* block_tables,
                           int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len,
                           float scale, float* out, void* workspace, cudaStream_t s);
+
+cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
+                               int kv_dtype, const void* q, int q_dtype, void* cache, int64_t n_pages,
+                               const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
+                               int max_seq_len, float scale, float* out, void* workspace, cudaStream_t s);
 
 }  // namespace tq

@@ -62,6 +62,26 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Logical right shift by a constant done on the multiplier (FMA) pipe instead
+// of the ALU pipe: the high word of x * 2^(32-k) is x >> k.
+template <int K>
+__device__ __forceinline__ uint32_t shr(uint32_t x) {
+  static_assert(K > 0 && K < 32, "shift");
+  return __umulhi(x, 1u << (32 - K));
+}
+
+// Hardware base-2 exponential / logarithm (MUFU), subnormals flushed to zero.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int m = 16; m; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
@@ -277,9 +297,10 @@ __device__ void store_value_token(uint8_t* blk, int tau, int bk, int bv, const V
   }
 }
 
+// Norm arrays keep tokens g and g + 8 in one 32-bit word: entry 2 (tau & 7) + (tau >> 3).
 __device__ __forceinline__ void store_norm(uint8_t* blk, int bk, int bv, int which, int tau, float v) {
   __half* nrm = reinterpret_cast<__half*>(blk + 256 * (bk + bv + 1));
-  nrm[16 * which + tau] = __float2half_rn(v);
+  nrm[16 * which + 2 * (tau & 7) + (tau >> 3)] = __float2half_rn(v);
 }
 
 // One warp per (token, KV head): quantize K and V and store them at the slot.
@@ -374,17 +395,17 @@ __global__ void __launch_bounds__(256) quantize_prefill_kernel(Tables T, const v
 }
 
 // ========================================================= query transform
-// Per (sequence, KV head, group of 4 query heads): q~ = H D_K q / sqrt(d) and
-// p = S q~, each quantised per head to a 24-bit integer Q = rint(x * 2^e)
-// (|Q| < 2^22) split into three int8 limbs Q = 2^16 Q2 + 2^8 Q1 + Q0. They are
-// written in the register order of the m16n8k32 A operand whose rows are
-//   rows 0-3: Q2 of heads 0-3, rows 4-7: Q0 of heads 0-3,
-//   rows 8-11: Q1 of heads 0-3, rows 12-15: zero,
-// so that every lane of quad g < 4 sees head g's top and middle limbs, and the
-// quad g + 4 (lane + 16) its bottom limb.
-//   qfrag[pair][hg][which (q, p)][kt 4][lane 32][reg 4]  (int32 words of 4 int8)
-//   qconst[pair][hg][slot 4][4] = {a, b, sum P (int), 0}: in log2 units the logit
-//   is l2 = |k| * <Q, C> * a + gamma * (2 <P, s> - sum P) * b.
+// Per (sequence, KV head, group of 4 query heads), computed in the prologue of
+// the decode kernel: q~ = H D_K q / sqrt(d) and p = S q~, each quantised per
+// head to a 24-bit integer Q = rint(x * 2^e) (|Q| < 2^22) split into three int8
+// limbs Q = 2^16 Q2 + 2^8 Q1 + Q0. They form the B operand (k = coordinate or
+// sketch row, n = column) of m16n8k32 products whose A operand is a 16-token
+// tile of codes or sign bits:
+//   n-tile 0: column 2h = Q2 of head h, column 2h + 1 = Q1 of head h,
+//   n-tile 1: column 2h = Q0 of head h, column 2h + 1 = 0,
+// so that lane (g, t) of the accumulator sees all three limbs of head t. In
+// log2 units the logit is l2 = |k| <Q, C> a + gamma (2 <P, s> - sum P) b with
+// a = scale log2(e) 2^(-e_q - k_exp), b = scale log2(e) sqrt(pi/2)/m 2^(-e_p).
 constexpr int kGroupHeads = 4;
 
 __device__ __forceinline__ int pick_exponent24(float maxabs) {
@@ -419,21 +440,20 @@ __device__ __forceinline__ int warp_isum(int v) {
   return v;
 }
 
-// grid (n_hg, n_kv, batch), 512 threads: warp w -> head slot w >> 2, sketch
-// column quarter w & 3.
-__global__ void __launch_bounds__(512) qtransform_kernel(Tables T, const void* q, int dtype, int n_q,
-                                                         int n_kv, int group, int n_hg, float scale,
-                                                         uint32_t* qfrag, float* qconst,
-                                                         unsigned* counters) {
-  asm volatile("griddepcontrol.launch_dependents;");
-  __shared__ float s_q[kGroupHeads][128];
-  __shared__ float s_p[4][kGroupHeads][128];
+// Query transform kernel: grid (n_hg, n_kv, batch), 512 threads; warp w -> head
+// slot w >> 2 of the group, sketch-column quarter w & 3. Writes
+//   qfrag[pair][hg][which (q, p)][kt 4][ntile 2][lane 32][reg 2]  (int32 words of 4 int8)
+//   qconst[pair][hg][slot 4][4] = {a, b, sum P (int bits), 0}.
+__device__ void qtransform_group(const Tables& T, const void* q, int dtype, int n_q, int n_kv, int group,
+                                 int n_hg, float scale, uint32_t* qfrag, float* qconst, unsigned* counters,
+                                 int hg, int hk, int b, float (*s_q)[128], float (*s_p)[kGroupHeads][128]) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int hs = w >> 2, cq = w & 3;
-  const int hg = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  // split-K completion counter of this (sequence, KV head): the attention kernel
+  // that follows in the same call counts its finished CTAs here
+  if (hg == 0 && threadIdx.x == 0) counters[b * n_kv + hk] = 0u;
   const int pair = b * n_kv + hk;
   const int slot = hg * kGroupHeads + hs;
-  if (hg == 0 && threadIdx.x == 0) counters[pair] = 0u;
   if (cq == 0) {
     float x[4] = {0.f, 0.f, 0.f, 0.f};
     if (slot < group) load_row4(q, static_cast<size_t>(b) * n_q + hk * group + slot, dtype, lane, x);
@@ -444,8 +464,7 @@ __global__ void __launch_bounds__(512) qtransform_kernel(Tables T, const void* q
     for (int e = 0; e < 4; ++e) s_q[hs][4 * lane + e] = x[e] * kInvSqrtD;
   }
   __syncthreads();
-  // partial p over the 32 sketch columns of this quarter: rows 4*lane .. 4*lane+3
-  {
+  {  // partial p over the 32 sketch columns of this quarter: rows 4*lane .. 4*lane+3
     const uint2* st = reinterpret_cast<const uint2*>(T.sketch_t);
     uint2 raw[32];
 #pragma unroll
@@ -478,19 +497,18 @@ __global__ void __launch_bounds__(512) qtransform_kernel(Tables T, const void* q
   const Limbs lq = split3(x, eq);
   const Limbs lp = split3(p, ep);
   const int psum = warp_isum(lp.sum);              // |sum| < 2^29
-  // lane l holds coordinates 4l..4l+3: k-tile kt = l>>3, half sub = (l>>2)&1, t = l&3
+  // lane l holds rows 4l..4l+3 of B: k-tile kt = l>>3, register sub = (l>>2)&1, t = l&3
   const int kt = lane >> 3, sub = (lane >> 2) & 1, t = lane & 3;
-  uint32_t* base = qfrag + (static_cast<size_t>(pair) * n_hg + hg) * 2 * 512;
-  const int fl_top = 4 * hs + t;           // quad hs: rows hs (Q2) and hs + 8 (Q1)
-  const int fl_bot = 4 * (hs + 4) + t;     // quad hs + 4: rows hs + 4 (Q0) and hs + 12 (zero)
+  uint32_t* base = qfrag + (static_cast<size_t>(pair) * n_hg + hg) * 1024;
+  const int ln_a = 4 * (2 * hs) + t, ln_b = 4 * (2 * hs + 1) + t;      // columns 2hs and 2hs + 1
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
-    const Limbs& L = which ? lp : lq;
-    uint32_t* f = base + (which * 4 + kt) * 128;
-    f[fl_top * 4 + 2 * sub + 0] = L.w2;
-    f[fl_top * 4 + 2 * sub + 1] = L.w1;
-    f[fl_bot * 4 + 2 * sub + 0] = L.w0;
-    f[fl_bot * 4 + 2 * sub + 1] = 0u;
+    const Limbs& Lm = which ? lp : lq;
+    uint32_t* f = base + (which * 4 + kt) * 128;      // [ntile 2][lane 32][reg 2]
+    f[0 * 64 + ln_a * 2 + sub] = Lm.w2;
+    f[0 * 64 + ln_b * 2 + sub] = Lm.w1;
+    f[1 * 64 + ln_a * 2 + sub] = Lm.w0;
+    f[1 * 64 + ln_b * 2 + sub] = 0u;
   }
   if (lane == 0) {
     float* qc = qconst + ((static_cast<size_t>(pair) * n_hg + hg) * kGroupHeads + hs) * 4;
@@ -502,9 +520,125 @@ __global__ void __launch_bounds__(512) qtransform_kernel(Tables T, const void* q
   }
 }
 
+__global__ void __launch_bounds__(512) qtransform_kernel(Tables T, const void* q, int dtype, int n_q,
+                                                         int n_kv, int group, int n_hg, float scale,
+                                                         uint32_t* qfrag, float* qconst, unsigned* counters) {
+  // the decode kernel may start now: it prefetches pages until it needs these outputs
+  asm volatile("griddepcontrol.launch_dependents;");
+  __shared__ float s_q[kGroupHeads][128];
+  __shared__ float s_p[4][kGroupHeads][128];
+  qtransform_group(T, q, dtype, n_q, n_kv, group, n_hg, scale, qfrag, qconst, counters, blockIdx.x, blockIdx.y,
+                   blockIdx.z, s_q, s_p);
+}
+
+// Decode step preparation: grid (n_hg + 1, n_kv, batch), 512 threads. CTAs with
+// x < n_hg run the query transform of group x; the CTA with x == n_hg quantizes
+// the new key and value of (sequence z, KV head y) and stores them at logical
+// position seq_lens[z] - 1 (sequences of length 0 append nothing).
+__global__ void __launch_bounds__(512) step_prep_kernel(Tables T, const void* q, int q_dtype, int n_q, int n_kv,
+                                                        int group, int n_hg, float scale, uint32_t* qfrag,
+                                                        float* qconst, unsigned* counters, const void* k_new,
+                                                        const void* v_new,
+                                                        int kv_dtype, uint8_t* cache, int64_t n_pages,
+                                                        const int32_t* block_tables, int max_pages_per_seq,
+                                                        const int32_t* seq_lens) {
+  asm volatile("griddepcontrol.launch_dependents;");
+  __shared__ float s_q[kGroupHeads][128];
+  __shared__ float s_p[4][kGroupHeads][128];
+  const int hg = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  if (hg < n_hg) {
+    qtransform_group(T, q, q_dtype, n_q, n_kv, group, n_hg, scale, qfrag, qconst, counters, hg, hk, b, s_q, s_p);
+    return;
+  }
+  const int L = seq_lens[b];
+  if (L <= 0) return;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int pos = L - 1, lpage = pos / kPage, tau = pos % kPage;
+  if (lpage >= max_pages_per_seq) {
+    if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_LENGTH);
+    return;
+  }
+  const int phys = block_tables[static_cast<int64_t>(b) * max_pages_per_seq + lpage];
+  if (phys < 0 || phys >= n_pages) {
+    if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_SLOT);
+    return;
+  }
+  uint8_t* blk = cache + (static_cast<int64_t>(phys) * n_kv + hk) * T.block_bytes;
+  float* s_u = &s_q[0][0];                          // residual of the key
+  __shared__ VecOut s_key[32];
+  const size_t row = static_cast<size_t>(b) * n_kv + hk;
+  float x[4];
+  if (w == 0) {                                     // key: rotation, codes, residual
+    load_row4(k_new, row, kv_dtype, lane, x);
+    VecOut o;
+    quantize_vector(x, T.signs_k, T.thr_k, T.cen_k, T.key_bits, nullptr, false, lane, o);
+    // residual u = y - c[code] recomputed from the codes (same arithmetic as quantize_vector)
+    float v4[4];
+    float ss = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) { ss = fmaf(x[e], x[e], ss); v4[e] = x[e] * T.signs_k[4 * lane + e]; }
+    ss = warp_sum(ss);
+    const float n = sqrtf(ss);
+    fwht128(v4, lane);
+    const float inv = n > 0.0f ? 1.0f / (n * 11.313708498984761f) : 0.0f;
+    float uu = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float u = v4[e] * inv - T.cen_k[o.code[e]];
+      s_u[4 * lane + e] = u;
+      uu = fmaf(u, u, uu);
+    }
+    uu = warp_sum(uu);
+    o.gamma = n * sqrtf(uu);
+    s_key[lane] = o;
+  } else if (w == 1) {                              // value: rotation, codes, store
+    load_row4(v_new, row, kv_dtype, lane, x);
+    VecOut o;
+    quantize_vector(x, T.signs_v, T.thr_v, T.cen_v, T.value_bits, nullptr, false, lane, o);
+    store_value_token(blk, tau, T.key_bits, T.value_bits, o, lane);
+    if (lane == 0) store_norm(blk, T.key_bits, T.value_bits, 2, tau, o.norm);
+  }
+  __syncthreads();
+  if (w < 4) {                                      // z = S u: warp w sums sketch columns 32w .. 32w+31
+    const uint2* st = reinterpret_cast<const uint2*>(T.sketch_t);
+    uint2 raw[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) raw[j] = __ldg(st + (32 * w + j) * 32 + lane);
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float uc = s_u[32 * w + j];
+      const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j].x));
+      const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j].y));
+      z[0] = fmaf(s01.x, uc, z[0]);
+      z[1] = fmaf(s01.y, uc, z[1]);
+      z[2] = fmaf(s23.x, uc, z[2]);
+      z[3] = fmaf(s23.y, uc, z[3]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s_p[w][0][4 * lane + e] = z[e];
+  }
+  __syncthreads();
+  if (w == 0) {
+    VecOut o = s_key[lane];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float z = s_p[0][0][4 * lane + e] + s_p[1][0][4 * lane + e] + s_p[2][0][4 * lane + e] +
+                      s_p[3][0][4 * lane + e];
+      o.sgn[e] = z >= 0.0f ? 1 : 0;
+    }
+    store_key_token(blk, tau, T.key_bits, o, lane);
+    if (lane == 0) {
+      store_norm(blk, T.key_bits, T.value_bits, 0, tau, o.norm);
+      store_norm(blk, T.key_bits, T.value_bits, 1, tau, o.gamma);
+    }
+  }
+}
+
 // ================================================================== decode
-constexpr int kWarps = 4;        // compute warps per CTA
+constexpr int kWarps = 8;        // compute warps per CTA
 constexpr int kStages = 6;       // TMA stages per warp
+static_assert(kWarps == 8, "the chunk merge pairs warps w and w + 4");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -527,6 +661,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
 }
 // Bounded wait: gives up after ~2^31 clock cycles (about a second).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > (1ll << 31)) return false;
@@ -549,22 +684,22 @@ __device__ __forceinline__ void key_selectors(const uint32_t* w, uint32_t (&sel)
   if constexpr (B == 2) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const uint32_t e = w[i] & 0x33333333u, o = (w[i] >> 2) & 0x33333333u;
+      const uint32_t e = w[i] & 0x33333333u, o = shr<2>(w[i]) & 0x33333333u;
       sel[4 * i + 0] = e;
-      sel[4 * i + 1] = e >> 16;
+      sel[4 * i + 1] = shr<16>(e);
       sel[4 * i + 2] = o;
-      sel[4 * i + 3] = o >> 16;
+      sel[4 * i + 3] = shr<16>(o);
     }
   } else if constexpr (B == 3) {
     const uint32_t a = w[0] & 0x77777777u, b = w[1] & 0x77777777u, c = w[2] & 0x77777777u;
-    const uint32_t sp = ((w[0] >> 3) & 0x11111111u) | ((w[1] >> 2) & 0x22222222u) | ((w[2] >> 1) & 0x44444444u);
-    sel[0] = a; sel[1] = a >> 16; sel[2] = b; sel[3] = b >> 16;
-    sel[4] = c; sel[5] = c >> 16; sel[6] = sp; sel[7] = sp >> 16;
+    const uint32_t sp = (shr<3>(w[0]) & 0x11111111u) | (shr<2>(w[1]) & 0x22222222u) | (shr<1>(w[2]) & 0x44444444u);
+    sel[0] = a; sel[1] = shr<16>(a); sel[2] = b; sel[3] = shr<16>(b);
+    sel[4] = c; sel[5] = shr<16>(c); sel[6] = sp; sel[7] = shr<16>(sp);
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       sel[2 * i] = w[i];
-      sel[2 * i + 1] = w[i] >> 16;
+      sel[2 * i + 1] = shr<16>(w[i]);
     }
   }
 }
@@ -597,27 +732,27 @@ __device__ __forceinline__ void value_selectors(const uint32_t* w, uint32_t (&se
   if constexpr (B == 2) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t e = w[i] & 0x33333333u, o = (w[i] >> 2) & 0x33333333u;
+      const uint32_t e = w[i] & 0x33333333u, o = shr<2>(w[i]) & 0x33333333u;
       sel[4 * i + 0] = e;
-      sel[4 * i + 1] = e >> 16;
+      sel[4 * i + 1] = shr<16>(e);
       sel[4 * i + 2] = o;
-      sel[4 * i + 3] = o >> 16;
+      sel[4 * i + 3] = shr<16>(o);
     }
   } else if constexpr (B == 3) {
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
       const uint32_t* x = w + 3 * g;
       const uint32_t a = x[0] & 0x77777777u, b = x[1] & 0x77777777u, c = x[2] & 0x77777777u;
-      const uint32_t sp = ((x[0] >> 3) & 0x11111111u) | ((x[1] >> 2) & 0x22222222u) | ((x[2] >> 1) & 0x44444444u);
+      const uint32_t sp = (shr<3>(x[0]) & 0x11111111u) | (shr<2>(x[1]) & 0x22222222u) | (shr<1>(x[2]) & 0x44444444u);
       uint32_t* s = sel + 8 * g;
-      s[0] = a; s[1] = a >> 16; s[2] = b; s[3] = b >> 16;
-      s[4] = c; s[5] = c >> 16; s[6] = sp; s[7] = sp >> 16;
+      s[0] = a; s[1] = shr<16>(a); s[2] = b; s[3] = shr<16>(b);
+      s[4] = c; s[5] = shr<16>(c); s[6] = sp; s[7] = shr<16>(sp);
     }
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       sel[2 * i] = w[i];
-      sel[2 * i + 1] = w[i] >> 16;
+      sel[2 * i + 1] = shr<16>(w[i]);
     }
   }
 }
@@ -646,34 +781,73 @@ struct DecodeArgs {
   int max_pages_per_seq;
   const int32_t* seq_lens;
   int max_seq_len;
-  const uint32_t* qfrag;
+  const uint32_t* qfrag;         // written by the query transform (see above)
   const float* qconst;
-  float* partial;      // [pair][chunk][hg][4 heads][132]
-  unsigned* counters;  // [pair]
-  float* out;          // [batch][n_q][128]
+  float* partial;                // [pair][chunk][hg][4 heads][132]
+  unsigned* counters;            // [pair]: finished CTAs, zeroed by the preceding kernel of the call
+  int hold_last_page;            // 1: a preceding kernel of this call appends to each sequence's last page
+  float* out;                    // [batch][n_q][128]
   int n_kv, n_q, group, n_hg, chunks, ppc;
 };
+
+// Load N 32-bit words from 8-byte-aligned shared memory with the widest accesses.
+template <int N>
+__device__ __forceinline__ void lds_words(const uint32_t* src, uint32_t (&dst)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+      dst[4 * i] = v.x; dst[4 * i + 1] = v.y; dst[4 * i + 2] = v.z; dst[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const uint2 v = reinterpret_cast<const uint2*>(src)[i];
+      dst[2 * i] = v.x; dst[2 * i + 1] = v.y;
+    }
+  }
+}
 
 // Split-K decode attention. grid (chunks, n_kv, batch), kWarps warps per CTA.
 // Each warp streams its pages (every kWarps-th page of the chunk) through a
 // private ring of kStages shared-memory stages filled by 1-D bulk TMA copies.
+//
+// Per 16-token page a warp computes, with tokens on the rows of the products:
+//   logits  int8 m16n8k32: A = key-code limbs (hi, lo) or 0/1 sign bytes of
+//           tokens g and g+8, B = query limbs -> lane (g, t) gets head t of
+//           tokens g and g + 8 with all limbs in its own registers;
+//   values  fp16 m16n8k16: A = value centroids (coordinates x tokens),
+//           B = softmax weights split into fp16 high parts (columns 0-3) and
+//           low parts (columns 4-7), transposed into place with shuffles.
 template <int BK, int BV, int NH>
 __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
   constexpr int kSignOff = 256 * BK, kVOff = 256 * (BK + 1), kNormOff = 256 * (BK + BV + 1);
+  constexpr bool kRegQ = NH <= 2;              // query fragments in registers (else shared memory)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const bool owner = g < kGroupHeads;          // quads 0-3 own heads 0-3 of each group
   const int chunk = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int pair = b * A.n_kv + hk;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kBlock);
-  uint32_t* s_qf = reinterpret_cast<uint32_t*>(bars + kWarps * kStages);   // [NH][2][4][128] query fragments
   __shared__ int s_last;
+  __shared__ int s_pageok[kWarps * kStages];
   uint8_t* stage0 = smem + warp * kStages * kBlock;
   uint64_t* mybar = bars + warp * kStages;
+  int* myok = s_pageok + warp * kStages;
 
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(mybar + s, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+
+  // Reads before griddepcontrol.wait: the launch that precedes this kernel on
+  // the stream is the query transform of the same call, which writes neither
+  // the cache nor the tables; everything before it has completed. When the call
+  // also appends tokens (hold_last_page), each sequence's last page is fetched
+  // only after the wait.
   int L = A.seq_lens[b];
   if (L < 0 || L > A.max_seq_len) {
     if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_LENGTH);
@@ -684,18 +858,24 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   const int p1 = min(p0 + A.ppc, seq_pages);
   const int nmine = (p1 > p0 + warp) ? (p1 - p0 - warp + kWarps - 1) / kWarps : 0;
   const int32_t* btab = A.block_tables + static_cast<int64_t>(b) * A.max_pages_per_seq;
+  const int held = A.hold_last_page ? seq_pages - 1 : -1;   // logical page fetched after the wait
 
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(mybar + s, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncwarp();
-
-  auto issue = [&](int kth) {
-    const int lp = p0 + warp + kth * kWarps;
-    int phys = btab[lp];
-    const int s = kth % kStages;
-    if (phys < 0 || phys >= A.n_pages) {
+  // Physical page ids of this warp's pages, 32 at a time: lane j holds page j of the window.
+  int win = 0;
+  int myphys = lane < nmine ? btab[p0 + warp + lane * kWarps] : -1;
+  auto page_id = [&](int kth) {           // all lanes (shuffle); reloads the window when needed
+    if ((kth >> 5) != win) {
+      win = kth >> 5;
+      const int j = 32 * win + lane;
+      myphys = j < nmine ? btab[p0 + warp + j * kWarps] : -1;
+    }
+    return __shfl_sync(kFull, myphys, kth & 31);
+  };
+  // lane 0 only: start the transfer of physical page `phys` into stage s
+  auto issue = [&](int phys, int s) {
+    const bool ok = phys >= 0 && phys < A.n_pages;
+    myok[s] = ok;
+    if (!ok) {
       set_error(T.err, TQ_DEV_BAD_PAGE);
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mybar + s)) : "memory");
     } else {
@@ -704,25 +884,56 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
                   mybar + s);
     }
   };
-  if (lane == 0)
-    for (int k = 0; k < min(nmine, kStages); ++k) issue(k);
+  const int n_first = min(nmine, kStages);
+  int n_early = 0;                        // stages issued before the wait, in ring order
+  while (n_early < n_first && p0 + warp + n_early * kWarps != held) ++n_early;
+  for (int k = 0; k < n_early; ++k) {
+    const int phys = __shfl_sync(kFull, myphys, k);
+    if (lane == 0) issue(phys, k);
+  }
 
-  // The query fragments come from the preceding kernel.
+  // The query fragments (and appended tokens) come from the preceding kernel.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(A.qfrag + static_cast<size_t>(pair) * A.n_hg * 1024);
-    for (int i = threadIdx.x; i < NH * 1024 / 4; i += blockDim.x) reinterpret_cast<uint4*>(s_qf)[i] = src[i];
+  for (int k = n_early; k < n_first; ++k) {
+    const int phys = __shfl_sync(kFull, myphys, k);
+    if (lane == 0) issue(phys, k);
   }
+  __syncwarp();                           // lane 0's page flags are visible to the warp
+
+  // B fragments of lane (g, t) and the constants of head t in each group of 4
+  const uint32_t* qfr = A.qfrag + static_cast<size_t>(pair) * A.n_hg * 1024;
+  auto qword = [&](int h, int which, int kt, int nt, int sub) -> uint32_t {
+    return __ldg(qfr + h * 1024 + ((which * 4 + kt) * 2 + nt) * 64 + lane * 2 + sub);
+  };
+  uint32_t bq[kRegQ ? NH : 1][4][2][2], bp[kRegQ ? NH : 1][4][2][2];
+  uint32_t* s_qf = reinterpret_cast<uint32_t*>(bars + kWarps * kStages);   // [NH][1024] when not in registers
+  if constexpr (kRegQ) {
+#pragma unroll
+    for (int h = 0; h < NH; ++h)
+#pragma unroll
+      for (int kt = 0; kt < 4; ++kt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint2 vq = __ldg(reinterpret_cast<const uint2*>(qfr + h * 1024 + ((0 * 4 + kt) * 2 + nt) * 64) + lane);
+          const uint2 vp = __ldg(reinterpret_cast<const uint2*>(qfr + h * 1024 + ((1 * 4 + kt) * 2 + nt) * 64) + lane);
+          bq[h][kt][nt][0] = vq.x; bq[h][kt][nt][1] = vq.y;
+          bp[h][kt][nt][0] = vp.x; bp[h][kt][nt][1] = vp.y;
+        }
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(qfr);
+    for (int i = threadIdx.x; i < NH * 1024 / 4; i += blockDim.x) reinterpret_cast<uint4*>(s_qf)[i] = src[i];
+    __syncthreads();
+  }
+  (void)qword;
   float ca[NH], cb[NH];
   int csum[NH];
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
-    const float4 c4 = *reinterpret_cast<const float4*>(
-        A.qconst + ((static_cast<size_t>(pair) * A.n_hg + h) * kGroupHeads + (g & 3)) * 4);
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(
+        A.qconst + ((static_cast<size_t>(pair) * A.n_hg + h) * kGroupHeads + t) * 4));
     ca[h] = c4.x; cb[h] = c4.y; csum[h] = __float_as_int(c4.z);
   }
-  __syncthreads();
   uint32_t kth_[4], ktl_[4], vlo_[4], vhi_[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -736,47 +947,41 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[h][mt][c] = 0.0f;
-  float m2[NH], lsum[NH], mp2[NH];
+  float lsum[NH], mp2[NH];
 #pragma unroll
-  for (int h = 0; h < NH; ++h) { m2[h] = kNegBig; lsum[h] = 0.0f; mp2[h] = kNegBig; }
+  for (int h = 0; h < NH; ++h) { lsum[h] = 0.0f; mp2[h] = kNegBig; }
+
+  // transpose sources for the value-product B operand (see below)
+  const int h4 = g & 3;
+  const int src0 = 4 * (2 * t) + h4, src1 = 4 * (2 * t + 1) + h4;
+  const bool hi_col = g < 4;
 
   bool alive = true;
-  for (int k = 0; k < nmine; ++k) {
-    const int s = k % kStages;
-    const unsigned parity = (k / kStages) & 1;
+  int s = 0;
+  unsigned parity = 0;
+  int lp = p0 + warp;
+  for (int k = 0; k < nmine; ++k, lp += kWarps) {
     if (!mbar_wait(mybar + s, parity)) {
       if (lane == 0) set_error(T.err, TQ_DEV_TIMEOUT);
       alive = false;
       break;
     }
-    const int lp = p0 + warp + k * kWarps;
-    const int phys = btab[lp];
-    const bool page_ok = phys >= 0 && phys < A.n_pages;
+    const bool page_ok = myok[s] != 0;
     const uint8_t* blk = stage0 + s * kBlock;
 
-    // ---- this lane's operands from the staged block
-    uint32_t kw[2][BK];
-#pragma unroll
-    for (int th = 0; th < 2; ++th)
-#pragma unroll
-      for (int i = 0; i < BK; ++i) kw[th][i] = reinterpret_cast<const uint32_t*>(blk)[lane * 2 * BK + th * BK + i];
+    // ---- this lane's operands from the staged block (tokens g and g + 8)
+    uint32_t kw[2 * BK];
+    lds_words<2 * BK>(reinterpret_cast<const uint32_t*>(blk) + lane * 2 * BK, kw);
     const uint2 sw = reinterpret_cast<const uint2*>(blk + kSignOff)[lane];
     uint32_t vw[2 * BV];
-#pragma unroll
-    for (int i = 0; i < 2 * BV; ++i) vw[i] = reinterpret_cast<const uint32_t*>(blk + kVOff)[lane * 2 * BV + i];
+    lds_words<2 * BV>(reinterpret_cast<const uint32_t*>(blk + kVOff) + lane * 2 * BV, vw);
     const uint32_t* nrm = reinterpret_cast<const uint32_t*>(blk + kNormOff);
-    float nK[4], gam[4], nV[4];
-    {
-      const uint32_t r[6] = {nrm[t], nrm[4 + t], nrm[8 + t], nrm[12 + t], nrm[16 + t], nrm[20 + t]};
-      float2 f[6];
-#pragma unroll
-      for (int i = 0; i < 6; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
-      nK[0] = f[0].x; nK[1] = f[0].y; nK[2] = f[1].x; nK[3] = f[1].y;
-      gam[0] = f[2].x; gam[1] = f[2].y; gam[2] = f[3].x; gam[3] = f[3].y;
-      nV[0] = f[4].x; nV[1] = f[4].y; nV[2] = f[5].x; nV[3] = f[5].y;
-    }
+    const uint32_t rk = nrm[g], rg = nrm[8 + g], rv = nrm[16 + g];
+    const float2 nK = __half22float2(*reinterpret_cast<const __half2*>(&rk));
+    const float2 gm = __half22float2(*reinterpret_cast<const __half2*>(&rg));
+    const float2 nV = __half22float2(*reinterpret_cast<const __half2*>(&rv));
 
-    // ---- logits: int8 tensor-core products of query limbs with code limbs
+    // ---- logits: int8 tensor-core products, tokens on the rows
     int dh[NH][2][4], dl[NH][2][4], ds[NH][2][4];
 #pragma unroll
     for (int h = 0; h < NH; ++h)
@@ -784,91 +989,95 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) dh[h][nt][c] = dl[h][nt][c] = ds[h][nt][c] = 0;
+    uint32_t sel0[8], sel1[8];
+    key_selectors<BK>(kw, sel0);
+    key_selectors<BK>(kw + BK, sel1);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      uint32_t sel[8];
-      key_selectors<BK>(kw[nt], sel);
-      const uint32_t swn = nt ? sw.y : sw.x;
+    for (int kt = 0; kt < 4; ++kt) {
+      uint32_t ah[4], al[4], as[4];
+      key_limbs<BK>(sel0[2 * kt], kth_, ktl_, ah[0], al[0]);          // token g,     k 4t..
+      key_limbs<BK>(sel1[2 * kt], kth_, ktl_, ah[1], al[1]);          // token g + 8, k 4t..
+      key_limbs<BK>(sel0[2 * kt + 1], kth_, ktl_, ah[2], al[2]);      // token g,     k 16+4t..
+      key_limbs<BK>(sel1[2 * kt + 1], kth_, ktl_, ah[3], al[3]);      // token g + 8, k 16+4t..
+      as[0] = (kt == 0 ? sw.x : __umulhi(sw.x, 1u << (32 - 2 * kt))) & 0x01010101u;
+      as[1] = (kt == 0 ? sw.y : __umulhi(sw.y, 1u << (32 - 2 * kt))) & 0x01010101u;
+      as[2] = __umulhi(sw.x, 1u << (31 - 2 * kt)) & 0x01010101u;
+      as[3] = __umulhi(sw.y, 1u << (31 - 2 * kt)) & 0x01010101u;
 #pragma unroll
-      for (int kt = 0; kt < 4; ++kt) {
-        uint32_t h0, l0, h1, l1;
-        key_limbs<BK>(sel[2 * kt], kth_, ktl_, h0, l0);
-        key_limbs<BK>(sel[2 * kt + 1], kth_, ktl_, h1, l1);
-        const uint32_t s0 = (swn >> (2 * kt)) & 0x01010101u, s1 = (swn >> (2 * kt + 1)) & 0x01010101u;
+      for (int h = 0; h < NH; ++h)
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          const uint4 fq = reinterpret_cast<const uint4*>(s_qf)[((h * 2 + 0) * 4 + kt) * 32 + lane];
-          const uint4 fp = reinterpret_cast<const uint4*>(s_qf)[((h * 2 + 1) * 4 + kt) * 32 + lane];
-          const uint32_t aq[4] = {fq.x, fq.y, fq.z, fq.w};
-          const uint32_t ap[4] = {fp.x, fp.y, fp.z, fp.w};
-          mma_s8(dh[h][nt], aq, h0, h1);
-          mma_s8(dl[h][nt], aq, l0, l1);
-          mma_s8(ds[h][nt], ap, s0, s1);
+        for (int nt = 0; nt < 2; ++nt) {
+          uint32_t q0, q1, r0, r1;
+          if constexpr (kRegQ) {
+            q0 = bq[h][kt][nt][0]; q1 = bq[h][kt][nt][1]; r0 = bp[h][kt][nt][0]; r1 = bp[h][kt][nt][1];
+          } else {
+            const uint2 vq = reinterpret_cast<const uint2*>(s_qf + h * 1024 + ((0 * 4 + kt) * 2 + nt) * 64)[lane];
+            const uint2 vp = reinterpret_cast<const uint2*>(s_qf + h * 1024 + ((1 * 4 + kt) * 2 + nt) * 64)[lane];
+            q0 = vq.x; q1 = vq.y; r0 = vp.x; r1 = vp.y;
+          }
+          mma_s8(dh[h][nt], ah, q0, q1);
+          mma_s8(dl[h][nt], al, q0, q1);
+          mma_s8(ds[h][nt], as, r0, r1);
         }
-      }
     }
 
-    // ---- softmax statistics and split fp16 weights per head group
-    const int tok_base = lp * kPage;
+    // ---- softmax: one running maximum of l2 + log2|v| per head. The fp16 weight
+    // of token t is w_t = 2^(l2_t + log2|v_t| - m) <= 2^8 (the maximum is only
+    // moved when it grows by more than 8), and the softmax denominator gathers
+    // w_t / |v_t| = 2^(l2_t - m). Norms are floored at 2^-24 so that a zero value
+    // vector still counts in the denominator.
+    const int n_valid = page_ok ? L - lp * kPage : 0;     // tokens of this page inside the sequence
+    const float lgv0 = lg2(fmaxf(nV.x, 5.9604645e-8f)), lgv1 = lg2(fmaxf(nV.y, 5.9604645e-8f));
+    const float rnv0 = ex2(-lgv0), rnv1 = ex2(-lgv1);
     uint32_t pb[NH][2];
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
-      float l2[4], lp2[4];
+      float lp2[2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int idx = 2 * nt + i;
-          // bottom-limb partial sums live in quad g + 4 (lane + 16)
-          const float x0 = fmaf(256.0f, static_cast<float>(dh[h][nt][i]), static_cast<float>(dl[h][nt][i]));
-          const float x0r = __shfl_xor_sync(kFull, x0, 16);
-          const int s0r = __shfl_xor_sync(kFull, ds[h][nt][i], 16);
-          const int tok = tok_base + 8 * nt + 2 * t + i;
-          const float main = fmaf(16777216.0f, static_cast<float>(dh[h][nt][i]),
-                                  fmaf(65536.0f, static_cast<float>(dl[h][nt][i] + dh[h][nt][2 + i]),
-                                       fmaf(256.0f, static_cast<float>(dl[h][nt][2 + i]), x0r)));
-          const int sj = 65536 * ds[h][nt][i] + 256 * ds[h][nt][2 + i] + s0r;
-          const float qj = static_cast<float>(2 * sj - csum[h]);
-          const float v = fmaf(nK[idx] * main, ca[h], gam[idx] * qj * cb[h]);
-          const bool ok = owner && page_ok && tok < L;
-          l2[idx] = ok ? v : -INFINITY;
-          lp2[idx] = ok ? v + __log2f(nV[idx]) : -INFINITY;
-        }
-      float pm = fmaxf(fmaxf(l2[0], l2[1]), fmaxf(l2[2], l2[3]));
-      float pmp = fmaxf(fmaxf(lp2[0], lp2[1]), fmaxf(lp2[2], lp2[3]));
-      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 1));
-      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 2));
-      pmp = fmaxf(pmp, __shfl_xor_sync(kFull, pmp, 1));
-      pmp = fmaxf(pmp, __shfl_xor_sync(kFull, pmp, 2));
-      if (pm > m2[h] + 8.0f) {
-        lsum[h] *= exp2f(m2[h] - pm);
-        m2[h] = pm;
+      for (int r = 0; r < 2; ++r) {
+        // accumulator columns: n-tile 0 -> (Q2, Q1) of head t, n-tile 1 -> (Q0, 0)
+        //   <Q,C> = 2^16 (256 Q2.Chi + Q2.Clo + Q1.Chi) + 256 (Q1.Clo + Q0.Chi) + Q0.Clo
+        const int hiw = 256 * dh[h][0][2 * r] + dl[h][0][2 * r] + dh[h][0][2 * r + 1];
+        const int low = 256 * (dl[h][0][2 * r + 1] + dh[h][1][2 * r]) + dl[h][1][2 * r];
+        const float main = fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
+        const int sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + ds[h][1][2 * r];
+        const float nk = r ? nK.y : nK.x, gg = r ? gm.y : gm.x, lv = r ? lgv1 : lgv0;
+        const float v = fmaf(nk * ca[h], main, fmaf(gg * cb[h], static_cast<float>(2 * sj - csum[h]), lv));
+        lp2[r] = (g + 8 * r) < n_valid ? v : -INFINITY;
       }
-      lsum[h] += exp2f(l2[0] - m2[h]) + exp2f(l2[1] - m2[h]) + exp2f(l2[2] - m2[h]) + exp2f(l2[3] - m2[h]);
-      const bool need = pmp > mp2[h] + 8.0f;
-      const float fac = need ? exp2f(mp2[h] - pmp) : 1.0f;
-      if (need) mp2[h] = pmp;
+      float pm = fmaxf(lp2[0], lp2[1]);
+      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 4));
+      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 8));
+      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 16));
+      const bool need = pm > mp2[h] + 8.0f;
       if (__any_sync(kFull, need)) {
-        // acc columns 2t, 2t+1 hold heads (2t)&3, (2t+1)&3 (columns 4-7: low parts)
-        const float f0 = __shfl_sync(kFull, fac, 4 * ((2 * t) & 3));
-        const float f1 = __shfl_sync(kFull, fac, 4 * ((2 * t + 1) & 3));
+        const float fac = need ? ex2(mp2[h] - pm) : 1.0f;
+        if (need) mp2[h] = pm;
+        lsum[h] *= fac;
+        // value accumulator columns 2t, 2t+1 hold heads (2t)&3, (2t+1)&3 (columns 4-7: low parts)
+        const float f0 = __shfl_sync(kFull, fac, (2 * t) & 3);
+        const float f1 = __shfl_sync(kFull, fac, (2 * t + 1) & 3);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
           acc[h][mt][0] *= f0; acc[h][mt][1] *= f1; acc[h][mt][2] *= f0; acc[h][mt][3] *= f1;
         }
       }
-      float w[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w[i] = exp2f(lp2[i] - mp2[h]);
-      const __half2 hi01 = __floats2half2_rn(w[0], w[1]), hi23 = __floats2half2_rn(w[2], w[3]);
-      const float2 r01 = __half22float2(hi01), r23 = __half22float2(hi23);
-      const __half2 lo01 = __floats2half2_rn(w[0] - r01.x, w[1] - r01.y);
-      const __half2 lo23 = __floats2half2_rn(w[2] - r23.x, w[3] - r23.y);
-      const uint32_t lo01u = *reinterpret_cast<const uint32_t*>(&lo01);
-      const uint32_t lo23u = *reinterpret_cast<const uint32_t*>(&lo23);
-      const uint32_t plo01 = __shfl_xor_sync(kFull, lo01u, 16), plo23 = __shfl_xor_sync(kFull, lo23u, 16);
-      pb[h][0] = owner ? *reinterpret_cast<const uint32_t*>(&hi01) : plo01;
-      pb[h][1] = owner ? *reinterpret_cast<const uint32_t*>(&hi23) : plo23;
+      const float w0 = ex2(lp2[0] - mp2[h]), w1 = ex2(lp2[1] - mp2[h]);
+      lsum[h] = fmaf(w0, rnv0, fmaf(w1, rnv1, lsum[h]));
+      // weights of (token g, head t) and (token g+8, head t): high fp16 parts and residuals
+      const __half2 whi = __floats2half2_rn(w0, w1);
+      const float2 wr = __half22float2(whi);
+      const __half2 wlo = __floats2half2_rn(w0 - wr.x, w1 - wr.y);
+      const uint32_t uhi = *reinterpret_cast<const uint32_t*>(&whi);
+      const uint32_t ulo = *reinterpret_cast<const uint32_t*>(&wlo);
+      // value-product B operand: lane (g', t') needs column g' (head g'&3, high part
+      // if g' < 4) at tokens 2t', 2t'+1 (-> b0) and 2t'+8, 2t'+9 (-> b1); tokens 2t'
+      // and 2t'+8 of a head live in lane 4*(2t') + head, tokens 2t'+1, 2t'+9 in the next quad.
+      const uint32_t x0h = __shfl_sync(kFull, uhi, src0), x0l = __shfl_sync(kFull, ulo, src0);
+      const uint32_t x1h = __shfl_sync(kFull, uhi, src1), x1l = __shfl_sync(kFull, ulo, src1);
+      const uint32_t x0 = hi_col ? x0h : x0l, x1 = hi_col ? x1h : x1l;
+      pb[h][0] = prmt(x0, x1, 0x5410u);
+      pb[h][1] = prmt(x0, x1, 0x7632u);
     }
 
     // ---- weighted value sum in the rotated domain: fp16 tensor-core products
@@ -884,10 +1093,18 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     }
 
     // ---- refill this stage with the page kStages ahead (all its reads are consumed)
-    __syncwarp();
-    if (lane == 0 && k + kStages < nmine) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(k + kStages);
+    if (k + kStages < nmine) {
+      const int phys = page_id(k + kStages);     // convergent: every lane reaches here
+      __syncwarp();
+      if (lane == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(phys, s);
+      }
+      __syncwarp();
+    }
+    if (++s == kStages) {
+      s = 0;
+      parity ^= 1u;
     }
   }
   if (!alive) {
@@ -897,14 +1114,15 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   }
   __syncwarp();
   if (lane == 0)
-    for (int s = 0; s < kStages; ++s)
-      asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(mybar + s)) : "memory");
+    for (int s2 = 0; s2 < kStages; ++s2)
+      asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(mybar + s2)) : "memory");
 
   // ---- merge the warps of this CTA (the pipeline buffers are free now)
 #pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    lsum[h] += __shfl_xor_sync(kFull, lsum[h], 1);
-    lsum[h] += __shfl_xor_sync(kFull, lsum[h], 2);
+  for (int h = 0; h < NH; ++h) {                 // sum each head's denominator over its 8 lanes
+    lsum[h] += __shfl_xor_sync(kFull, lsum[h], 4);
+    lsum[h] += __shfl_xor_sync(kFull, lsum[h], 8);
+    lsum[h] += __shfl_xor_sync(kFull, lsum[h], 16);
   }
   __syncthreads();
   float* s_acc = reinterpret_cast<float*>(smem);                       // [warp][NH][8 columns][128]
@@ -918,9 +1136,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
         const int coord = 16 * mt + g + 8 * (c >> 1), col = 2 * t + (c & 1);
         s_acc[((warp * NH + h) * 8 + col) * 128 + coord] = acc[h][mt][c];
       }
-    if (t == 0 && owner) {
-      float* st = s_st + ((warp * NH + h) * kGroupHeads + g) * 3;
-      st[0] = m2[h]; st[1] = lsum[h]; st[2] = mp2[h];
+    if (g == 0) {
+      float* st = s_st + ((warp * NH + h) * kGroupHeads + t) * 3;
+      st[0] = mp2[h]; st[1] = lsum[h];
     }
   }
   __syncthreads();
@@ -928,25 +1146,22 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   for (int i = threadIdx.x; i < NH * kGroupHeads * 128; i += blockDim.x) {
     const int hh = i >> 7, coord = i & 127;          // hh = group * 4 + head
     const int h = hh >> 2, h4 = hh & 3;
-    float M = kNegBig, Mp = kNegBig;
+    float M = kNegBig;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      M = fmaxf(M, s_st[((w * NH + h) * kGroupHeads + h4) * 3 + 0]);
-      Mp = fmaxf(Mp, s_st[((w * NH + h) * kGroupHeads + h4) * 3 + 2]);
-    }
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_st[((w * NH + h) * kGroupHeads + h4) * 3 + 0]);
     float a = 0.0f, l = 0.0f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       const float* st = s_st + ((w * NH + h) * kGroupHeads + h4) * 3;
       const float* ac = s_acc + ((w * NH + h) * 8) * 128;
-      a += (ac[h4 * 128 + coord] + ac[(h4 + 4) * 128 + coord]) * exp2f(st[2] - Mp);
-      l += st[1] * exp2f(st[0] - M);
+      const float f = ex2(st[0] - M);
+      a = fmaf(ac[h4 * 128 + coord] + ac[(h4 + 4) * 128 + coord], f, a);
+      l = fmaf(st[1], f, l);
     }
     part[hh * 132 + coord] = a;
     if (coord == 0) {
       part[hh * 132 + 128] = M;
       part[hh * 132 + 129] = l;
-      part[hh * 132 + 130] = Mp;
     }
   }
   __threadfence();
@@ -959,48 +1174,61 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   if (!s_last) return;
   __threadfence();
 
-  // ---- last CTA of this (sequence, KV head): merge chunks, de-rotate, store
+  // ---- last CTA of this (sequence, KV head): merge chunks, de-rotate, store.
+  // Warp w takes head slot w % 4 (+4 per round) and every second chunk from
+  // w / 4; the two halves meet in shared memory.
   const float* pbase = A.partial + static_cast<size_t>(pair) * A.chunks * NH * kGroupHeads * 132;
-  for (int slot = warp; slot < A.group; slot += kWarps) {
-    float M = kNegBig, Mp = kNegBig;
-    for (int c = lane; c < A.chunks; c += 32) {
-      const float* st = pbase + (static_cast<size_t>(c) * NH * kGroupHeads + slot) * 132 + 128;
-      M = fmaxf(M, __ldcg(st));
-      Mp = fmaxf(Mp, __ldcg(st + 2));
-    }
-    M = warp_max(M);
-    Mp = warp_max(Mp);
-    float l = 0.0f;
+  float* s_mrg = reinterpret_cast<float*>(smem);            // [2 halves][4 slots][132]
+  for (int base = 0; base < A.group; base += kGroupHeads) {
+    const int slot = base + (warp & 3), half = warp >> 2;
+    float M = kNegBig, l = 0.0f;
     float a[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < A.chunks; ++c) {
-      const float* pc = pbase + (static_cast<size_t>(c) * NH * kGroupHeads + slot) * 132;
-      const float wl = exp2f(__ldcg(pc + 128) - M);
-      const float wa = exp2f(__ldcg(pc + 130) - Mp);
-      l = fmaf(__ldcg(pc + 129), wl, l);
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(pc) + lane);
-      a[0] = fmaf(v.x, wa, a[0]); a[1] = fmaf(v.y, wa, a[1]);
-      a[2] = fmaf(v.z, wa, a[2]); a[3] = fmaf(v.w, wa, a[3]);
+    if (slot < A.group) {
+      for (int c = half + 2 * lane; c < A.chunks; c += 64)
+        M = fmaxf(M, __ldcg(pbase + (static_cast<size_t>(c) * NH * kGroupHeads + slot) * 132 + 128));
+      M = warp_max(M);
+#pragma unroll 4
+      for (int c = half; c < A.chunks; c += 2) {
+        const float* pc = pbase + (static_cast<size_t>(c) * NH * kGroupHeads + slot) * 132;
+        const float wc = ex2(__ldcg(pc + 128) - M);
+        l = fmaf(__ldcg(pc + 129), wc, l);
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(pc) + lane);
+        a[0] = fmaf(v.x, wc, a[0]); a[1] = fmaf(v.y, wc, a[1]);
+        a[2] = fmaf(v.z, wc, a[2]); a[3] = fmaf(v.w, wc, a[3]);
+      }
     }
-    const float f = l > 0.0f ? exp2f(Mp - M) / l : 0.0f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) a[e] *= f;
-    fwht128(a, lane);
-    float4 o;
-    o.x = a[0] * T.signs_v[4 * lane + 0] * kInvSqrtD;
-    o.y = a[1] * T.signs_v[4 * lane + 1] * kInvSqrtD;
-    o.z = a[2] * T.signs_v[4 * lane + 2] * kInvSqrtD;
-    o.w = a[3] * T.signs_v[4 * lane + 3] * kInvSqrtD;
-    const int qh = hk * A.group + slot;
-    reinterpret_cast<float4*>(A.out + (static_cast<size_t>(b) * A.n_q + qh) * 128)[lane] = o;
+    float* mine = s_mrg + (half * 4 + (warp & 3)) * 132;
+    reinterpret_cast<float4*>(mine)[lane] = make_float4(a[0], a[1], a[2], a[3]);
+    if (lane == 0) { mine[128] = M; mine[129] = l; }
+    __syncthreads();
+    if (half == 0 && slot < A.group) {
+      const float* other = s_mrg + (4 + (warp & 3)) * 132;
+      const float Mo = other[128];
+      const float Mx = fmaxf(M, Mo);
+      const float f0 = ex2(M - Mx), f1 = ex2(Mo - Mx);
+      const float lt = l * f0 + other[129] * f1;
+      const float4 ao = reinterpret_cast<const float4*>(other)[lane];
+      const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+      a[0] = (a[0] * f0 + ao.x * f1) * inv; a[1] = (a[1] * f0 + ao.y * f1) * inv;
+      a[2] = (a[2] * f0 + ao.z * f1) * inv; a[3] = (a[3] * f0 + ao.w * f1) * inv;
+      fwht128(a, lane);
+      float4 o;
+      o.x = a[0] * T.signs_v[4 * lane + 0] * kInvSqrtD;
+      o.y = a[1] * T.signs_v[4 * lane + 1] * kInvSqrtD;
+      o.z = a[2] * T.signs_v[4 * lane + 2] * kInvSqrtD;
+      o.w = a[3] * T.signs_v[4 * lane + 3] * kInvSqrtD;
+      const int qh = hk * A.group + slot;
+      reinterpret_cast<float4*>(A.out + (static_cast<size_t>(b) * A.n_q + qh) * 128)[lane] = o;
+    }
+    __syncthreads();
   }
-  if (threadIdx.x == 0) A.counters[pair] = 0u;
 }
 
 template <int BK, int BV, int NH>
 cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
-  const size_t pipe = static_cast<size_t>(kWarps) * kStages * kBlock + kWarps * kStages * sizeof(uint64_t) +
-                      static_cast<size_t>(NH) * 1024 * 4;
+  constexpr size_t kPro = NH > 2 ? static_cast<size_t>(NH) * 1024 * 4 : 0;   // query fragments in smem
+  const size_t pipe = static_cast<size_t>(kWarps) * kStages * kBlock + kWarps * kStages * sizeof(uint64_t) + kPro;
   const size_t merge = static_cast<size_t>(kWarps) * NH * 8 * 128 * 4 + kWarps * NH * kGroupHeads * 3 * 4;
   const size_t smem = pipe > merge ? pipe : merge;
   auto fn = decode_kernel<BK, BV, NH>;
@@ -1069,6 +1297,27 @@ cudaError_t launch_quantize_prefill(const Tables& t, const void* k, const void* 
   return cudaGetLastError();
 }
 
+cudaError_t launch_decode_common(const Tables& t, const DecodePlan& plan, const void* cache, int64_t n_pages,
+                                 const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
+                                 int max_seq_len, float* out, void* workspace, int hold_last_page,
+                                 cudaStream_t s);
+
+cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
+                               int kv_dtype, const void* q, int q_dtype, void* cache, int64_t n_pages,
+                               const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
+                               int max_seq_len, float scale, float* out, void* workspace, cudaStream_t s) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  step_prep_kernel<<<dim3(plan.n_hg + 1, plan.n_kv, plan.batch), 512, 0, s>>>(
+      t, q, q_dtype, plan.n_q, plan.n_kv, plan.group, plan.n_hg, scale,
+      reinterpret_cast<uint32_t*>(ws + plan.off_qfrag), reinterpret_cast<float*>(ws + plan.off_qconst),
+      reinterpret_cast<unsigned*>(ws + plan.off_counter), k_new,
+      v_new, kv_dtype, static_cast<uint8_t*>(cache), n_pages, block_tables, max_pages_per_seq, seq_lens);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_decode_common(t, plan, cache, n_pages, block_tables, max_pages_per_seq, seq_lens, max_seq_len,
+                              out, workspace, 1, s);
+}
+
 cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype,
                           const void* cache, int64_t n_pages, const int32_t* block_tables,
                           int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len, float scale,
@@ -1076,12 +1325,20 @@ cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws + plan.off_qfrag);
   float* qconst = reinterpret_cast<float*>(ws + plan.off_qconst);
-  float* partial = reinterpret_cast<float*>(ws + plan.off_partial);
-  unsigned* counters = reinterpret_cast<unsigned*>(ws + plan.off_counter);
   qtransform_kernel<<<dim3(plan.n_hg, plan.n_kv, plan.batch), 512, 0, s>>>(
-      t, q, q_dtype, plan.n_q, plan.n_kv, plan.group, plan.n_hg, scale, qfrag, qconst, counters);
+      t, q, q_dtype, plan.n_q, plan.n_kv, plan.group, plan.n_hg, scale, qfrag, qconst,
+      reinterpret_cast<unsigned*>(ws + plan.off_counter));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  return launch_decode_common(t, plan, cache, n_pages, block_tables, max_pages_per_seq, seq_lens, max_seq_len,
+                              out, workspace, 0, s);
+}
+
+cudaError_t launch_decode_common(const Tables& t, const DecodePlan& plan, const void* cache, int64_t n_pages,
+                                 const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
+                                 int max_seq_len, float* out, void* workspace, int hold_last_page,
+                                 cudaStream_t s) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeArgs a;
   a.cache = static_cast<const uint8_t*>(cache);
   a.n_pages = n_pages;
@@ -1089,10 +1346,11 @@ cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q
   a.max_pages_per_seq = max_pages_per_seq;
   a.seq_lens = seq_lens;
   a.max_seq_len = max_seq_len;
-  a.qfrag = qfrag;
-  a.qconst = qconst;
-  a.partial = partial;
-  a.counters = counters;
+  a.qfrag = reinterpret_cast<const uint32_t*>(ws + plan.off_qfrag);
+  a.qconst = reinterpret_cast<const float*>(ws + plan.off_qconst);
+  a.partial = reinterpret_cast<float*>(ws + plan.off_partial);
+  a.counters = reinterpret_cast<unsigned*>(ws + plan.off_counter);
+  a.hold_last_page = hold_last_page;
   a.out = out;
   a.n_kv = plan.n_kv;
   a.n_q = plan.n_q;

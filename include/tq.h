@@ -150,6 +150,23 @@ tq_status tq_decode_attention(tq_ctx* ctx, const void* q, tq_dtype q_dtype, cons
                               float* out, void* workspace, size_t workspace_bytes,
                               tq_stream stream);
 
+/*
+ * One decode step: append one new token per sequence, then attend. For each
+ * sequence b with seq_lens[b] > 0, the key/value k_new[b], v_new[b]
+ * ([batch, n_kv_heads, 128], dtype kv_dtype) are quantized exactly as by
+ * tq_quantize_append and stored at logical position seq_lens[b] - 1 (page
+ * block_tables[b][(seq_lens[b]-1)/16]); then q is attended over positions
+ * [0, seq_lens[b]) exactly as by tq_decode_attention, so the new token is seen.
+ * Same arguments, workspace and error behaviour as tq_decode_attention. The
+ * attention kernel starts streaming the cache while the new token is being
+ * quantized (every page except each sequence's last one).
+ */
+tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+                         const void* q, tq_dtype q_dtype, void* cache, int64_t n_cache_pages,
+                         const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
+                         int batch, int n_q_heads, int n_kv_heads, int max_seq_len, float scale, float* out,
+                         void* workspace, size_t workspace_bytes, tq_stream stream);
+
 /* Synchronise `stream`, then read and clear the device error word (TQ_DEV_* bits). */
 tq_status tq_get_device_error(tq_ctx* ctx, uint32_t* code, tq_stream stream);
 

@@ -3,7 +3,9 @@
 Oracle module (test infrastructure only). The pages give no byte format (the
 llama.cpp fork's own formats are not shown), so this layout is a reading,
 chosen so that a GPU warp can turn the bytes straight into tensor-core
-operands. It is written out here from its definition, bit by bit.
+operands (key codes and sign bits: the A operand of a 16-token tile, one token
+per row; value codes: the A operand of the transposed value tile; the norms of
+tokens g and g + 8 share one 32-bit word). It is written out here from its definition, bit by bit.
 
 Block for one (page, KV head), head_dim d = 128, m = 128 sketch rows, with
 b_k-bit key codes and b_v-bit value codes:
@@ -11,7 +13,8 @@ b_k-bit key codes and b_v-bit value codes:
     offset 0                 K codes   256*b_k bytes = 32 lane chunks of 8*b_k bytes
     offset 256*b_k           sign bits 256 bytes     = 32 lane chunks of 8 bytes
     offset 256*(b_k+1)       V codes   256*b_v bytes = 32 lane chunks of 8*b_v bytes
-    offset 256*(b_k+b_v+1)   norms     96 bytes: ||k|| fp16[16], gamma fp16[16], ||v|| fp16[16]
+    offset 256*(b_k+b_v+1)   norms     96 bytes: ||k|| fp16[16], gamma fp16[16], ||v|| fp16[16];
+                             token tau sits at entry 2*(tau & 7) + (tau >> 3) of each array
 
 Words are 32-bit little endian; bit x of word w of a section is bit (x mod 8)
 of byte 4w + x // 8.
@@ -138,6 +141,11 @@ def _get_bits(block: np.ndarray, idx: np.ndarray) -> np.ndarray:
     return (block[idx // 8] >> (idx % 8).astype(np.uint8)) & 1
 
 
+def norm_slot(tau: int) -> int:
+    """Entry of token tau in each 16-entry fp16 norm array."""
+    return 2 * (tau & 7) + (tau >> 3)
+
+
 def write_token(block, tau, bk, bv, k_codes, sign_bits, v_codes, k_norm16, gamma16, v_norm16):
     """Store one token's fields into a block (uint8 view), leaving other tokens' bits alone."""
     kb = k_bit_index(bk)[tau]                      # [128, bk]
@@ -148,9 +156,10 @@ def write_token(block, tau, bk, bv, k_codes, sign_bits, v_codes, k_norm16, gamma
     vval = (np.asarray(v_codes)[:, None] >> np.arange(bv)) & 1
     _set_bits(block, vb, vval)
     no = section_offsets(bk, bv)["norm"]
+    e = norm_slot(tau)
     for arr_off, val in ((0, k_norm16), (32, gamma16), (64, v_norm16)):
         h = np.array([val], dtype=np.float16).view(np.uint8)
-        block[no + arr_off + 2 * tau: no + arr_off + 2 * tau + 2] = h
+        block[no + arr_off + 2 * e: no + arr_off + 2 * e + 2] = h
 
 
 def read_page(block, bk, bv):
@@ -163,4 +172,5 @@ def read_page(block, bk, bv):
     v_codes = np.sum(_get_bits(block, vb).astype(np.int64) << np.arange(bv), axis=-1)
     no = section_offsets(bk, bv)["norm"]
     norms = block[no:no + 96].view(np.float16).astype(np.float64).reshape(3, PAGE)
-    return k_codes, sign_bits, v_codes, norms[0], norms[1], norms[2]
+    order = [norm_slot(tau) for tau in range(PAGE)]
+    return k_codes, sign_bits, v_codes, norms[0][order], norms[1][order], norms[2][order]

@@ -238,3 +238,40 @@ def test_decode_step_attends_the_appended_token():
         want = odec.decode_paged(host, bt, [L], q.astype(np.float64), tab)
         assert_outputs_close(out.cpu().numpy().astype(np.float64), want)
     assert ctx.device_error() == 0
+
+
+def test_decode_step_api_matches_oracle():
+    """tq_decode_step: append one token per sequence at seq_len - 1, then attend (batch 2)."""
+    bk, bv, n_kv, g = 3, 2, 2, 4
+    seeds = (8, 9, 10)
+    tab = oracle_tables(seeds, bk, bv)
+    rng = np.random.default_rng(11)
+    L0 = [47, 16]                                   # appends cross a page boundary in both
+    steps = 3
+    kv = [_rand_kv(rng, L + steps, n_kv, "bf16") for L in L0]
+    bt, n_pages = _pool([L + steps for L in L0], 4)
+    ctx = _ctx(bk, bv, seeds)
+    cache = torch.zeros(n_pages * ctx.page_bytes(n_kv), dtype=torch.uint8, device=DEV)
+    btt = torch.from_numpy(bt).to(DEV)
+    for b, L in enumerate(L0):
+        ctx.quantize_prefill(_t(kv[b][0][:L], "bf16"), _t(kv[b][1][:L], "bf16"), btt[b], 0, cache, n_pages)
+    max_len = max(L0) + steps
+    ws = torch.empty(ctx.decode_workspace_bytes(2, n_kv * g, n_kv, max_len), dtype=torch.uint8, device=DEV)
+    for step in range(steps):
+        lens = [L + step + 1 for L in L0]
+        k_new = np.stack([kv[b][0][lens[b] - 1] for b in range(2)])
+        v_new = np.stack([kv[b][1][lens[b] - 1] for b in range(2)])
+        q = synth.round_to_bf16(rng.standard_normal((2, n_kv * g, 128)).astype(np.float32))
+        out = torch.full((2, n_kv * g, 128), float("nan"), device=DEV)
+        ctx.decode_step(_t(k_new, "bf16"), _t(v_new, "bf16"), _t(q, "bf16"), cache, n_pages, btt,
+                        torch.tensor(lens, dtype=torch.int32, device=DEV), n_kv, max_len, out, ws)
+        host = cache.cpu().numpy().reshape(n_pages, n_kv, -1)
+        # the appended token equals the oracle's quantization of it
+        for b in range(2):
+            for h in range(n_kv):
+                qk, qv = oracle_quantize(k_new[b:b + 1, h].astype(np.float64), v_new[b:b + 1, h].astype(np.float64), tab)
+                rep = compare_tokens(unpack_tokens(host, bt[b], lens[b] - 1, 1, h, bk, bv), qk, qv, tab)
+                assert all(val == 0 for key, val in rep.items() if key.startswith("bad")), rep
+        want = odec.decode_paged(host, bt, lens, q.astype(np.float64), tab)
+        assert_outputs_close(out.cpu().numpy().astype(np.float64), want)
+    assert ctx.device_error() == 0
