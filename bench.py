@@ -5,7 +5,8 @@ Workload (default ``llama8b``): Llama-3.1-8B-shaped decode, batch 1, 32 query /
 3-bit + QJL (m = 128), values 2-bit, 32 layers. One step = one generated token:
 for each of the 32 layers, one tq_decode_step call quantizes and appends the new
 token's K/V (8 heads) and runs decode attention for the 32 query heads over the
-whole cache (two kernel launches: step preparation, then split-K attention). The 32 layer
+whole cache (one kernel launch per layer: the CTA that owns the sequence's last page
+quantizes the new token while the other CTAs already stream their pages). The 32 layer
 caches (about 0.86 GB) exceed the 126 MB L2, so every step streams from HBM.
 
 ``value``   decode tokens/s with inputs resident in HBM (CUDA-graph replay of
@@ -13,8 +14,8 @@ caches (about 0.86 GB) exceed the 126 MB L2, so every step streams from HBM.
 ``e2e``     the same steps through the C ABI with host buffers: per step the
             new K/V and queries are copied from pinned host memory and the
             attention outputs copied back, inside the timed region.
-``roofline`` decode attention (tq_decode_attention: query transform + split-K
-            decode) against the measured HBM copy bandwidth: algorithmic bytes =
+``roofline`` decode attention (tq_decode_attention: one kernel doing the query
+            transform, split-K decode and the split merge) against the measured HBM copy bandwidth: algorithmic bytes =
             compressed bytes of every cached token-head read (102 B each).
 ``cpu_baseline`` the float64 oracle on the host, on a bounded sample.
 
@@ -179,7 +180,7 @@ class DecodeBench:
                                  device=device).reshape(-1, 1)
         self.out = torch.zeros((self.n_layers, B, nq, 128), dtype=torch.float32, device=device)
         self.ws_bytes = self.ctx.decode_workspace_bytes(B, nq, n_kv, self.max_len)
-        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=device)
         # host-side buffers for the end-to-end arm
         self.h_newk = torch.empty((self.total_steps, self.n_layers, n_kv, 128), dtype=torch.bfloat16,
                                   pin_memory=True)
@@ -434,9 +435,9 @@ def main():
         "e2e": {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                     "kernel": "tq_decode_attention (qtransform + split-K decode)",
+                     "kernel": "decode_kernel via tq_decode_attention (query transform, split-K decode, merge)",
                      "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
-        "gpu_launches": K * bench.n_layers * 2,
+        "gpu_launches": K * bench.n_layers,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -294,14 +294,10 @@ DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int block_by
   p.chunks = (p.max_pages + ppc - 1) / ppc;
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   size_t off = 0;
-  p.off_qfrag = off;
-  off = al(off + static_cast<size_t>(pairs) * p.n_hg * 1024 * sizeof(uint32_t));
-  p.off_qconst = off;
-  off = al(off + static_cast<size_t>(pairs) * p.n_hg * 4 * 4 * sizeof(float));
   p.off_partial = off;
   off = al(off + static_cast<size_t>(pairs) * p.chunks * p.n_hg * 4 * 132 * sizeof(float));
   p.off_counter = off;
-  off = al(off + static_cast<size_t>(pairs) * sizeof(unsigned long long));
+  off = al(off + static_cast<size_t>(pairs) * sizeof(unsigned));
   p.total = off;
   return p;
 }

@@ -37,7 +37,7 @@ struct Tables {
 struct DecodePlan {
   int batch, n_q, n_kv, group, n_hg;  // n_hg = ceil(group / 4) groups of 4 query heads
   int max_pages, pages_per_chunk, chunks;
-  size_t off_qfrag, off_qconst, off_partial, off_counter, total;
+  size_t off_partial, off_counter, total;
 };
 
 DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int block_bytes);

@@ -22,6 +22,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cstddef>
 #include <cstdint>
 
 namespace tq {
@@ -440,201 +441,6 @@ __device__ __forceinline__ int warp_isum(int v) {
   return v;
 }
 
-// Query transform kernel: grid (n_hg, n_kv, batch), 512 threads; warp w -> head
-// slot w >> 2 of the group, sketch-column quarter w & 3. Writes
-//   qfrag[pair][hg][which (q, p)][kt 4][ntile 2][lane 32][reg 2]  (int32 words of 4 int8)
-//   qconst[pair][hg][slot 4][4] = {a, b, sum P (int bits), 0}.
-__device__ void qtransform_group(const Tables& T, const void* q, int dtype, int n_q, int n_kv, int group,
-                                 int n_hg, float scale, uint32_t* qfrag, float* qconst, unsigned* counters,
-                                 int hg, int hk, int b, float (*s_q)[128], float (*s_p)[kGroupHeads][128]) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int hs = w >> 2, cq = w & 3;
-  // split-K completion counter of this (sequence, KV head): the attention kernel
-  // that follows in the same call counts its finished CTAs here
-  if (hg == 0 && threadIdx.x == 0) counters[b * n_kv + hk] = 0u;
-  const int pair = b * n_kv + hk;
-  const int slot = hg * kGroupHeads + hs;
-  if (cq == 0) {
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
-    if (slot < group) load_row4(q, static_cast<size_t>(b) * n_q + hk * group + slot, dtype, lane, x);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] *= T.signs_k[4 * lane + e];
-    fwht128(x, lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s_q[hs][4 * lane + e] = x[e] * kInvSqrtD;
-  }
-  __syncthreads();
-  {  // partial p over the 32 sketch columns of this quarter: rows 4*lane .. 4*lane+3
-    const uint2* st = reinterpret_cast<const uint2*>(T.sketch_t);
-    uint2 raw[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) raw[j] = __ldg(st + (32 * cq + j) * 32 + lane);
-    float p[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float qc = s_q[hs][32 * cq + j];
-      const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j].x));
-      const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j].y));
-      p[0] = fmaf(s01.x, qc, p[0]);
-      p[1] = fmaf(s01.y, qc, p[1]);
-      p[2] = fmaf(s23.x, qc, p[2]);
-      p[3] = fmaf(s23.y, qc, p[3]);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s_p[cq][hs][4 * lane + e] = p[e];
-  }
-  __syncthreads();
-  if (cq != 0) return;
-  float x[4], p[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    x[e] = s_q[hs][4 * lane + e];
-    p[e] = s_p[0][hs][4 * lane + e] + s_p[1][hs][4 * lane + e] + s_p[2][hs][4 * lane + e] +
-           s_p[3][hs][4 * lane + e];
-  }
-  const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
-  const int ep = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(p[0]), fabsf(p[1])), fmaxf(fabsf(p[2]), fabsf(p[3])))));
-  const Limbs lq = split3(x, eq);
-  const Limbs lp = split3(p, ep);
-  const int psum = warp_isum(lp.sum);              // |sum| < 2^29
-  // lane l holds rows 4l..4l+3 of B: k-tile kt = l>>3, register sub = (l>>2)&1, t = l&3
-  const int kt = lane >> 3, sub = (lane >> 2) & 1, t = lane & 3;
-  uint32_t* base = qfrag + (static_cast<size_t>(pair) * n_hg + hg) * 1024;
-  const int ln_a = 4 * (2 * hs) + t, ln_b = 4 * (2 * hs + 1) + t;      // columns 2hs and 2hs + 1
-#pragma unroll
-  for (int which = 0; which < 2; ++which) {
-    const Limbs& Lm = which ? lp : lq;
-    uint32_t* f = base + (which * 4 + kt) * 128;      // [ntile 2][lane 32][reg 2]
-    f[0 * 64 + ln_a * 2 + sub] = Lm.w2;
-    f[0 * 64 + ln_b * 2 + sub] = Lm.w1;
-    f[1 * 64 + ln_a * 2 + sub] = Lm.w0;
-    f[1 * 64 + ln_b * 2 + sub] = 0u;
-  }
-  if (lane == 0) {
-    float* qc = qconst + ((static_cast<size_t>(pair) * n_hg + hg) * kGroupHeads + hs) * 4;
-    const bool real = slot < group;
-    qc[0] = real ? scale * kLog2e * ldexpf(1.0f, -eq - T.k_exp) : 0.0f;
-    qc[1] = real ? scale * kLog2e * kSqrtPiOver2 / kQjlRows * ldexpf(1.0f, -ep) : 0.0f;
-    qc[2] = __int_as_float(real ? psum : 0);
-    qc[3] = 0.0f;
-  }
-}
-
-__global__ void __launch_bounds__(512) qtransform_kernel(Tables T, const void* q, int dtype, int n_q,
-                                                         int n_kv, int group, int n_hg, float scale,
-                                                         uint32_t* qfrag, float* qconst, unsigned* counters) {
-  // the decode kernel may start now: it prefetches pages until it needs these outputs
-  asm volatile("griddepcontrol.launch_dependents;");
-  __shared__ float s_q[kGroupHeads][128];
-  __shared__ float s_p[4][kGroupHeads][128];
-  qtransform_group(T, q, dtype, n_q, n_kv, group, n_hg, scale, qfrag, qconst, counters, blockIdx.x, blockIdx.y,
-                   blockIdx.z, s_q, s_p);
-}
-
-// Decode step preparation: grid (n_hg + 1, n_kv, batch), 512 threads. CTAs with
-// x < n_hg run the query transform of group x; the CTA with x == n_hg quantizes
-// the new key and value of (sequence z, KV head y) and stores them at logical
-// position seq_lens[z] - 1 (sequences of length 0 append nothing).
-__global__ void __launch_bounds__(512) step_prep_kernel(Tables T, const void* q, int q_dtype, int n_q, int n_kv,
-                                                        int group, int n_hg, float scale, uint32_t* qfrag,
-                                                        float* qconst, unsigned* counters, const void* k_new,
-                                                        const void* v_new,
-                                                        int kv_dtype, uint8_t* cache, int64_t n_pages,
-                                                        const int32_t* block_tables, int max_pages_per_seq,
-                                                        const int32_t* seq_lens) {
-  asm volatile("griddepcontrol.launch_dependents;");
-  __shared__ float s_q[kGroupHeads][128];
-  __shared__ float s_p[4][kGroupHeads][128];
-  const int hg = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  if (hg < n_hg) {
-    qtransform_group(T, q, q_dtype, n_q, n_kv, group, n_hg, scale, qfrag, qconst, counters, hg, hk, b, s_q, s_p);
-    return;
-  }
-  const int L = seq_lens[b];
-  if (L <= 0) return;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int pos = L - 1, lpage = pos / kPage, tau = pos % kPage;
-  if (lpage >= max_pages_per_seq) {
-    if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_LENGTH);
-    return;
-  }
-  const int phys = block_tables[static_cast<int64_t>(b) * max_pages_per_seq + lpage];
-  if (phys < 0 || phys >= n_pages) {
-    if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_SLOT);
-    return;
-  }
-  uint8_t* blk = cache + (static_cast<int64_t>(phys) * n_kv + hk) * T.block_bytes;
-  float* s_u = &s_q[0][0];                          // residual of the key
-  __shared__ VecOut s_key[32];
-  const size_t row = static_cast<size_t>(b) * n_kv + hk;
-  float x[4];
-  if (w == 0) {                                     // key: rotation, codes, residual
-    load_row4(k_new, row, kv_dtype, lane, x);
-    VecOut o;
-    quantize_vector(x, T.signs_k, T.thr_k, T.cen_k, T.key_bits, nullptr, false, lane, o);
-    // residual u = y - c[code] recomputed from the codes (same arithmetic as quantize_vector)
-    float v4[4];
-    float ss = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) { ss = fmaf(x[e], x[e], ss); v4[e] = x[e] * T.signs_k[4 * lane + e]; }
-    ss = warp_sum(ss);
-    const float n = sqrtf(ss);
-    fwht128(v4, lane);
-    const float inv = n > 0.0f ? 1.0f / (n * 11.313708498984761f) : 0.0f;
-    float uu = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float u = v4[e] * inv - T.cen_k[o.code[e]];
-      s_u[4 * lane + e] = u;
-      uu = fmaf(u, u, uu);
-    }
-    uu = warp_sum(uu);
-    o.gamma = n * sqrtf(uu);
-    s_key[lane] = o;
-  } else if (w == 1) {                              // value: rotation, codes, store
-    load_row4(v_new, row, kv_dtype, lane, x);
-    VecOut o;
-    quantize_vector(x, T.signs_v, T.thr_v, T.cen_v, T.value_bits, nullptr, false, lane, o);
-    store_value_token(blk, tau, T.key_bits, T.value_bits, o, lane);
-    if (lane == 0) store_norm(blk, T.key_bits, T.value_bits, 2, tau, o.norm);
-  }
-  __syncthreads();
-  if (w < 4) {                                      // z = S u: warp w sums sketch columns 32w .. 32w+31
-    const uint2* st = reinterpret_cast<const uint2*>(T.sketch_t);
-    uint2 raw[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) raw[j] = __ldg(st + (32 * w + j) * 32 + lane);
-    float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float uc = s_u[32 * w + j];
-      const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j].x));
-      const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j].y));
-      z[0] = fmaf(s01.x, uc, z[0]);
-      z[1] = fmaf(s01.y, uc, z[1]);
-      z[2] = fmaf(s23.x, uc, z[2]);
-      z[3] = fmaf(s23.y, uc, z[3]);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s_p[w][0][4 * lane + e] = z[e];
-  }
-  __syncthreads();
-  if (w == 0) {
-    VecOut o = s_key[lane];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float z = s_p[0][0][4 * lane + e] + s_p[1][0][4 * lane + e] + s_p[2][0][4 * lane + e] +
-                      s_p[3][0][4 * lane + e];
-      o.sgn[e] = z >= 0.0f ? 1 : 0;
-    }
-    store_key_token(blk, tau, T.key_bits, o, lane);
-    if (lane == 0) {
-      store_norm(blk, T.key_bits, T.value_bits, 0, tau, o.norm);
-      store_norm(blk, T.key_bits, T.value_bits, 1, tau, o.gamma);
-    }
-  }
-}
-
 // ================================================================== decode
 constexpr int kWarps = 8;        // compute warps per CTA
 constexpr int kStages = 6;       // TMA stages per warp
@@ -774,22 +580,6 @@ __device__ __forceinline__ void value_regs(uint32_t sel, const uint32_t (&vl)[4]
   r1 = prmt(lo, hi, 0x7362u);
 }
 
-struct DecodeArgs {
-  const uint8_t* cache;
-  int64_t n_pages;
-  const int32_t* block_tables;
-  int max_pages_per_seq;
-  const int32_t* seq_lens;
-  int max_seq_len;
-  const uint32_t* qfrag;         // written by the query transform (see above)
-  const float* qconst;
-  float* partial;                // [pair][chunk][hg][4 heads][132]
-  unsigned* counters;            // [pair]: finished CTAs, zeroed by the preceding kernel of the call
-  int hold_last_page;            // 1: a preceding kernel of this call appends to each sequence's last page
-  float* out;                    // [batch][n_q][128]
-  int n_kv, n_q, group, n_hg, chunks, ppc;
-};
-
 // Load N 32-bit words from 8-byte-aligned shared memory with the widest accesses.
 template <int N>
 __device__ __forceinline__ void lds_words(const uint32_t* src, uint32_t (&dst)[N]) {
@@ -808,9 +598,76 @@ __device__ __forceinline__ void lds_words(const uint32_t* src, uint32_t (&dst)[N
   }
 }
 
-// Split-K decode attention. grid (chunks, n_kv, batch), kWarps warps per CTA.
-// Each warp streams its pages (every kWarps-th page of the chunk) through a
-// private ring of kStages shared-memory stages filled by 1-D bulk TMA copies.
+struct DecodeArgs {
+  const void* q;                 // [batch][n_q][128]
+  int q_dtype;
+  float scale;
+  const void* k_new;             // [batch][n_kv][128] (decode step only)
+  const void* v_new;
+  int kv_dtype;
+  uint8_t* cache;
+  int64_t n_pages;
+  const int32_t* block_tables;
+  int max_pages_per_seq;
+  const int32_t* seq_lens;
+  int max_seq_len;
+  float* partial;                // [pair][chunk][hg][4 heads][132]
+  unsigned* counters;            // [pair]: finished CTAs; zero between calls
+  float* out;                    // [batch][n_q][128]
+  int n_kv, n_q, group, n_hg, chunks, ppc;
+};
+
+// Shared-memory scratch of the prologue (after the stages and barriers).
+// Every member starts on a 16-byte boundary (vector loads read qt and u).
+template <int NH>
+struct alignas(16) Prologue {
+  alignas(16) float qt[NH * kGroupHeads][128];     // rotated queries q~
+  alignas(16) float pp[NH * kGroupHeads][128];     // sketch products S q~
+  alignas(16) uint32_t limb[NH * kGroupHeads][192];  // [which (q, p)][limb 0..2][32 words of 4 int8]
+  alignas(16) float cst[NH * kGroupHeads][4];      // a, b, sum P (int bits)
+  alignas(16) float u[128];                        // residual of the appended key
+  alignas(16) float z[128];                        // S u
+  alignas(16) float tab[64];                       // key / value thresholds and centroids
+  alignas(16) VecOut key[32];                      // appended key: codes and norms per lane
+  alignas(16) int sig[NH * kGroupHeads + 1];       // fp16 scaling exponents (last: appended key residual)
+};
+static_assert(offsetof(Prologue<1>, u) % 16 == 0 && offsetof(Prologue<3>, u) % 16 == 0, "alignment");
+
+// Rotate and code one vector held 4 per lane; returns codes in o, n and (keys) gamma,
+// and the residual u = y - c[code] per lane.
+__device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float* signs, const float* thr,
+                                                const float* cen, int bits, int lane, VecOut& o, float (&u)[4]) {
+  float v[4];
+  float ss = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    ss = fmaf(x[e], x[e], ss);
+    v[e] = x[e] * signs[4 * lane + e];
+  }
+  ss = warp_sum(ss);
+  const float n = sqrtf(ss);
+  fwht128(v, lane);
+  const float inv = n > 0.0f ? 1.0f / (n * 11.313708498984761f) : 0.0f;
+  const int n_thr = (1 << bits) - 1;
+  float uu = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float y = v[e] * inv;
+    o.code[e] = encode(y, thr, n_thr);
+    u[e] = y - cen[o.code[e]];
+    uu = fmaf(u[e], u[e], uu);
+    o.sgn[e] = 0;
+  }
+  o.norm = n;
+  o.gamma = n * sqrtf(warp_sum(uu));
+}
+
+// Split-K decode attention, one launch per call. grid (chunks, n_kv, batch),
+// kWarps warps per CTA. Each warp streams its pages (every kWarps-th page of the
+// chunk) through a private ring of kStages shared-memory stages filled by 1-D
+// bulk TMA copies; the copies are issued first thing, and the prologue (query
+// transform, and with APPEND the quantization of the new token) runs while
+// they are in flight.
 //
 // Per 16-token page a warp computes, with tokens on the rows of the products:
 //   logits  int8 m16n8k32: A = key-code limbs (hi, lo) or 0/1 sign bytes of
@@ -819,11 +676,15 @@ __device__ __forceinline__ void lds_words(const uint32_t* src, uint32_t (&dst)[N
 //   values  fp16 m16n8k16: A = value centroids (coordinates x tokens),
 //           B = softmax weights split into fp16 high parts (columns 0-3) and
 //           low parts (columns 4-7), transposed into place with shuffles.
-template <int BK, int BV, int NH>
+// APPEND: the CTA whose chunk holds a sequence's last page first quantizes
+// (k_new, v_new) of that sequence into position seq_len - 1, then fetches the
+// page.
+template <int BK, int BV, int NH, bool APPEND>
 __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
   constexpr int kSignOff = 256 * BK, kVOff = 256 * (BK + 1), kNormOff = 256 * (BK + BV + 1);
+  constexpr int kHeads = NH * kGroupHeads;
   constexpr bool kRegQ = NH <= 2;              // query fragments in registers (else shared memory)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -831,6 +692,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   const int pair = b * A.n_kv + hk;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kBlock);
+  static_assert((kWarps * kStages * kBlock + kWarps * kStages * 8) % 16 == 0, "prologue alignment");
+  Prologue<NH>& P = *reinterpret_cast<Prologue<NH>*>(bars + kWarps * kStages);
   __shared__ int s_last;
   __shared__ int s_pageok[kWarps * kStages];
   uint8_t* stage0 = smem + warp * kStages * kBlock;
@@ -843,11 +706,6 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   }
   __syncwarp();
 
-  // Reads before griddepcontrol.wait: the launch that precedes this kernel on
-  // the stream is the query transform of the same call, which writes neither
-  // the cache nor the tables; everything before it has completed. When the call
-  // also appends tokens (hold_last_page), each sequence's last page is fetched
-  // only after the wait.
   int L = A.seq_lens[b];
   if (L < 0 || L > A.max_seq_len) {
     if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_LENGTH);
@@ -858,7 +716,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   const int p1 = min(p0 + A.ppc, seq_pages);
   const int nmine = (p1 > p0 + warp) ? (p1 - p0 - warp + kWarps - 1) / kWarps : 0;
   const int32_t* btab = A.block_tables + static_cast<int64_t>(b) * A.max_pages_per_seq;
-  const int held = A.hold_last_page ? seq_pages - 1 : -1;   // logical page fetched after the wait
+  // the CTA holding the last page appends the new token before fetching that page
+  const bool appender = APPEND && L > 0 && chunk == (seq_pages - 1) / A.ppc;
+  const int held = appender ? seq_pages - 1 : -1;
 
   // Physical page ids of this warp's pages, 32 at a time: lane j holds page j of the window.
   int win = 0;
@@ -885,54 +745,193 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     }
   };
   const int n_first = min(nmine, kStages);
-  int n_early = 0;                        // stages issued before the wait, in ring order
+  int n_early = 0;                        // stages issued now, in ring order, up to the held page
   while (n_early < n_first && p0 + warp + n_early * kWarps != held) ++n_early;
   for (int k = 0; k < n_early; ++k) {
     const int phys = __shfl_sync(kFull, myphys, k);
     if (lane == 0) issue(phys, k);
   }
 
-  // The query fragments (and appended tokens) come from the preceding kernel.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-
-  for (int k = n_early; k < n_first; ++k) {
+  // ---- prologue, while the first pages are in flight
+  // sketch rows 16w .. 16w+15 as m16n8k16 A fragments (fp16 pairs, row-major [128][64])
+  uint32_t af[8][4];
+  {
+    const uint32_t* S32 = reinterpret_cast<const uint32_t*>(T.sketch);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      af[ks][0] = __ldg(S32 + (16 * warp + g) * 64 + 8 * ks + t);
+      af[ks][1] = __ldg(S32 + (16 * warp + g + 8) * 64 + 8 * ks + t);
+      af[ks][2] = __ldg(S32 + (16 * warp + g) * 64 + 8 * ks + 4 + t);
+      af[ks][3] = __ldg(S32 + (16 * warp + g + 8) * 64 + 8 * ks + 4 + t);
+    }
+  }
+  if (threadIdx.x < 16) {
+    P.tab[threadIdx.x] = T.thr_k[threadIdx.x];
+    P.tab[16 + threadIdx.x] = T.cen_k[threadIdx.x];
+    P.tab[32 + threadIdx.x] = T.thr_v[threadIdx.x];
+    P.tab[48 + threadIdx.x] = T.cen_v[threadIdx.x];
+  }
+  __syncthreads();
+  const size_t kv_row = static_cast<size_t>(b) * A.n_kv + hk;
+  const int pos = L - 1;
+  uint8_t* ablk = nullptr;                // block receiving the appended token
+  if (appender) {
+    const int phys = btab[pos / kPage];
+    if (phys >= 0 && phys < A.n_pages) ablk = A.cache + (static_cast<int64_t>(phys) * A.n_kv + hk) * kBlock;
+    else if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_SLOT);
+  }
+  // jobs: kHeads query rotations, then (appender) the key and the value of the new token
+  const int n_jobs = kHeads + (ablk ? 2 : 0);
+  for (int j = warp; j < n_jobs; j += kWarps) {
+    if (j < kHeads) {
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j < A.group) load_row4(A.q, static_cast<size_t>(b) * A.n_q + hk * A.group + j, A.q_dtype, lane, x);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] *= T.signs_k[4 * lane + e];
+      fwht128(x, lane);
+      float mx = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[e] *= kInvSqrtD;
+        P.qt[j][4 * lane + e] = x[e];
+        mx = fmaxf(mx, fabsf(x[e]));
+      }
+      mx = warp_max(mx);
+      int E = 0;
+      if (mx > 0.0f) frexpf(mx, &E);
+      if (lane == 0) P.sig[j] = 10 - E;      // fp16 high/low split near 2^10
+    } else if (j == kHeads) {
+      float x[4], u[4];
+      load_row4(A.k_new, kv_row, A.kv_dtype, lane, x);
+      VecOut o;
+      rotate_and_code(x, T.signs_k, P.tab, P.tab + 16, BK, lane, o, u);
+      float mx = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        P.u[4 * lane + e] = u[e];
+        mx = fmaxf(mx, fabsf(u[e]));
+      }
+      mx = warp_max(mx);
+      int E = 0;
+      if (mx > 0.0f) frexpf(mx, &E);
+      if (lane == 0) P.sig[kHeads] = 10 - E;
+      P.key[lane] = o;
+    } else {
+      float x[4], u[4];
+      load_row4(A.v_new, kv_row, A.kv_dtype, lane, x);
+      VecOut o;
+      rotate_and_code(x, T.signs_v, P.tab + 32, P.tab + 48, BV, lane, o, u);
+      store_value_token(ablk, pos % kPage, BK, BV, o, lane);
+      if (lane == 0) store_norm(ablk, BK, BV, 2, pos % kPage, o.norm);
+    }
+  }
+  __syncthreads();
+  // sketch products on the tensor cores: warp w owns sketch rows 16w .. 16w+15; the B
+  // columns are (head h, fp16 high part) and (head h, fp16 low part) of x * 2^sig
+  auto sketch_product = [&](const float* vec4, const int* sig4, int cols, float* out4) {
+    // vec4: column-pair sources (cols/2 vectors of 128); out4: destinations [cols/2][128]
+    const int src = g >> 1;
+    const bool has = src < cols / 2;
+    const float sc = has ? ldexpf(1.0f, sig4[src]) : 0.0f;
+    const bool lo_col = g & 1;
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
+      if (has) {
+        u0 = *reinterpret_cast<const float2*>(vec4 + src * 128 + 16 * ks + 2 * t);
+        u1 = *reinterpret_cast<const float2*>(vec4 + src * 128 + 16 * ks + 2 * t + 8);
+      }
+      const float2 v0 = make_float2(u0.x * sc, u0.y * sc), v1 = make_float2(u1.x * sc, u1.y * sc);
+      const __half2 h0 = __floats2half2_rn(v0.x, v0.y), h1 = __floats2half2_rn(v1.x, v1.y);
+      __half2 b0 = h0, b1 = h1;
+      if (lo_col) {
+        const float2 r0 = __half22float2(h0), r1 = __half22float2(h1);
+        b0 = __floats2half2_rn(v0.x - r0.x, v0.y - r0.y);
+        b1 = __floats2half2_rn(v1.x - r1.x, v1.y - r1.y);
+      }
+      mma_f16(c, af[ks][0], af[ks][1], af[ks][2], af[ks][3], *reinterpret_cast<uint32_t*>(&b0),
+              *reinterpret_cast<uint32_t*>(&b1));
+    }
+    if (t < cols / 2) {                     // columns 2t (high) and 2t+1 (low) of source t
+      const float inv = ldexpf(1.0f, -sig4[t]);
+      out4[t * 128 + 16 * warp + g] = (c[0] + c[1]) * inv;
+      out4[t * 128 + 16 * warp + g + 8] = (c[2] + c[3]) * inv;
+    }
+  };
+#pragma unroll
+  for (int h = 0; h < NH; ++h) sketch_product(&P.qt[4 * h][0], &P.sig[4 * h], 8, &P.pp[4 * h][0]);
+  if (ablk) sketch_product(P.u, &P.sig[kHeads], 2, P.z);
+  __syncthreads();
+  for (int j = warp; j < kHeads + (ablk ? 1 : 0); j += kWarps) {
+    if (j < kHeads) {
+      float x[4], pv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[e] = P.qt[j][4 * lane + e];
+        pv[e] = P.pp[j][4 * lane + e];
+      }
+      const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
+      const int ep = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(pv[0]), fabsf(pv[1])), fmaxf(fabsf(pv[2]), fabsf(pv[3])))));
+      const Limbs lq = split3(x, eq);
+      const Limbs lp = split3(pv, ep);
+      const int psum = warp_isum(lp.sum);            // |sum| < 2^29
+      uint32_t* lm = P.limb[j];                      // [which][limb][32]
+      lm[0 * 32 + lane] = lq.w0;  lm[1 * 32 + lane] = lq.w1;  lm[2 * 32 + lane] = lq.w2;
+      lm[96 + 0 * 32 + lane] = lp.w0; lm[96 + 1 * 32 + lane] = lp.w1; lm[96 + 2 * 32 + lane] = lp.w2;
+      if (lane == 0) {
+        const bool real = j < A.group;
+        P.cst[j][0] = real ? A.scale * kLog2e * ldexpf(1.0f, -eq - T.k_exp) : 0.0f;
+        P.cst[j][1] = real ? A.scale * kLog2e * kSqrtPiOver2 / kQjlRows * ldexpf(1.0f, -ep) : 0.0f;
+        P.cst[j][2] = __int_as_float(real ? psum : 0);
+      }
+    } else {                                         // the appended key: sign bits, store
+      VecOut o = P.key[lane];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o.sgn[e] = P.z[4 * lane + e] >= 0.0f ? 1 : 0;
+      store_key_token(ablk, pos % kPage, BK, o, lane);
+      if (lane == 0) {
+        store_norm(ablk, BK, BV, 0, pos % kPage, o.norm);
+        store_norm(ablk, BK, BV, 1, pos % kPage, o.gamma);
+      }
+    }
+  }
+  if (ablk) asm volatile("fence.proxy.async.global;" ::: "memory");   // the page is next read by the TMA unit
+  __syncthreads();
+  for (int k = n_early; k < n_first; ++k) {  // the held page (appender only) and what follows it
     const int phys = __shfl_sync(kFull, myphys, k);
     if (lane == 0) issue(phys, k);
   }
   __syncwarp();                           // lane 0's page flags are visible to the warp
 
-  // B fragments of lane (g, t) and the constants of head t in each group of 4
-  const uint32_t* qfr = A.qfrag + static_cast<size_t>(pair) * A.n_hg * 1024;
+  // B fragment of lane (g, t): column g -> head 4h + g/2; rows 4t.. (+16 for reg 1) of k-tile kt
+  //   n-tile 0: limb 2 (g even) or 1 (g odd); n-tile 1: limb 0 (g even) or zero (g odd)
   auto qword = [&](int h, int which, int kt, int nt, int sub) -> uint32_t {
-    return __ldg(qfr + h * 1024 + ((which * 4 + kt) * 2 + nt) * 64 + lane * 2 + sub);
+    const int limb = nt == 0 ? ((g & 1) ? 1 : 2) : 0;
+    const uint32_t v = P.limb[4 * h + (g >> 1)][which * 96 + limb * 32 + 8 * kt + 4 * sub + t];
+    return (nt == 1 && (g & 1)) ? 0u : v;
   };
   uint32_t bq[kRegQ ? NH : 1][4][2][2], bp[kRegQ ? NH : 1][4][2][2];
-  uint32_t* s_qf = reinterpret_cast<uint32_t*>(bars + kWarps * kStages);   // [NH][1024] when not in registers
   if constexpr (kRegQ) {
 #pragma unroll
     for (int h = 0; h < NH; ++h)
 #pragma unroll
       for (int kt = 0; kt < 4; ++kt)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const uint2 vq = __ldg(reinterpret_cast<const uint2*>(qfr + h * 1024 + ((0 * 4 + kt) * 2 + nt) * 64) + lane);
-          const uint2 vp = __ldg(reinterpret_cast<const uint2*>(qfr + h * 1024 + ((1 * 4 + kt) * 2 + nt) * 64) + lane);
-          bq[h][kt][nt][0] = vq.x; bq[h][kt][nt][1] = vq.y;
-          bp[h][kt][nt][0] = vp.x; bp[h][kt][nt][1] = vp.y;
-        }
-  } else {
-    const uint4* src = reinterpret_cast<const uint4*>(qfr);
-    for (int i = threadIdx.x; i < NH * 1024 / 4; i += blockDim.x) reinterpret_cast<uint4*>(s_qf)[i] = src[i];
-    __syncthreads();
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            bq[h][kt][nt][sub] = qword(h, 0, kt, nt, sub);
+            bp[h][kt][nt][sub] = qword(h, 1, kt, nt, sub);
+          }
   }
-  (void)qword;
   float ca[NH], cb[NH];
   int csum[NH];
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
-    const float4 c4 = __ldg(reinterpret_cast<const float4*>(
-        A.qconst + ((static_cast<size_t>(pair) * A.n_hg + h) * kGroupHeads + t) * 4));
-    ca[h] = c4.x; cb[h] = c4.y; csum[h] = __float_as_int(c4.z);
+    ca[h] = P.cst[4 * h + t][0];
+    cb[h] = P.cst[4 * h + t][1];
+    csum[h] = __float_as_int(P.cst[4 * h + t][2]);
   }
   uint32_t kth_[4], ktl_[4], vlo_[4], vhi_[4];
 #pragma unroll
@@ -1011,9 +1010,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
           if constexpr (kRegQ) {
             q0 = bq[h][kt][nt][0]; q1 = bq[h][kt][nt][1]; r0 = bp[h][kt][nt][0]; r1 = bp[h][kt][nt][1];
           } else {
-            const uint2 vq = reinterpret_cast<const uint2*>(s_qf + h * 1024 + ((0 * 4 + kt) * 2 + nt) * 64)[lane];
-            const uint2 vp = reinterpret_cast<const uint2*>(s_qf + h * 1024 + ((1 * 4 + kt) * 2 + nt) * 64)[lane];
-            q0 = vq.x; q1 = vq.y; r0 = vp.x; r1 = vp.y;
+            q0 = qword(h, 0, kt, nt, 0); q1 = qword(h, 0, kt, nt, 1);
+            r0 = qword(h, 1, kt, nt, 0); r1 = qword(h, 1, kt, nt, 1);
           }
           mma_s8(dh[h][nt], ah, q0, q1);
           mma_s8(dl[h][nt], al, q0, q1);
@@ -1222,52 +1220,79 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     }
     __syncthreads();
   }
+  if (threadIdx.x == 0) A.counters[pair] = 0u;    // ready for the next call
 }
 
-template <int BK, int BV, int NH>
+template <int BK, int BV, int NH, bool APPEND>
 cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
-  constexpr size_t kPro = NH > 2 ? static_cast<size_t>(NH) * 1024 * 4 : 0;   // query fragments in smem
-  const size_t pipe = static_cast<size_t>(kWarps) * kStages * kBlock + kWarps * kStages * sizeof(uint64_t) + kPro;
+  const size_t pipe = static_cast<size_t>(kWarps) * kStages * kBlock + kWarps * kStages * sizeof(uint64_t) +
+                      sizeof(Prologue<NH>);
   const size_t merge = static_cast<size_t>(kWarps) * NH * 8 * 128 * 4 + kWarps * NH * kGroupHeads * 3 * 4;
   const size_t smem = pipe > merge ? pipe : merge;
-  auto fn = decode_kernel<BK, BV, NH>;
+  auto fn = decode_kernel<BK, BV, NH, APPEND>;
   static size_t configured = 0;     // raise the shared-memory limit once per instantiation
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kWarps * 32);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fn, T, a);
+  fn<<<grid, kWarps * 32, smem, s>>>(T, a);
+  return cudaGetLastError();
 }
 
-template <int BK, int BV>
+template <int BK, int BV, bool APPEND>
 cudaError_t dispatch_nh(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   switch (a.n_hg) {
-    case 1: return launch_decode_t<BK, BV, 1>(T, a, grid, s);
-    case 2: return launch_decode_t<BK, BV, 2>(T, a, grid, s);
-    case 3: return launch_decode_t<BK, BV, 3>(T, a, grid, s);
-    default: return launch_decode_t<BK, BV, 4>(T, a, grid, s);
+    case 1: return launch_decode_t<BK, BV, 1, APPEND>(T, a, grid, s);
+    case 2: return launch_decode_t<BK, BV, 2, APPEND>(T, a, grid, s);
+    case 3: return launch_decode_t<BK, BV, 3, APPEND>(T, a, grid, s);
+    default: return launch_decode_t<BK, BV, 4, APPEND>(T, a, grid, s);
   }
 }
 
-template <int BK>
+template <int BK, bool APPEND>
 cudaError_t dispatch_bv(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   switch (T.value_bits) {
-    case 2: return dispatch_nh<BK, 2>(T, a, grid, s);
-    case 3: return dispatch_nh<BK, 3>(T, a, grid, s);
-    default: return dispatch_nh<BK, 4>(T, a, grid, s);
+    case 2: return dispatch_nh<BK, 2, APPEND>(T, a, grid, s);
+    case 3: return dispatch_nh<BK, 3, APPEND>(T, a, grid, s);
+    default: return dispatch_nh<BK, 4, APPEND>(T, a, grid, s);
   }
+}
+
+template <bool APPEND>
+cudaError_t dispatch_bk(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
+  switch (T.key_bits) {
+    case 2: return dispatch_bv<2, APPEND>(T, a, grid, s);
+    case 3: return dispatch_bv<3, APPEND>(T, a, grid, s);
+    default: return dispatch_bv<4, APPEND>(T, a, grid, s);
+  }
+}
+
+DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float scale, const void* cache,
+                       int64_t n_pages, const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
+                       int max_seq_len, float* out, void* workspace) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeArgs a{};
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.scale = scale;
+  a.cache = static_cast<uint8_t*>(const_cast<void*>(cache));
+  a.n_pages = n_pages;
+  a.block_tables = block_tables;
+  a.max_pages_per_seq = max_pages_per_seq;
+  a.seq_lens = seq_lens;
+  a.max_seq_len = max_seq_len;
+  a.partial = reinterpret_cast<float*>(ws + plan.off_partial);
+  a.counters = reinterpret_cast<unsigned*>(ws + plan.off_counter);
+  a.out = out;
+  a.n_kv = plan.n_kv;
+  a.n_q = plan.n_q;
+  a.group = plan.group;
+  a.n_hg = plan.n_hg;
+  a.chunks = plan.chunks;
+  a.ppc = plan.pages_per_chunk;
+  return a;
 }
 
 }  // namespace
@@ -1297,73 +1322,25 @@ cudaError_t launch_quantize_prefill(const Tables& t, const void* k, const void* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_common(const Tables& t, const DecodePlan& plan, const void* cache, int64_t n_pages,
-                                 const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
-                                 int max_seq_len, float* out, void* workspace, int hold_last_page,
-                                 cudaStream_t s);
+cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype,
+                          const void* cache, int64_t n_pages, const int32_t* block_tables,
+                          int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len, float scale,
+                          float* out, void* workspace, cudaStream_t s) {
+  const DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq,
+                                   seq_lens, max_seq_len, out, workspace);
+  return dispatch_bk<false>(t, a, dim3(plan.chunks, plan.n_kv, plan.batch), s);
+}
 
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, const void* q, int q_dtype, void* cache, int64_t n_pages,
                                const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
                                int max_seq_len, float scale, float* out, void* workspace, cudaStream_t s) {
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  step_prep_kernel<<<dim3(plan.n_hg + 1, plan.n_kv, plan.batch), 512, 0, s>>>(
-      t, q, q_dtype, plan.n_q, plan.n_kv, plan.group, plan.n_hg, scale,
-      reinterpret_cast<uint32_t*>(ws + plan.off_qfrag), reinterpret_cast<float*>(ws + plan.off_qconst),
-      reinterpret_cast<unsigned*>(ws + plan.off_counter), k_new,
-      v_new, kv_dtype, static_cast<uint8_t*>(cache), n_pages, block_tables, max_pages_per_seq, seq_lens);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_decode_common(t, plan, cache, n_pages, block_tables, max_pages_per_seq, seq_lens, max_seq_len,
-                              out, workspace, 1, s);
-}
-
-cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype,
-                          const void* cache, int64_t n_pages, const int32_t* block_tables,
-                          int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len, float scale,
-                          float* out, void* workspace, cudaStream_t s) {
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws + plan.off_qfrag);
-  float* qconst = reinterpret_cast<float*>(ws + plan.off_qconst);
-  qtransform_kernel<<<dim3(plan.n_hg, plan.n_kv, plan.batch), 512, 0, s>>>(
-      t, q, q_dtype, plan.n_q, plan.n_kv, plan.group, plan.n_hg, scale, qfrag, qconst,
-      reinterpret_cast<unsigned*>(ws + plan.off_counter));
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_decode_common(t, plan, cache, n_pages, block_tables, max_pages_per_seq, seq_lens, max_seq_len,
-                              out, workspace, 0, s);
-}
-
-cudaError_t launch_decode_common(const Tables& t, const DecodePlan& plan, const void* cache, int64_t n_pages,
-                                 const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
-                                 int max_seq_len, float* out, void* workspace, int hold_last_page,
-                                 cudaStream_t s) {
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  DecodeArgs a;
-  a.cache = static_cast<const uint8_t*>(cache);
-  a.n_pages = n_pages;
-  a.block_tables = block_tables;
-  a.max_pages_per_seq = max_pages_per_seq;
-  a.seq_lens = seq_lens;
-  a.max_seq_len = max_seq_len;
-  a.qfrag = reinterpret_cast<const uint32_t*>(ws + plan.off_qfrag);
-  a.qconst = reinterpret_cast<const float*>(ws + plan.off_qconst);
-  a.partial = reinterpret_cast<float*>(ws + plan.off_partial);
-  a.counters = reinterpret_cast<unsigned*>(ws + plan.off_counter);
-  a.hold_last_page = hold_last_page;
-  a.out = out;
-  a.n_kv = plan.n_kv;
-  a.n_q = plan.n_q;
-  a.group = plan.group;
-  a.n_hg = plan.n_hg;
-  a.chunks = plan.chunks;
-  a.ppc = plan.pages_per_chunk;
-  dim3 grid(plan.chunks, plan.n_kv, plan.batch);
-  switch (t.key_bits) {
-    case 2: return dispatch_bv<2>(t, a, grid, s);
-    case 3: return dispatch_bv<3>(t, a, grid, s);
-    default: return dispatch_bv<4>(t, a, grid, s);
-  }
+  DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq, seq_lens,
+                             max_seq_len, out, workspace);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.kv_dtype = kv_dtype;
+  return dispatch_bk<true>(t, a, dim3(plan.chunks, plan.n_kv, plan.batch), s);
 }
 
 }  // namespace tq

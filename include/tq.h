@@ -121,9 +121,11 @@ tq_status tq_quantize_prefill(tq_ctx* ctx, const void* k, const void* v, tq_dtyp
                               int start_pos, void* cache, int64_t n_cache_pages, tq_stream stream);
 
 /*
- * Workspace for tq_decode_attention (caller-allocated device memory, 256-byte
- * aligned). It holds the transformed queries, split-K partials and one counter
- * per (sequence, KV head); its contents need no initialisation.
+ * Workspace for tq_decode_attention / tq_decode_step (caller-allocated device
+ * memory, 256-byte aligned). It holds split-K partials and one completion
+ * counter per (sequence, KV head). Zero-fill it once before its first use
+ * (e.g. cudaMemsetAsync); every call leaves the counters at zero again. Calls
+ * that share a workspace must not run concurrently.
  */
 size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int n_q_heads, int n_kv_heads,
                                  int max_seq_len);

@@ -121,7 +121,7 @@ def _decode_case(bk, bv, seq_lens, n_kv, g, qdtype="bf16", seed=0):
     ctx = _ctx(bk, bv, seeds)
     cache = torch.from_numpy(cache_np.reshape(-1)).to(DEV)
     max_len = max(max(seq_lens), 1)
-    ws = torch.empty(ctx.decode_workspace_bytes(len(seq_lens), n_kv * g, n_kv, max_len), dtype=torch.uint8,
+    ws = torch.zeros(ctx.decode_workspace_bytes(len(seq_lens), n_kv * g, n_kv, max_len), dtype=torch.uint8,
                      device=DEV)
     out = torch.full((len(seq_lens), n_kv * g, 128), float("nan"), device=DEV)
     ctx.decode_attention(_t(q, qdtype), cache, n_pages, torch.from_numpy(bt).to(DEV),
@@ -174,7 +174,7 @@ def test_decode_fp32_query_and_tiny_workload():
     assert all(val == 0 for key, val in rep.items() if key.startswith("bad")), rep
     q = gen.queries()
     out = torch.zeros(1, 1, 128, device=DEV)
-    ws = torch.empty(ctx.decode_workspace_bytes(1, 1, 1, 1024), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(ctx.decode_workspace_bytes(1, 1, 1, 1024), dtype=torch.uint8, device=DEV)
     ctx.decode_attention(_t(q, "fp32"), cache, n_pages, btt, torch.tensor([1024], dtype=torch.int32, device=DEV),
                          1, 1024, out, ws)
     want = odec.decode_paged(host, bt, [1024], q.astype(np.float64), tab)
@@ -186,7 +186,7 @@ def test_decode_bad_page_sets_device_error():
     n_pages = 4
     cache = torch.zeros(n_pages * ctx.page_bytes(1), dtype=torch.uint8, device=DEV)
     bt = torch.tensor([[0, 99]], dtype=torch.int32, device=DEV)
-    ws = torch.empty(ctx.decode_workspace_bytes(1, 4, 1, 32), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(ctx.decode_workspace_bytes(1, 4, 1, 32), dtype=torch.uint8, device=DEV)
     out = torch.zeros(1, 4, 128, device=DEV)
     ctx.decode_attention(torch.randn(1, 4, 128, device=DEV), cache, n_pages, bt,
                          torch.tensor([32], dtype=torch.int32, device=DEV), 1, 32, out, ws)
@@ -197,7 +197,7 @@ def test_decode_bad_page_sets_device_error():
 def test_invalid_arguments_are_rejected_before_launch():
     ctx = _ctx(3, 2, (1, 2, 3))
     L = binding.lib()
-    ws = torch.empty(1024, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(1024, dtype=torch.uint8, device=DEV)
     out = torch.zeros(1, 4, 128, device=DEV)
     q = torch.zeros(1, 4, 128, device=DEV)
     bt = torch.zeros(1, 1, dtype=torch.int32, device=DEV)
@@ -225,7 +225,7 @@ def test_decode_step_attends_the_appended_token():
     cache = torch.zeros(n_pages * ctx.page_bytes(n_kv), dtype=torch.uint8, device=DEV)
     btt = torch.from_numpy(bt).to(DEV)
     ctx.quantize_prefill(_t(k[:L0], "bf16"), _t(v[:L0], "bf16"), btt[0], 0, cache, n_pages)
-    ws = torch.empty(ctx.decode_workspace_bytes(1, n_kv * g, n_kv, L0 + 3), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(ctx.decode_workspace_bytes(1, n_kv * g, n_kv, L0 + 3), dtype=torch.uint8, device=DEV)
     for step in range(3):
         L = L0 + step + 1
         slots = torch.from_numpy(synth.slots_for(bt[0], L - 1, 1)).to(DEV)
@@ -256,7 +256,7 @@ def test_decode_step_api_matches_oracle():
     for b, L in enumerate(L0):
         ctx.quantize_prefill(_t(kv[b][0][:L], "bf16"), _t(kv[b][1][:L], "bf16"), btt[b], 0, cache, n_pages)
     max_len = max(L0) + steps
-    ws = torch.empty(ctx.decode_workspace_bytes(2, n_kv * g, n_kv, max_len), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(ctx.decode_workspace_bytes(2, n_kv * g, n_kv, max_len), dtype=torch.uint8, device=DEV)
     for step in range(steps):
         lens = [L + step + 1 for L in L0]
         k_new = np.stack([kv[b][0][lens[b] - 1] for b in range(2)])
