@@ -198,7 +198,7 @@ struct tq_ctx {
   int device = 0;
   bool rot_ready = false, cb_ready = false;
   float* d_signs = nullptr;        // [2][128]: D_K then D_V
-  uint16_t* d_sketch_t = nullptr;  // [128][128] fp16 bits of S^T, then S (row-major)
+  uint16_t* d_sketch_t = nullptr;  // [128][128] fp16 bits of S^T, then S in A-fragment order
   unsigned* d_err = nullptr;
   tq::Tables tables;
 };
@@ -404,10 +404,22 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
     signs[d + i] = sv[i];
   }
   for (int r = 0; r < m; ++r)
-    for (int c = 0; c < d; ++c) {
-      st[c * m + r] = s[r * d + c];            // S^T
-      st[m * d + r * d + c] = s[r * d + c];    // S
-    }
+    for (int c = 0; c < d; ++c) st[c * m + r] = s[r * d + c];   // S^T
+  // S as m16n8k16 A fragments: warp w (rows 16w..16w+15), k-step ks (columns
+  // 16ks..16ks+15), lane (g, t), register j -> row 16w + g + 8(j&1), fp16 pair at
+  // columns 16ks + 2t + 8(j>>1) (+0, +1). Stored [w][ks][lane][j], so one warp's
+  // register set for one k-step is 512 contiguous bytes.
+  uint16_t* frag = st.data() + m * d;
+  for (int w = 0; w < m / 16; ++w)
+    for (int ks = 0; ks < d / 16; ++ks)
+      for (int lane = 0; lane < 32; ++lane)
+        for (int j = 0; j < 4; ++j) {
+          const int row = 16 * w + (lane >> 2) + 8 * (j & 1);
+          const int col = 16 * ks + 2 * (lane & 3) + 8 * (j >> 1);
+          const int o = (((w * (d / 16) + ks) * 32 + lane) * 4 + j) * 2;
+          frag[o] = s[row * d + col];
+          frag[o + 1] = s[row * d + col + 1];
+        }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // Synchronous copies from pageable memory: this is the cold set-up path.
   cudaError_t e = cudaMemcpyAsync(ctx->d_signs, signs.data(), 2 * d * sizeof(float),

@@ -409,11 +409,21 @@ __global__ void __launch_bounds__(256) quantize_prefill_kernel(Tables T, const v
 // a = scale log2(e) 2^(-e_q - k_exp), b = scale log2(e) sqrt(pi/2)/m 2^(-e_p).
 constexpr int kGroupHeads = 4;
 
+// Powers of two built from the IEEE-754 exponent field (exact).
+// pow2i(n) = 2^n for -149 <= n <= 127 (n is clamped to that range).
+__device__ __forceinline__ float pow2i(int n) {
+  n = min(max(n, -149), 127);
+  return n >= -126 ? __uint_as_float(static_cast<unsigned>(n + 127) << 23)
+                   : __uint_as_float(static_cast<unsigned>(n + 127 + 64) << 23) * 5.421010862427522e-20f;  // 2^-64
+}
+// E with x < 2^E for finite x > 0 (the exponent frexp returns, for normal x).
+__device__ __forceinline__ int exp_above(float x) {
+  return static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 126;
+}
+
 __device__ __forceinline__ int pick_exponent24(float maxabs) {
   if (!(maxabs > 0.0f)) return 0;
-  int E;
-  frexpf(maxabs, &E);               // maxabs < 2^E
-  return 22 - E;                    // maxabs * 2^e < 2^22
+  return min(22 - exp_above(maxabs), 127);   // maxabs * 2^e < 2^22
 }
 
 struct Limbs { uint32_t w2, w1, w0; int sum; };
@@ -422,7 +432,7 @@ __device__ __forceinline__ Limbs split3(const float (&x)[4], int e) {
   Limbs r{0u, 0u, 0u, 0};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int Q = __float2int_rn(ldexpf(x[i], e));
+    const int Q = __float2int_rn(x[i] * pow2i(e));
     const int q0 = ((Q + 128) & 255) - 128;
     const int r1 = (Q - q0) >> 8;
     const int q1 = ((r1 + 128) & 255) - 128;
@@ -615,6 +625,7 @@ struct DecodeArgs {
   unsigned* counters;            // [pair]: finished CTAs; zero between calls
   float* out;                    // [batch][n_q][128]
   int n_kv, n_q, group, n_hg, chunks, ppc;
+  int merge_cap;                 // chunk records that fit in shared memory for the final merge
 };
 
 // Shared-memory scratch of the prologue (after the stages and barriers).
@@ -635,14 +646,14 @@ static_assert(offsetof(Prologue<1>, u) % 16 == 0 && offsetof(Prologue<3>, u) % 1
 
 // Rotate and code one vector held 4 per lane; returns codes in o, n and (keys) gamma,
 // and the residual u = y - c[code] per lane.
-__device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float* signs, const float* thr,
+__device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float4 sg, const float* thr,
                                                 const float* cen, int bits, int lane, VecOut& o, float (&u)[4]) {
   float v[4];
   float ss = 0.0f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     ss = fmaf(x[e], x[e], ss);
-    v[e] = x[e] * signs[4 * lane + e];
+    v[e] = x[e] * (&sg.x)[e];
   }
   ss = warp_sum(ss);
   const float n = sqrtf(ss);
@@ -700,6 +711,35 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   uint64_t* mybar = bars + warp * kStages;
   int* myok = s_pageok + warp * kStages;
 
+  // The prologue's own loads go out first, ahead of the page stream, so that they
+  // do not queue behind it: this warp's sketch rows as m16n8k16 A fragments and
+  // the input of its first job (query head `warp`, or the new key / value).
+  uint4 afv[8];
+  {
+    const uint4* F = reinterpret_cast<const uint4*>(T.sketch) + warp * 8 * 32 + lane;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) afv[ks] = __ldg(F + ks * 32);
+  }
+  const size_t kv_row = static_cast<size_t>(b) * A.n_kv + hk;
+  auto job_input = [&](int j, float (&x)[4]) {
+    x[0] = x[1] = x[2] = x[3] = 0.0f;
+    if (j < kHeads) {
+      if (j < A.group) load_row4(A.q, static_cast<size_t>(b) * A.n_q + hk * A.group + j, A.q_dtype, lane, x);
+    } else if (APPEND && j < kHeads + 2) {
+      load_row4(j == kHeads ? A.k_new : A.v_new, kv_row, A.kv_dtype, lane, x);
+    }
+  };
+  float xin[4];
+  job_input(warp, xin);
+  const float4 sgk = __ldg(reinterpret_cast<const float4*>(T.signs_k) + lane);
+  const float4 sgv = __ldg(reinterpret_cast<const float4*>(T.signs_v) + lane);
+  // this warp's first 32 block-table entries, fetched before the length is known
+  // (bounded by the table width; entries past the sequence are discarded below)
+  const int32_t* btab = A.block_tables + static_cast<int64_t>(b) * A.max_pages_per_seq;
+  const int p0 = chunk * A.ppc;
+  const int first_j = p0 + warp + lane * kWarps;
+  const int spec_phys = first_j < A.max_pages_per_seq ? __ldg(btab + first_j) : -1;
+
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(mybar + s, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -712,17 +752,15 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     L = L < 0 ? 0 : A.max_seq_len;
   }
   const int seq_pages = (L + kPage - 1) / kPage;
-  const int p0 = chunk * A.ppc;
   const int p1 = min(p0 + A.ppc, seq_pages);
   const int nmine = (p1 > p0 + warp) ? (p1 - p0 - warp + kWarps - 1) / kWarps : 0;
-  const int32_t* btab = A.block_tables + static_cast<int64_t>(b) * A.max_pages_per_seq;
   // the CTA holding the last page appends the new token before fetching that page
   const bool appender = APPEND && L > 0 && chunk == (seq_pages - 1) / A.ppc;
   const int held = appender ? seq_pages - 1 : -1;
 
   // Physical page ids of this warp's pages, 32 at a time: lane j holds page j of the window.
   int win = 0;
-  int myphys = lane < nmine ? btab[p0 + warp + lane * kWarps] : -1;
+  int myphys = lane < nmine ? spec_phys : -1;
   auto page_id = [&](int kth) {           // all lanes (shuffle); reloads the window when needed
     if ((kth >> 5) != win) {
       win = kth >> 5;
@@ -753,18 +791,6 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   }
 
   // ---- prologue, while the first pages are in flight
-  // sketch rows 16w .. 16w+15 as m16n8k16 A fragments (fp16 pairs, row-major [128][64])
-  uint32_t af[8][4];
-  {
-    const uint32_t* S32 = reinterpret_cast<const uint32_t*>(T.sketch);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      af[ks][0] = __ldg(S32 + (16 * warp + g) * 64 + 8 * ks + t);
-      af[ks][1] = __ldg(S32 + (16 * warp + g + 8) * 64 + 8 * ks + t);
-      af[ks][2] = __ldg(S32 + (16 * warp + g) * 64 + 8 * ks + 4 + t);
-      af[ks][3] = __ldg(S32 + (16 * warp + g + 8) * 64 + 8 * ks + 4 + t);
-    }
-  }
   if (threadIdx.x < 16) {
     P.tab[threadIdx.x] = T.thr_k[threadIdx.x];
     P.tab[16 + threadIdx.x] = T.cen_k[threadIdx.x];
@@ -772,7 +798,6 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     P.tab[48 + threadIdx.x] = T.cen_v[threadIdx.x];
   }
   __syncthreads();
-  const size_t kv_row = static_cast<size_t>(b) * A.n_kv + hk;
   const int pos = L - 1;
   uint8_t* ablk = nullptr;                // block receiving the appended token
   if (appender) {
@@ -783,11 +808,16 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   // jobs: kHeads query rotations, then (appender) the key and the value of the new token
   const int n_jobs = kHeads + (ablk ? 2 : 0);
   for (int j = warp; j < n_jobs; j += kWarps) {
-    if (j < kHeads) {
-      float x[4] = {0.f, 0.f, 0.f, 0.f};
-      if (j < A.group) load_row4(A.q, static_cast<size_t>(b) * A.n_q + hk * A.group + j, A.q_dtype, lane, x);
+    float x[4];
+    if (j == warp) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] *= T.signs_k[4 * lane + e];
+      for (int e = 0; e < 4; ++e) x[e] = xin[e];
+    } else {
+      job_input(j, x);
+    }
+    if (j < kHeads) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] *= (&sgk.x)[e];
       fwht128(x, lane);
       float mx = 0.0f;
 #pragma unroll
@@ -798,13 +828,12 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
       }
       mx = warp_max(mx);
       int E = 0;
-      if (mx > 0.0f) frexpf(mx, &E);
+      if (mx > 0.0f) E = max(exp_above(mx), -115);   // 2^(10-E) stays a normal float
       if (lane == 0) P.sig[j] = 10 - E;      // fp16 high/low split near 2^10
     } else if (j == kHeads) {
-      float x[4], u[4];
-      load_row4(A.k_new, kv_row, A.kv_dtype, lane, x);
+      float u[4];
       VecOut o;
-      rotate_and_code(x, T.signs_k, P.tab, P.tab + 16, BK, lane, o, u);
+      rotate_and_code(x, sgk, P.tab, P.tab + 16, BK, lane, o, u);
       float mx = 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -813,14 +842,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
       }
       mx = warp_max(mx);
       int E = 0;
-      if (mx > 0.0f) frexpf(mx, &E);
+      if (mx > 0.0f) E = max(exp_above(mx), -115);   // 2^(10-E) stays a normal float
       if (lane == 0) P.sig[kHeads] = 10 - E;
       P.key[lane] = o;
     } else {
-      float x[4], u[4];
-      load_row4(A.v_new, kv_row, A.kv_dtype, lane, x);
+      float u[4];
       VecOut o;
-      rotate_and_code(x, T.signs_v, P.tab + 32, P.tab + 48, BV, lane, o, u);
+      rotate_and_code(x, sgv, P.tab + 32, P.tab + 48, BV, lane, o, u);
       store_value_token(ablk, pos % kPage, BK, BV, o, lane);
       if (lane == 0) store_norm(ablk, BK, BV, 2, pos % kPage, o.norm);
     }
@@ -832,7 +860,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     // vec4: column-pair sources (cols/2 vectors of 128); out4: destinations [cols/2][128]
     const int src = g >> 1;
     const bool has = src < cols / 2;
-    const float sc = has ? ldexpf(1.0f, sig4[src]) : 0.0f;
+    const float sc = has ? pow2i(sig4[src]) : 0.0f;
     const bool lo_col = g & 1;
     float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -850,11 +878,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
         b0 = __floats2half2_rn(v0.x - r0.x, v0.y - r0.y);
         b1 = __floats2half2_rn(v1.x - r1.x, v1.y - r1.y);
       }
-      mma_f16(c, af[ks][0], af[ks][1], af[ks][2], af[ks][3], *reinterpret_cast<uint32_t*>(&b0),
+      mma_f16(c, afv[ks].x, afv[ks].y, afv[ks].z, afv[ks].w, *reinterpret_cast<uint32_t*>(&b0),
               *reinterpret_cast<uint32_t*>(&b1));
     }
     if (t < cols / 2) {                     // columns 2t (high) and 2t+1 (low) of source t
-      const float inv = ldexpf(1.0f, -sig4[t]);
+      const float inv = pow2i(-sig4[t]);
       out4[t * 128 + 16 * warp + g] = (c[0] + c[1]) * inv;
       out4[t * 128 + 16 * warp + g + 8] = (c[2] + c[3]) * inv;
     }
@@ -881,8 +909,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
       lm[96 + 0 * 32 + lane] = lp.w0; lm[96 + 1 * 32 + lane] = lp.w1; lm[96 + 2 * 32 + lane] = lp.w2;
       if (lane == 0) {
         const bool real = j < A.group;
-        P.cst[j][0] = real ? A.scale * kLog2e * ldexpf(1.0f, -eq - T.k_exp) : 0.0f;
-        P.cst[j][1] = real ? A.scale * kLog2e * kSqrtPiOver2 / kQjlRows * ldexpf(1.0f, -ep) : 0.0f;
+        P.cst[j][0] = real ? A.scale * kLog2e * pow2i(-eq - T.k_exp) : 0.0f;
+        P.cst[j][1] = real ? A.scale * kLog2e * kSqrtPiOver2 / kQjlRows * pow2i(-ep) : 0.0f;
         P.cst[j][2] = __int_as_float(real ? psum : 0);
       }
     } else {                                         // the appended key: sign bits, store
@@ -1171,56 +1199,98 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (threadIdx.x == 0) A.counters[pair] = 0u;    // every CTA has counted: ready for the next call
 
-  // ---- last CTA of this (sequence, KV head): merge chunks, de-rotate, store.
-  // Warp w takes head slot w % 4 (+4 per round) and every second chunk from
-  // w / 4; the two halves meet in shared memory.
-  const float* pbase = A.partial + static_cast<size_t>(pair) * A.chunks * NH * kGroupHeads * 132;
-  float* s_mrg = reinterpret_cast<float*>(smem);            // [2 halves][4 slots][132]
-  for (int base = 0; base < A.group; base += kGroupHeads) {
-    const int slot = base + (warp & 3), half = warp >> 2;
-    float M = kNegBig, l = 0.0f;
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
-    if (slot < A.group) {
-      for (int c = half + 2 * lane; c < A.chunks; c += 64)
-        M = fmaxf(M, __ldcg(pbase + (static_cast<size_t>(c) * NH * kGroupHeads + slot) * 132 + 128));
-      M = warp_max(M);
+  // ---- last CTA of this (sequence, KV head): merge the chunks, de-rotate, store.
+  // The chunk records (written by the other CTAs, published by the counter) come
+  // into shared memory by bulk copies, merge_cap chunks at a time. Warp w merges
+  // head slots w % 4 (+4, +8, ...) over the chunks of parity w / 4 with an online
+  // maximum; the two parities meet in shared memory.
+  constexpr int kRec = 132;                                  // floats per (chunk, head slot) record
+  constexpr int kSlots = NH * kGroupHeads;
+  const unsigned chunk_bytes = kSlots * kRec * 4;
+  const float* pbase = A.partial + static_cast<size_t>(pair) * A.chunks * kSlots * kRec;
+  float* s_part = reinterpret_cast<float*>(smem);            // [merge_cap][kSlots][kRec]
+  float* s_mrg = s_part + static_cast<size_t>(A.merge_cap) * kSlots * kRec;   // [2][kSlots][kRec]
+  uint64_t* fbar = reinterpret_cast<uint64_t*>(s_mrg + 2 * kSlots * kRec);
+  const float4 sv = __ldg(reinterpret_cast<const float4*>(T.signs_v) + lane);
+  if (threadIdx.x == 0) {
+    mbar_init(fbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const int half = warp / kGroupHeads, sl0 = warp % kGroupHeads;
+  float M[NH], l[NH], a[NH][4];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    M[h] = kNegBig; l[h] = 0.0f;
+    a[h][0] = a[h][1] = a[h][2] = a[h][3] = 0.0f;
+  }
+  bool landed = true;
+  unsigned ph = 0;
+  for (int c0 = 0; c0 < A.chunks; c0 += A.merge_cap, ph ^= 1u) {
+    const int nc = min(A.merge_cap, A.chunks - c0);
+    if (threadIdx.x == 0) {
+      // generic-proxy writes of the other CTAs, read next by the bulk-copy unit
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      mbar_expect_tx(fbar, nc * chunk_bytes);
+      tma_load_1d(s_part, pbase + static_cast<size_t>(c0) * kSlots * kRec, nc * chunk_bytes, fbar);
+    }
+    if (!mbar_wait(fbar, ph)) {
+      if (threadIdx.x == 0) set_error(T.err, TQ_DEV_TIMEOUT);
+      landed = false;
+      break;
+    }
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      const int slot = sl0 + kGroupHeads * h;
+      if (slot >= A.group) continue;
 #pragma unroll 4
-      for (int c = half; c < A.chunks; c += 2) {
-        const float* pc = pbase + (static_cast<size_t>(c) * NH * kGroupHeads + slot) * 132;
-        const float wc = ex2(__ldcg(pc + 128) - M);
-        l = fmaf(__ldcg(pc + 129), wc, l);
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(pc) + lane);
-        a[0] = fmaf(v.x, wc, a[0]); a[1] = fmaf(v.y, wc, a[1]);
-        a[2] = fmaf(v.z, wc, a[2]); a[3] = fmaf(v.w, wc, a[3]);
+      for (int c = half; c < nc; c += 2) {
+        const float* rec = s_part + (c * kSlots + slot) * kRec;
+        const float Mc = rec[128];
+        const float Mn = fmaxf(M[h], Mc);
+        const float fo = ex2(M[h] - Mn), fc = ex2(Mc - Mn);
+        const float4 v = reinterpret_cast<const float4*>(rec)[lane];
+        l[h] = fmaf(l[h], fo, rec[129] * fc);
+        a[h][0] = fmaf(a[h][0], fo, v.x * fc); a[h][1] = fmaf(a[h][1], fo, v.y * fc);
+        a[h][2] = fmaf(a[h][2], fo, v.z * fc); a[h][3] = fmaf(a[h][3], fo, v.w * fc);
+        M[h] = Mn;
       }
     }
-    float* mine = s_mrg + (half * 4 + (warp & 3)) * 132;
-    reinterpret_cast<float4*>(mine)[lane] = make_float4(a[0], a[1], a[2], a[3]);
-    if (lane == 0) { mine[128] = M; mine[129] = l; }
-    __syncthreads();
-    if (half == 0 && slot < A.group) {
-      const float* other = s_mrg + (4 + (warp & 3)) * 132;
-      const float Mo = other[128];
-      const float Mx = fmaxf(M, Mo);
-      const float f0 = ex2(M - Mx), f1 = ex2(Mo - Mx);
-      const float lt = l * f0 + other[129] * f1;
-      const float4 ao = reinterpret_cast<const float4*>(other)[lane];
-      const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-      a[0] = (a[0] * f0 + ao.x * f1) * inv; a[1] = (a[1] * f0 + ao.y * f1) * inv;
-      a[2] = (a[2] * f0 + ao.z * f1) * inv; a[3] = (a[3] * f0 + ao.w * f1) * inv;
-      fwht128(a, lane);
-      float4 o;
-      o.x = a[0] * T.signs_v[4 * lane + 0] * kInvSqrtD;
-      o.y = a[1] * T.signs_v[4 * lane + 1] * kInvSqrtD;
-      o.z = a[2] * T.signs_v[4 * lane + 2] * kInvSqrtD;
-      o.w = a[3] * T.signs_v[4 * lane + 3] * kInvSqrtD;
-      const int qh = hk * A.group + slot;
-      reinterpret_cast<float4*>(A.out + (static_cast<size_t>(b) * A.n_q + qh) * 128)[lane] = o;
-    }
-    __syncthreads();
+    __syncthreads();                                          // s_part is free for the next piece
   }
-  if (threadIdx.x == 0) A.counters[pair] = 0u;    // ready for the next call
+  if (!landed) {
+    mbar_wait(fbar, ph);                                      // bounded: let the copy land before exit
+    return;
+  }
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    const int slot = sl0 + kGroupHeads * h;
+    float* mine = s_mrg + (half * kSlots + slot) * kRec;
+    reinterpret_cast<float4*>(mine)[lane] = make_float4(a[h][0], a[h][1], a[h][2], a[h][3]);
+    if (lane == 0) { mine[128] = M[h]; mine[129] = l[h]; }
+  }
+  __syncthreads();
+  for (int slot = warp; slot < A.group; slot += kWarps) {
+    const float* r0 = s_mrg + slot * kRec;
+    const float* r1 = s_mrg + (kSlots + slot) * kRec;
+    const float Mx = fmaxf(r0[128], r1[128]);
+    const float f0 = ex2(r0[128] - Mx), f1 = ex2(r1[128] - Mx);
+    const float lt = r0[129] * f0 + r1[129] * f1;
+    const float4 x0 = reinterpret_cast<const float4*>(r0)[lane], x1 = reinterpret_cast<const float4*>(r1)[lane];
+    const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+    float v[4] = {(x0.x * f0 + x1.x * f1) * inv, (x0.y * f0 + x1.y * f1) * inv,
+                  (x0.z * f0 + x1.z * f1) * inv, (x0.w * f0 + x1.w * f1) * inv};
+    fwht128(v, lane);
+    float4 o;
+    o.x = v[0] * sv.x * kInvSqrtD;
+    o.y = v[1] * sv.y * kInvSqrtD;
+    o.z = v[2] * sv.z * kInvSqrtD;
+    o.w = v[3] * sv.w * kInvSqrtD;
+    const int qh = hk * A.group + slot;
+    reinterpret_cast<float4*>(A.out + (static_cast<size_t>(b) * A.n_q + qh) * 128)[lane] = o;
+  }
 }
 
 template <int BK, int BV, int NH, bool APPEND>
@@ -1230,6 +1300,11 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
                       sizeof(Prologue<NH>);
   const size_t merge = static_cast<size_t>(kWarps) * NH * 8 * 128 * 4 + kWarps * NH * kGroupHeads * 3 * 4;
   const size_t smem = pipe > merge ? pipe : merge;
+  // final merge: chunk records, then [2][slots][132] floats and one barrier
+  const size_t chunk_bytes = static_cast<size_t>(NH) * kGroupHeads * 132 * 4;
+  DecodeArgs args = a;
+  args.merge_cap = static_cast<int>((smem - 2 * chunk_bytes - 16) / chunk_bytes);
+  if (args.merge_cap < 1) return cudaErrorInvalidConfiguration;
   auto fn = decode_kernel<BK, BV, NH, APPEND>;
   static size_t configured = 0;     // raise the shared-memory limit once per instantiation
   if (configured < smem) {
@@ -1237,7 +1312,7 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  fn<<<grid, kWarps * 32, smem, s>>>(T, a);
+  fn<<<grid, kWarps * 32, smem, s>>>(T, args);
   return cudaGetLastError();
 }
 
