@@ -45,6 +45,9 @@ _SIGS = {
                                   _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int, _c.c_int,
                                   _c.c_int, _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p, _c.c_size_t,
                                   _c.c_void_p]),
+    "tq_decode_attention_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int64,
+                                               _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int,
+                                               _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p]),
     "tq_get_device_error": (_c.c_int, [_c.c_void_p, _c.POINTER(_c.c_uint32), _c.c_void_p]),
     "tq_host_sign_vector": (_c.c_int, [_c.c_uint64, _c.c_int, _c.c_void_p]),
     "tq_host_gaussian_sketch": (_c.c_int, [_c.c_uint64, _c.c_int, _c.c_int, _c.c_void_p]),
@@ -179,6 +182,15 @@ class Context:
             self._h, _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(q), _dtype_code(q), _ptr(cache),
             n_cache_pages, _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), batch, n_q, n_kv_heads,
             max_seq_len, scale, _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream)))
+
+    def decode_attention_noalloc(self, q, cache, n_cache_pages: int, block_tables, seq_lens, n_kv_heads: int,
+                                 max_seq_len: int, out, scale: float = 0.0, stream=None):
+        """decode_attention with the library's fixed per-device scratch instead of a workspace."""
+        batch, n_q = q.shape[0], q.shape[1]
+        _check("tq_decode_attention_noalloc", lib().tq_decode_attention_noalloc(
+            self._h, _ptr(q), _dtype_code(q), _ptr(cache), n_cache_pages, _ptr(block_tables),
+            block_tables.shape[1], _ptr(seq_lens), batch, n_q, n_kv_heads, max_seq_len, scale, _ptr(out),
             _stream(stream)))
 
     def device_error(self, stream=None) -> int:

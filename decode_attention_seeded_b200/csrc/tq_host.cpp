@@ -564,6 +564,38 @@ tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_d
                                           scale, out, workspace, static_cast<cudaStream_t>(stream)));
 }
 
+tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
+                                      int64_t n_cache_pages, const int32_t* block_tables,
+                                      int max_pages_per_seq, const int32_t* seq_lens, int batch,
+                                      int n_q_heads, int n_kv_heads, int max_seq_len, float scale,
+                                      float* out, tq_stream stream) {
+  if (!ctx) return TQ_ERR_INVALID_ARG;
+  if (tq_status st = check_device(ctx)) return st;
+  // The scratch address is looked up once per device and kept for the process.
+  static std::mutex mu;
+  static std::map<int, void*> scratch_of_device;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = scratch_of_device.find(ctx->device);
+    if (it != scratch_of_device.end()) {
+      scratch = it->second;
+    } else {
+      if (tq::noalloc_scratch(&scratch) != cudaSuccess || !scratch) return TQ_ERR_CUDA;
+      scratch_of_device[ctx->device] = scratch;
+    }
+  }
+  tq::DecodePlan plan;
+  if (tq_status st = check_decode_args(ctx, q, q_dtype, cache, n_cache_pages, block_tables, max_pages_per_seq,
+                                       seq_lens, batch, n_q_heads, n_kv_heads, max_seq_len, scale, out,
+                                       scratch, tq::kNoAllocScratchBytes, &plan))
+    return st;   // TQ_ERR_WORKSPACE: the call needs more than the fixed scratch holds
+  if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
+  return from_cuda(tq::launch_decode(ctx->tables, plan, q, q_dtype, cache, n_cache_pages,
+                                     block_tables, max_pages_per_seq, seq_lens, max_seq_len,
+                                     scale, out, scratch, static_cast<cudaStream_t>(stream)));
+}
+
 tq_status tq_get_device_error(tq_ctx* ctx, uint32_t* code, tq_stream stream) {
   if (!ctx || !code) return TQ_ERR_INVALID_ARG;
   if (tq_status st = check_device(ctx)) return st;

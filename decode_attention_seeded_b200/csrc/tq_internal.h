@@ -58,4 +58,9 @@ cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const vo
                                const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
                                int max_seq_len, float scale, float* out, void* workspace, cudaStream_t s);
 
+// Device address (current device) of the fixed decode scratch used by
+// tq_decode_attention_noalloc; kNoAllocScratchBytes bytes, 256-byte aligned.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+cudaError_t noalloc_scratch(void** ptr);
+
 }  // namespace tq

@@ -1344,6 +1344,12 @@ cudaError_t dispatch_bk(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStr
   }
 }
 
+// ---- fixed scratch for callers that cannot allocate device memory ----------
+// Split-K records and completion counters of tq_decode_attention_noalloc. One
+// copy per device, zero when the module is loaded; every decode that runs to the
+// end leaves the counters at zero again.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float scale, const void* cache,
                        int64_t n_pages, const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
                        int max_seq_len, float* out, void* workspace) {
@@ -1371,6 +1377,8 @@ DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float
 }
 
 }  // namespace
+
+cudaError_t noalloc_scratch(void** ptr) { return cudaGetSymbolAddress(ptr, g_noalloc_scratch); }
 
 cudaError_t launch_quantize_append(const Tables& t, const void* k, const void* v, int dtype, int n_tokens,
                                    int n_kv, const int64_t* slots, void* cache, int64_t n_pages,

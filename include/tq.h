@@ -169,6 +169,43 @@ tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_d
                          int batch, int n_q_heads, int n_kv_heads, int max_seq_len, float scale, float* out,
                          void* workspace, size_t workspace_bytes, tq_stream stream);
 
+/*
+ * tq_decode_attention without a caller workspace. The pages have no counterpart
+ * to this call: it is a library convenience, computing exactly what
+ * tq_decode_attention computes, with the same arguments minus the workspace.
+ *
+ * Who needs it: callers that cannot hand the library device memory of their
+ * own -- a host program that reaches the GPU only through this C ABI and has no
+ * CUDA allocator binding, a runtime that has reserved its whole device budget
+ * in a pool it does not lend out, or a decode path where an allocation that
+ * can fail or stall is not acceptable. Instead of a workspace, the call uses a
+ * fixed scratch array compiled into libtq.so: 4 MiB (4194304 bytes) per device,
+ * 256-byte aligned, allocated when the library's device code is loaded. It
+ * allocates nothing, itself or through any library routine.
+ *
+ * Size limit: the call needs tq_decode_workspace_bytes(ctx, batch, n_q_heads,
+ * n_kv_heads, max_seq_len) bytes of scratch; above 4194304 it returns
+ * TQ_ERR_WORKSPACE and enqueues nothing (use tq_decode_attention then).
+ *
+ * State: the scratch's completion counters must be zero when a call starts.
+ * They are zero when the device code is loaded, and every call that runs to
+ * the end -- including one that records a device error -- leaves them at zero.
+ * The scratch is shared by every context of the process on that device, so
+ * calls on one device must not overlap: issue them on one stream, or order
+ * them with events. Two calls in flight at once race on the scratch and give
+ * wrong results.
+ *
+ * First call: the first call on a device looks up the scratch's device
+ * address (cudaGetSymbolAddress), which may load the library's device code on
+ * that device. Make that first call before any stream capture begins; later
+ * calls only enqueue the kernel.
+ */
+tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
+                                      int64_t n_cache_pages, const int32_t* block_tables,
+                                      int max_pages_per_seq, const int32_t* seq_lens, int batch,
+                                      int n_q_heads, int n_kv_heads, int max_seq_len, float scale,
+                                      float* out, tq_stream stream);
+
 /* Synchronise `stream`, then read and clear the device error word (TQ_DEV_* bits). */
 tq_status tq_get_device_error(tq_ctx* ctx, uint32_t* code, tq_stream stream);
 
