@@ -196,6 +196,7 @@ StoredCodebook make_codebook(int bits, int d) {
 // ====================================================================== context
 struct tq_ctx {
   int device = 0;
+  int sm_count = 0;                // streaming multiprocessors of the device (sizes decode grids)
   bool rot_ready = false, cb_ready = false;
   float* d_signs = nullptr;        // [2][128]: D_K then D_V
   uint16_t* d_sketch_t = nullptr;  // [128][128] fp16 bits of S^T, then S in A-fragment order
@@ -276,8 +277,7 @@ tq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CU
 
 namespace tq {
 
-DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int block_bytes) {
-  (void)block_bytes;
+DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int sm_count) {
   DecodePlan p{};
   p.batch = batch;
   p.n_q = n_q;
@@ -286,10 +286,13 @@ DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int block_by
   p.n_hg = (p.group + 3) / 4;                    // groups of 4 query heads
   p.max_pages = std::max(1, (max_seq_len + kPage - 1) / kPage);
   const int pairs = batch * n_kv;
-  const int target_ctas = 148 * 2;               // two resident CTAs of 8 warps per SM
-  int chunks = std::max(1, (target_ctas + pairs - 1) / pairs);
+  p.n_pairs = pairs;
+  // One resident CTA per SM: split each (sequence, KV head) into as many chunks
+  // as keep every SM busy in one wave, each chunk at least kMinChunkPages pages
+  // and at most kMaxChunkPages (its block-table window is cached in shared memory).
+  int chunks = std::max(1, sm_count / pairs);
   int ppc = (p.max_pages + chunks - 1) / chunks;
-  ppc = std::max(ppc, 16);                        // at least two pages per warp
+  ppc = std::min(std::max(ppc, kMinChunkPages), kMaxChunkPages);
   p.pages_per_chunk = ppc;
   p.chunks = (p.max_pages + ppc - 1) / ppc;
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
@@ -360,7 +363,9 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   DeviceGuard guard(device);
   tq_ctx* c = new tq_ctx;
   c->device = device;
-  cudaError_t e = cudaMalloc(&c->d_signs, 2 * tq::kHeadDim * sizeof(float));
+  cudaError_t e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, device);
+  if (e == cudaSuccess && c->sm_count <= 0) e = cudaErrorInvalidDevice;
+  if (e == cudaSuccess) e = cudaMalloc(&c->d_signs, 2 * tq::kHeadDim * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 2 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
   if (e == cudaSuccess) e = cudaMalloc(&c->d_err, sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(unsigned));
@@ -500,7 +505,7 @@ size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int n_q_heads, in
   if (!ctx || batch <= 0 || n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads ||
       max_seq_len < 0)
     return 0;
-  return tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len, 0).total;
+  return tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len, ctx->sm_count).total;
 }
 
 static tq_status check_decode_args(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
@@ -521,7 +526,7 @@ static tq_status check_decode_args(tq_ctx* ctx, const void* q, tq_dtype q_dtype,
   const size_t es = q_dtype == TQ_F32 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(q) % (4 * es)) return TQ_ERR_INVALID_ARG;
   if (!(scale >= 0.0f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
-  *plan = tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len, ctx->tables.block_bytes);
+  *plan = tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len, ctx->sm_count);
   if (workspace_bytes < plan->total || reinterpret_cast<uintptr_t>(workspace) % 256) return TQ_ERR_WORKSPACE;
   return check_device(ctx);
 }

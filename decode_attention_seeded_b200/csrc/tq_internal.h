@@ -34,13 +34,18 @@ struct Tables {
 };
 
 // Workspace carve-up for one decode call; all offsets in bytes, 256-aligned.
+// Decode grid: one CTA per (chunk, sequence x KV head pair), CTA index =
+// chunk * n_pairs + pair, one resident CTA per SM.
+constexpr int kMinChunkPages = 16;
+constexpr int kMaxChunkPages = 8192;
 struct DecodePlan {
   int batch, n_q, n_kv, group, n_hg;  // n_hg = ceil(group / 4) groups of 4 query heads
+  int n_pairs;                         // batch * n_kv
   int max_pages, pages_per_chunk, chunks;
   size_t off_partial, off_counter, total;
 };
 
-DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int block_bytes);
+DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int sm_count);
 
 cudaError_t launch_quantize_append(const Tables& t, const void* k, const void* v, int dtype,
                                    int n_tokens, int n_kv, const int64_t* slots, void* cache,

@@ -452,9 +452,13 @@ __device__ __forceinline__ int warp_isum(int v) {
 }
 
 // ================================================================== decode
-constexpr int kWarps = 8;        // compute warps per CTA
-constexpr int kStages = 6;       // TMA stages per warp
-static_assert(kWarps == 8, "the chunk merge pairs warps w and w + 4");
+// Warps per decode CTA: 16 when a CTA serves one group of 4 query heads (the
+// kernel then fits 128 registers), else 8; either way one CTA per SM.
+template <int NH>
+struct DecodeWarps { static constexpr int value = NH == 1 ? 16 : 8; };
+// TMA stages per warp: six when they fit in 160 KB of shared memory, else four.
+__host__ __device__ constexpr int decode_stages(int warps, int block) { return warps * 6 * block <= 160 * 1024 ? 6 : 4; }
+constexpr int kStatic = 2;       // pages per warp assigned before the block-table window is cached
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -624,7 +628,7 @@ struct DecodeArgs {
   float* partial;                // [pair][chunk][hg][4 heads][132]
   unsigned* counters;            // [pair]: finished CTAs; zero between calls
   float* out;                    // [batch][n_q][128]
-  int n_kv, n_q, group, n_hg, chunks, ppc;
+  int n_kv, n_q, group, n_hg, chunks, ppc, n_pairs;
   int merge_cap;                 // chunk records that fit in shared memory for the final merge
 };
 
@@ -673,12 +677,16 @@ __device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float
   o.gamma = n * sqrtf(warp_sum(uu));
 }
 
-// Split-K decode attention, one launch per call. grid (chunks, n_kv, batch),
-// kWarps warps per CTA. Each warp streams its pages (every kWarps-th page of the
-// chunk) through a private ring of kStages shared-memory stages filled by 1-D
-// bulk TMA copies; the copies are issued first thing, and the prologue (query
-// transform, and with APPEND the quantization of the new token) runs while
-// they are in flight.
+// Split-K decode attention, one launch per call. 1-D grid: CTA i serves chunk
+// i / n_pairs of (sequence, KV head) pair i % n_pairs, so that CTAs launched
+// together cover every pair. W warps per CTA, one CTA per SM. A chunk is
+// ppc consecutive pages; each warp streams pages through a private ring of S
+// shared-memory stages filled by 1-D bulk TMA copies. The first kStatic pages
+// of every warp are fixed (page p0 + warp + W k) and their copies go out before
+// any barrier; all later pages are claimed one at a time from a shared counter,
+// so warps that the scheduler favours take more pages and the warps of a CTA
+// finish together. The prologue (query transform, and with APPEND the
+// quantization of the new token) runs while the first copies are in flight.
 //
 // Per 16-token page a warp computes, with tokens on the rows of the products:
 //   logits  int8 m16n8k32: A = key-code limbs (hi, lo) or 0/1 sign bytes of
@@ -688,34 +696,39 @@ __device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float
 //           B = softmax weights split into fp16 high parts (columns 0-3) and
 //           low parts (columns 4-7), transposed into place with shuffles.
 // APPEND: the CTA whose chunk holds a sequence's last page first quantizes
-// (k_new, v_new) of that sequence into position seq_len - 1, then fetches the
-// page.
+// (k_new, v_new) of that sequence into position seq_len - 1; a warp that is
+// given that page before then holds its copy back until the token is written.
 template <int BK, int BV, int NH, bool APPEND>
-__global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArgs A) {
+__global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int W = DecodeWarps<NH>::value;
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
+  constexpr int S = decode_stages(W, kBlock);
   constexpr int kSignOff = 256 * BK, kVOff = 256 * (BK + 1), kNormOff = 256 * (BK + BV + 1);
   constexpr int kHeads = NH * kGroupHeads;
   constexpr bool kRegQ = NH <= 2;              // query fragments in registers (else shared memory)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int chunk = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int pair = b * A.n_kv + hk;
+  const int pair = static_cast<int>(blockIdx.x % static_cast<unsigned>(A.n_pairs));
+  const int chunk = static_cast<int>(blockIdx.x / static_cast<unsigned>(A.n_pairs));
+  const int b = pair / A.n_kv, hk = pair % A.n_kv;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kBlock);
-  static_assert((kWarps * kStages * kBlock + kWarps * kStages * 8) % 16 == 0, "prologue alignment");
-  Prologue<NH>& P = *reinterpret_cast<Prologue<NH>*>(bars + kWarps * kStages);
-  __shared__ int s_last;
-  __shared__ int s_pageok[kWarps * kStages];
-  uint8_t* stage0 = smem + warp * kStages * kBlock;
-  uint64_t* mybar = bars + warp * kStages;
-  int* myok = s_pageok + warp * kStages;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + W * S * kBlock);
+  static_assert((W * S * kBlock + W * S * 8) % 16 == 0, "prologue alignment");
+  Prologue<NH>& P = *reinterpret_cast<Prologue<NH>*>(bars + W * S);
+  int* s_btab = reinterpret_cast<int*>(&P + 1);   // physical ids of the chunk's claimable pages
+  __shared__ int s_last, s_claim;
+  __shared__ int s_lp[W * S];                     // logical page of each stage (-1: bad page id)
+  __shared__ int s_def[W];                        // physical id of a copy held back for the append
+  uint8_t* stage0 = smem + warp * S * kBlock;
+  uint64_t* mybar = bars + warp * S;
+  int* mylp = s_lp + warp * S;
 
   // The prologue's own loads go out first, ahead of the page stream, so that they
   // do not queue behind it: this warp's sketch rows as m16n8k16 A fragments and
   // the input of its first job (query head `warp`, or the new key / value).
   uint4 afv[8];
-  {
+  if (warp < kQjlRows / 16) {
     const uint4* F = reinterpret_cast<const uint4*>(T.sketch) + warp * 8 * 32 + lane;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) afv[ks] = __ldg(F + ks * 32);
@@ -733,15 +746,16 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   job_input(warp, xin);
   const float4 sgk = __ldg(reinterpret_cast<const float4*>(T.signs_k) + lane);
   const float4 sgv = __ldg(reinterpret_cast<const float4*>(T.signs_v) + lane);
-  // this warp's first 32 block-table entries, fetched before the length is known
-  // (bounded by the table width; entries past the sequence are discarded below)
+  // this warp's static pages (lane k holds page p0 + warp + W k), fetched before
+  // the length is known (bounded by the table width; pages past the sequence are
+  // discarded below)
   const int32_t* btab = A.block_tables + static_cast<int64_t>(b) * A.max_pages_per_seq;
   const int p0 = chunk * A.ppc;
-  const int first_j = p0 + warp + lane * kWarps;
-  const int spec_phys = first_j < A.max_pages_per_seq ? __ldg(btab + first_j) : -1;
+  const int first_j = p0 + warp + lane * W;
+  const int spec_phys = (lane < kStatic && first_j < A.max_pages_per_seq) ? __ldg(btab + first_j) : -1;
 
   if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(mybar + s, 1);
+    for (int s = 0; s < S; ++s) mbar_init(mybar + s, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncwarp();
@@ -753,26 +767,16 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   }
   const int seq_pages = (L + kPage - 1) / kPage;
   const int p1 = min(p0 + A.ppc, seq_pages);
-  const int nmine = (p1 > p0 + warp) ? (p1 - p0 - warp + kWarps - 1) / kWarps : 0;
-  // the CTA holding the last page appends the new token before fetching that page
+  const int n_static = p1 > p0 + warp ? min(kStatic, (p1 - p0 - warp + W - 1) / W) : 0;
+  const int n_dyn = max(0, p1 - p0 - W * kStatic);      // pages handed out by the claim counter
+  // the CTA holding the last page appends the new token before that page is fetched
   const bool appender = APPEND && L > 0 && chunk == (seq_pages - 1) / A.ppc;
   const int held = appender ? seq_pages - 1 : -1;
 
-  // Physical page ids of this warp's pages, 32 at a time: lane j holds page j of the window.
-  int win = 0;
-  int myphys = lane < nmine ? spec_phys : -1;
-  auto page_id = [&](int kth) {           // all lanes (shuffle); reloads the window when needed
-    if ((kth >> 5) != win) {
-      win = kth >> 5;
-      const int j = 32 * win + lane;
-      myphys = j < nmine ? btab[p0 + warp + j * kWarps] : -1;
-    }
-    return __shfl_sync(kFull, myphys, kth & 31);
-  };
-  // lane 0 only: start the transfer of physical page `phys` into stage s
-  auto issue = [&](int phys, int s) {
+  // lane 0 only: start the transfer of logical page lp (physical `phys`) into stage s
+  auto issue = [&](int phys, int lp, int s) {
     const bool ok = phys >= 0 && phys < A.n_pages;
-    myok[s] = ok;
+    mylp[s] = ok ? lp : -1;
     if (!ok) {
       set_error(T.err, TQ_DEV_BAD_PAGE);
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mybar + s)) : "memory");
@@ -782,12 +786,22 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
                   mybar + s);
     }
   };
-  const int n_first = min(nmine, kStages);
-  int n_early = 0;                        // stages issued now, in ring order, up to the held page
-  while (n_early < n_first && p0 + warp + n_early * kWarps != held) ++n_early;
-  for (int k = 0; k < n_early; ++k) {
-    const int phys = __shfl_sync(kFull, myphys, k);
-    if (lane == 0) issue(phys, k);
+  // Ring bookkeeping (lane 0): stages [0, filled) are taken in ring order; stage
+  // `def_stage` (if >= 0) holds the page being appended, issued after the append.
+  int filled = 0, def_stage = -1;
+  for (int k = 0; k < n_static; ++k) {
+    const int phys = __shfl_sync(kFull, spec_phys, k);
+    const int lp = p0 + warp + W * k;
+    if (lane == 0) {
+      if (lp == held) {
+        def_stage = k;
+        s_def[warp] = phys;
+        mylp[k] = lp;
+      } else {
+        issue(phys, lp, k);
+      }
+    }
+    ++filled;
   }
 
   // ---- prologue, while the first pages are in flight
@@ -797,7 +811,34 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     P.tab[32 + threadIdx.x] = T.thr_v[threadIdx.x];
     P.tab[48 + threadIdx.x] = T.cen_v[threadIdx.x];
   }
+  if (threadIdx.x == 0) s_claim = W * kStatic;
+  for (int i = threadIdx.x; i < n_dyn; i += W * 32) s_btab[i] = btab[p0 + W * kStatic + i];
   __syncthreads();
+  // fill the rest of the ring from the claim counter, and claim one more page to
+  // keep pending for the first refill (lane 0 owns the ring bookkeeping)
+  int pend = -1;                          // lane 0: next claimed logical page (-1: none)
+  if (lane == 0) {
+    const int want = S - filled + 1;
+    const int base = atomicAdd(&s_claim, want);
+    for (int k = 0; k < want; ++k) {
+      const int lp = p0 + base + k;
+      if (lp >= p1) break;
+      if (k == want - 1) {
+        pend = lp;
+        break;
+      }
+      const int phys = s_btab[lp - p0 - W * kStatic];
+      if (lp == held) {
+        def_stage = filled;
+        s_def[warp] = phys;
+        mylp[filled] = lp;
+      } else {
+        issue(phys, lp, filled);
+      }
+      ++filled;
+    }
+  }
+  filled = __shfl_sync(kFull, filled, 0);
   const int pos = L - 1;
   uint8_t* ablk = nullptr;                // block receiving the appended token
   if (appender) {
@@ -807,7 +848,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   }
   // jobs: kHeads query rotations, then (appender) the key and the value of the new token
   const int n_jobs = kHeads + (ablk ? 2 : 0);
-  for (int j = warp; j < n_jobs; j += kWarps) {
+  for (int j = warp; j < n_jobs; j += W) {
     float x[4];
     if (j == warp) {
 #pragma unroll
@@ -887,11 +928,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
       out4[t * 128 + 16 * warp + g + 8] = (c[2] + c[3]) * inv;
     }
   };
+  if (warp < kQjlRows / 16) {             // warp-uniform: eight warps own the 128 sketch rows
 #pragma unroll
-  for (int h = 0; h < NH; ++h) sketch_product(&P.qt[4 * h][0], &P.sig[4 * h], 8, &P.pp[4 * h][0]);
-  if (ablk) sketch_product(P.u, &P.sig[kHeads], 2, P.z);
+    for (int h = 0; h < NH; ++h) sketch_product(&P.qt[4 * h][0], &P.sig[4 * h], 8, &P.pp[4 * h][0]);
+    if (ablk) sketch_product(P.u, &P.sig[kHeads], 2, P.z);
+  }
   __syncthreads();
-  for (int j = warp; j < kHeads + (ablk ? 1 : 0); j += kWarps) {
+  for (int j = warp; j < kHeads + (ablk ? 1 : 0); j += W) {
     if (j < kHeads) {
       float x[4], pv[4];
 #pragma unroll
@@ -926,11 +969,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   }
   if (ablk) asm volatile("fence.proxy.async.global;" ::: "memory");   // the page is next read by the TMA unit
   __syncthreads();
-  for (int k = n_early; k < n_first; ++k) {  // the held page (appender only) and what follows it
-    const int phys = __shfl_sync(kFull, myphys, k);
-    if (lane == 0) issue(phys, k);
-  }
-  __syncwarp();                           // lane 0's page flags are visible to the warp
+  if (lane == 0 && def_stage >= 0) issue(s_def[warp], held, def_stage);   // the appended page
+  __syncwarp();                           // lane 0's stage records are visible to the warp
 
   // B fragment of lane (g, t): column g -> head 4h + g/2; rows 4t.. (+16 for reg 1) of k-tile kt
   //   n-tile 0: limb 2 (g even) or 1 (g odd); n-tile 1: limb 0 (g even) or zero (g odd)
@@ -986,14 +1026,15 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   bool alive = true;
   int s = 0;
   unsigned parity = 0;
-  int lp = p0 + warp;
-  for (int k = 0; k < nmine; ++k, lp += kWarps) {
+  int inflight = filled;                  // stages holding a page not yet consumed (warp-uniform)
+  while (inflight > 0) {
     if (!mbar_wait(mybar + s, parity)) {
       if (lane == 0) set_error(T.err, TQ_DEV_TIMEOUT);
       alive = false;
       break;
     }
-    const bool page_ok = myok[s] != 0;
+    const int lp = mylp[s];
+    const bool page_ok = lp >= 0;
     const uint8_t* blk = stage0 + s * kBlock;
 
     // ---- this lane's operands from the staged block (tokens g and g + 8)
@@ -1118,17 +1159,19 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
       for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pb[h][0], pb[h][1]);
     }
 
-    // ---- refill this stage with the page kStages ahead (all its reads are consumed)
-    if (k + kStages < nmine) {
-      const int phys = page_id(k + kStages);     // convergent: every lane reaches here
-      __syncwarp();
-      if (lane == 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(phys, s);
-      }
-      __syncwarp();
+    // ---- refill this stage with the pending claim (all its reads are consumed),
+    // and claim the next page; that claim is only used at the next refill
+    const bool refill = __shfl_sync(kFull, pend, 0) >= 0;
+    __syncwarp();
+    if (lane == 0 && refill) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(s_btab[pend - p0 - W * kStatic], pend, s);
+      const int next = p0 + atomicAdd(&s_claim, 1);
+      pend = next < p1 ? next : -1;
     }
-    if (++s == kStages) {
+    __syncwarp();
+    if (!refill) --inflight;
+    if (++s == S) {
       s = 0;
       parity ^= 1u;
     }
@@ -1136,11 +1179,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   if (!alive) {
     // A wait ran out: give every transfer this warp still has in flight a
     // bounded chance to land before the shared memory is reused.
-    for (int k2 = 0; k2 < nmine; ++k2) mbar_wait(mybar + (k2 % kStages), (k2 / kStages) & 1);
+    for (int i = 0; i < inflight; ++i) mbar_wait(mybar + (s + i) % S, s + i >= S ? parity ^ 1u : parity);
   }
   __syncwarp();
   if (lane == 0)
-    for (int s2 = 0; s2 < kStages; ++s2)
+    for (int s2 = 0; s2 < S; ++s2)
       asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(mybar + s2)) : "memory");
 
   // ---- merge the warps of this CTA (the pipeline buffers are free now)
@@ -1152,7 +1195,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   }
   __syncthreads();
   float* s_acc = reinterpret_cast<float*>(smem);                       // [warp][NH][8 columns][128]
-  float* s_st = s_acc + kWarps * NH * 8 * 128;                           // [warp][NH][4 heads][3]
+  float* s_st = s_acc + W * NH * 8 * 128;                                // [warp][NH][4 heads][3]
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
 #pragma unroll
@@ -1174,10 +1217,10 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
     const int h = hh >> 2, h4 = hh & 3;
     float M = kNegBig;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_st[((w * NH + h) * kGroupHeads + h4) * 3 + 0]);
+    for (int w = 0; w < W; ++w) M = fmaxf(M, s_st[((w * NH + h) * kGroupHeads + h4) * 3 + 0]);
     float a = 0.0f, l = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < W; ++w) {
       const float* st = s_st + ((w * NH + h) * kGroupHeads + h4) * 3;
       const float* ac = s_acc + ((w * NH + h) * 8) * 128;
       const float f = ex2(st[0] - M);
@@ -1204,22 +1247,23 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
   // ---- last CTA of this (sequence, KV head): merge the chunks, de-rotate, store.
   // The chunk records (written by the other CTAs, published by the counter) come
   // into shared memory by bulk copies, merge_cap chunks at a time. Warp w merges
-  // head slots w % 4 (+4, +8, ...) over the chunks of parity w / 4 with an online
-  // maximum; the two parities meet in shared memory.
+  // head slots w % 4 (+4, +8, ...) over the chunks c with c % (W / 4) == w / 4,
+  // with an online maximum; the W / 4 partial merges meet in shared memory.
   constexpr int kRec = 132;                                  // floats per (chunk, head slot) record
   constexpr int kSlots = NH * kGroupHeads;
   const unsigned chunk_bytes = kSlots * kRec * 4;
   const float* pbase = A.partial + static_cast<size_t>(pair) * A.chunks * kSlots * kRec;
   float* s_part = reinterpret_cast<float*>(smem);            // [merge_cap][kSlots][kRec]
-  float* s_mrg = s_part + static_cast<size_t>(A.merge_cap) * kSlots * kRec;   // [2][kSlots][kRec]
-  uint64_t* fbar = reinterpret_cast<uint64_t*>(s_mrg + 2 * kSlots * kRec);
+  constexpr int kGroups = W / kGroupHeads;                   // warps per head slot
+  float* s_mrg = s_part + static_cast<size_t>(A.merge_cap) * kSlots * kRec;   // [kGroups][kSlots][kRec]
+  uint64_t* fbar = reinterpret_cast<uint64_t*>(s_mrg + kGroups * kSlots * kRec);
   const float4 sv = __ldg(reinterpret_cast<const float4*>(T.signs_v) + lane);
   if (threadIdx.x == 0) {
     mbar_init(fbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  const int half = warp / kGroupHeads, sl0 = warp % kGroupHeads;
+  const int grp = warp / kGroupHeads, sl0 = warp % kGroupHeads;
   float M[NH], l[NH], a[NH][4];
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
@@ -1246,7 +1290,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
       const int slot = sl0 + kGroupHeads * h;
       if (slot >= A.group) continue;
 #pragma unroll 4
-      for (int c = half; c < nc; c += 2) {
+      for (int c = grp; c < nc; c += kGroups) {
         const float* rec = s_part + (c * kSlots + slot) * kRec;
         const float Mc = rec[128];
         const float Mn = fmaxf(M[h], Mc);
@@ -1267,21 +1311,27 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     const int slot = sl0 + kGroupHeads * h;
-    float* mine = s_mrg + (half * kSlots + slot) * kRec;
+    float* mine = s_mrg + (grp * kSlots + slot) * kRec;
     reinterpret_cast<float4*>(mine)[lane] = make_float4(a[h][0], a[h][1], a[h][2], a[h][3]);
     if (lane == 0) { mine[128] = M[h]; mine[129] = l[h]; }
   }
   __syncthreads();
-  for (int slot = warp; slot < A.group; slot += kWarps) {
-    const float* r0 = s_mrg + slot * kRec;
-    const float* r1 = s_mrg + (kSlots + slot) * kRec;
-    const float Mx = fmaxf(r0[128], r1[128]);
-    const float f0 = ex2(r0[128] - Mx), f1 = ex2(r1[128] - Mx);
-    const float lt = r0[129] * f0 + r1[129] * f1;
-    const float4 x0 = reinterpret_cast<const float4*>(r0)[lane], x1 = reinterpret_cast<const float4*>(r1)[lane];
+  for (int slot = warp; slot < A.group; slot += W) {
+    float Mx = kNegBig;
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) Mx = fmaxf(Mx, s_mrg[(q * kSlots + slot) * kRec + 128]);
+    float lt = 0.0f, v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) {
+      const float* r = s_mrg + (q * kSlots + slot) * kRec;
+      const float f = ex2(r[128] - Mx);
+      const float4 x = reinterpret_cast<const float4*>(r)[lane];
+      lt = fmaf(r[129], f, lt);
+      v[0] = fmaf(x.x, f, v[0]); v[1] = fmaf(x.y, f, v[1]); v[2] = fmaf(x.z, f, v[2]); v[3] = fmaf(x.w, f, v[3]);
+    }
     const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-    float v[4] = {(x0.x * f0 + x1.x * f1) * inv, (x0.y * f0 + x1.y * f1) * inv,
-                  (x0.z * f0 + x1.z * f1) * inv, (x0.w * f0 + x1.w * f1) * inv};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] *= inv;
     fwht128(v, lane);
     float4 o;
     o.x = v[0] * sv.x * kInvSqrtD;
@@ -1295,16 +1345,21 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(Tables T, DecodeArg
 
 template <int BK, int BV, int NH, bool APPEND>
 cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
+  constexpr int W = DecodeWarps<NH>::value;
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
-  const size_t pipe = static_cast<size_t>(kWarps) * kStages * kBlock + kWarps * kStages * sizeof(uint64_t) +
-                      sizeof(Prologue<NH>);
-  const size_t merge = static_cast<size_t>(kWarps) * NH * 8 * 128 * 4 + kWarps * NH * kGroupHeads * 3 * 4;
+  constexpr int S = decode_stages(W, kBlock);
+  // main loop: stages, barriers, prologue scratch, the chunk's block-table window
+  const size_t pipe = static_cast<size_t>(W) * S * kBlock + W * S * sizeof(uint64_t) + sizeof(Prologue<NH>) +
+                      ((static_cast<size_t>(a.ppc) * 4 + 15) & ~static_cast<size_t>(15));
+  // CTA merge: every warp's accumulators and softmax state
+  const size_t merge = static_cast<size_t>(W) * NH * 8 * 128 * 4 + W * NH * kGroupHeads * 3 * 4;
   const size_t smem = pipe > merge ? pipe : merge;
-  // final merge: chunk records, then [2][slots][132] floats and one barrier
+  // final merge: merge_cap chunk records, then [W / 4][slots][132] floats and one barrier
   const size_t chunk_bytes = static_cast<size_t>(NH) * kGroupHeads * 132 * 4;
+  const size_t groups = W / kGroupHeads;
+  if (smem > 227 * 1024 || smem < (groups + 1) * chunk_bytes + 16) return cudaErrorInvalidConfiguration;
   DecodeArgs args = a;
-  args.merge_cap = static_cast<int>((smem - 2 * chunk_bytes - 16) / chunk_bytes);
-  if (args.merge_cap < 1) return cudaErrorInvalidConfiguration;
+  args.merge_cap = static_cast<int>((smem - groups * chunk_bytes - 16) / chunk_bytes);
   auto fn = decode_kernel<BK, BV, NH, APPEND>;
   static size_t configured = 0;     // raise the shared-memory limit once per instantiation
   if (configured < smem) {
@@ -1312,7 +1367,7 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  fn<<<grid, kWarps * 32, smem, s>>>(T, args);
+  fn<<<grid, W * 32, smem, s>>>(T, args);
   return cudaGetLastError();
 }
 
@@ -1373,6 +1428,7 @@ DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float
   a.n_hg = plan.n_hg;
   a.chunks = plan.chunks;
   a.ppc = plan.pages_per_chunk;
+  a.n_pairs = plan.n_pairs;
   return a;
 }
 
@@ -1411,7 +1467,7 @@ cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q
                           float* out, void* workspace, cudaStream_t s) {
   const DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq,
                                    seq_lens, max_seq_len, out, workspace);
-  return dispatch_bk<false>(t, a, dim3(plan.chunks, plan.n_kv, plan.batch), s);
+  return dispatch_bk<false>(t, a, dim3(plan.chunks * plan.n_pairs), s);
 }
 
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
@@ -1423,7 +1479,7 @@ cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const vo
   a.k_new = k_new;
   a.v_new = v_new;
   a.kv_dtype = kv_dtype;
-  return dispatch_bk<true>(t, a, dim3(plan.chunks, plan.n_kv, plan.batch), s);
+  return dispatch_bk<true>(t, a, dim3(plan.chunks * plan.n_pairs), s);
 }
 
 }  // namespace tq
