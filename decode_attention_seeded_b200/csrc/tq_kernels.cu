@@ -753,6 +753,16 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   const int p0 = chunk * A.ppc;
   const int first_j = p0 + warp + lane * W;
   const int spec_phys = (lane < kStatic && first_j < A.max_pages_per_seq) ? __ldg(btab + first_j) : -1;
+  // the first kSpecWin entries of the chunk's claimable window, also fetched now
+  // (entries past the table width are skipped; past the sequence, never claimed)
+  constexpr int kSpecPer = 2, kSpecWin = kSpecPer * W * 32;
+  const int win_lim = min(A.ppc, A.max_pages_per_seq - p0) - W * kStatic;
+  int spec_win[kSpecPer];
+#pragma unroll
+  for (int r = 0; r < kSpecPer; ++r) {
+    const int i = threadIdx.x + r * W * 32;
+    spec_win[r] = i < win_lim ? __ldg(btab + p0 + W * kStatic + i) : -1;
+  }
 
   if (lane == 0) {
     for (int s = 0; s < S; ++s) mbar_init(mybar + s, 1);
@@ -786,22 +796,21 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
                   mybar + s);
     }
   };
-  // Ring bookkeeping (lane 0): stages [0, filled) are taken in ring order; stage
-  // `def_stage` (if >= 0) holds the page being appended, issued after the append.
-  int filled = 0, def_stage = -1;
-  for (int k = 0; k < n_static; ++k) {
-    const int phys = __shfl_sync(kFull, spec_phys, k);
-    const int lp = p0 + warp + W * k;
-    if (lane == 0) {
-      if (lp == held) {
-        def_stage = k;
-        s_def[warp] = phys;
-        mylp[k] = lp;
-      } else {
-        issue(phys, lp, k);
-      }
+  // Ring bookkeeping (warp-uniform): stages [0, filled) are taken in ring order;
+  // stage def_stage (if >= 0) holds the page being appended, issued after the
+  // append. Lane k issues stage k of the static pages.
+  int filled = n_static, def_stage = -1;
+  {
+    const int lp = p0 + warp + W * lane;
+    const bool mine = lane < n_static, defer = mine && lp == held;
+    if (defer) {
+      s_def[warp] = spec_phys;
+      mylp[lane] = lp;
+    } else if (mine) {
+      issue(spec_phys, lp, lane);
     }
-    ++filled;
+    const unsigned dm = __ballot_sync(kFull, defer);
+    if (dm) def_stage = __ffs(dm) - 1;
   }
 
   // ---- prologue, while the first pages are in flight
@@ -812,33 +821,39 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     P.tab[48 + threadIdx.x] = T.cen_v[threadIdx.x];
   }
   if (threadIdx.x == 0) s_claim = W * kStatic;
-  for (int i = threadIdx.x; i < n_dyn; i += W * 32) s_btab[i] = btab[p0 + W * kStatic + i];
-  __syncthreads();
-  // fill the rest of the ring from the claim counter, and claim one more page to
-  // keep pending for the first refill (lane 0 owns the ring bookkeeping)
-  int pend = -1;                          // lane 0: next claimed logical page (-1: none)
-  if (lane == 0) {
-    const int want = S - filled + 1;
-    const int base = atomicAdd(&s_claim, want);
-    for (int k = 0; k < want; ++k) {
-      const int lp = p0 + base + k;
-      if (lp >= p1) break;
-      if (k == want - 1) {
-        pend = lp;
-        break;
-      }
-      const int phys = s_btab[lp - p0 - W * kStatic];
-      if (lp == held) {
-        def_stage = filled;
-        s_def[warp] = phys;
-        mylp[filled] = lp;
-      } else {
-        issue(phys, lp, filled);
-      }
-      ++filled;
-    }
+#pragma unroll
+  for (int r = 0; r < kSpecPer; ++r) {
+    const int i = threadIdx.x + r * W * 32;
+    if (i < n_dyn) s_btab[i] = spec_win[r];
   }
-  filled = __shfl_sync(kFull, filled, 0);
+  for (int i = kSpecWin + threadIdx.x; i < n_dyn; i += W * 32) s_btab[i] = btab[p0 + W * kStatic + i];
+  __syncthreads();
+  // Fill the rest of the ring from the claim counter (lane k takes stage
+  // filled + k), and claim one more page to keep pending for the first refill.
+  int pend;                               // next claimed logical page (-1: none); lane 0 updates it
+  {
+    const int want = S - filled + 1;
+    int base = 0;
+    if (lane == 0) base = atomicAdd(&s_claim, want);
+    base = __shfl_sync(kFull, base, 0);
+    const int nvalid = min(max(p1 - p0 - base, 0), want);   // claims that fall inside the chunk
+    const int nfill = min(nvalid, want - 1);
+    const int lp = p0 + base + lane;
+    const bool mine = lane < nfill, defer = mine && lp == held;
+    if (mine) {
+      const int phys = s_btab[lp - p0 - W * kStatic];
+      if (defer) {
+        s_def[warp] = phys;
+        mylp[filled + lane] = lp;
+      } else {
+        issue(phys, lp, filled + lane);
+      }
+    }
+    const unsigned dm = __ballot_sync(kFull, defer);
+    if (dm) def_stage = filled + __ffs(dm) - 1;
+    pend = nvalid == want ? p0 + base + want - 1 : -1;
+    filled += nfill;
+  }
   const int pos = L - 1;
   uint8_t* ablk = nullptr;                // block receiving the appended token
   if (appender) {
@@ -970,6 +985,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   if (ablk) asm volatile("fence.proxy.async.global;" ::: "memory");   // the page is next read by the TMA unit
   __syncthreads();
   if (lane == 0 && def_stage >= 0) issue(s_def[warp], held, def_stage);   // the appended page
+  __syncwarp();
   __syncwarp();                           // lane 0's stage records are visible to the warp
 
   // B fragment of lane (g, t): column g -> head 4h + g/2; rows 4t.. (+16 for reg 1) of k-tile kt
