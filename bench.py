@@ -237,6 +237,41 @@ class DecodeBench:
         torch.cuda.current_stream(self.dev).wait_stream(s)
         return g
 
+    def quantize_timing(self, reps=5):
+        """Quantize-prefill of one layer's full context (K and V of every KV head).
+
+        Algorithmic bytes = the K/V inputs read + the compressed blocks written.
+        Layers rotate so that the inputs (0.13 GB per layer) are not L2-resident."""
+        torch, wl = self.torch, self.wl
+        n_kv = wl.n_kv_heads
+        g = torch.Generator(device=self.dev)
+        g.manual_seed(wl.seed * 7 + 11)
+        bufs = []
+        for i in range(2):
+            gen = self.synth.Generator(wl, layer=i)
+            sc = torch.from_numpy(gen.scales["k"]).float().to(self.dev)
+            k = (torch.randn((self.T0, n_kv, 128), generator=g, device=self.dev) * sc).to(torch.bfloat16)
+            v = (torch.randn((self.T0, n_kv, 128), generator=g, device=self.dev) * sc).to(torch.bfloat16)
+            bufs.append((k, v))
+        cache, n_pages = self.caches[0]
+        bt = self.btabs[0][0]
+        self.ctx.quantize_prefill(bufs[0][0], bufs[0][1], bt, 0, cache, n_pages)
+        torch.cuda.synchronize(self.dev)
+        st = torch.cuda.current_stream(self.dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for r in range(reps):
+            k, v = bufs[r % 2]
+            evs[r][0].record(st)
+            self.ctx.quantize_prefill(k, v, bt, 0, cache, n_pages)
+            evs[r][1].record(st)
+        torch.cuda.synchronize(self.dev)
+        secs = statistics.median(a.elapsed_time(b) for a, b in evs) / 1e3
+        bytes_in = 2 * self.T0 * n_kv * 128 * 2
+        bytes_out = self.T0 * n_kv * (self.ctx.block_bytes // 16)
+        return {"gbs": (bytes_in + bytes_out) / secs / 1e9, "us_per_call": secs * 1e6,
+                "tokens": self.T0, "kv_heads": n_kv, "bytes_in": bytes_in, "bytes_out": bytes_out,
+                "kernel": "quantize_prefill_kernel via tq_quantize_prefill (bf16 K/V, one layer)"}
+
     def decode_only_graph(self, reps):
         """reps x (32 layers of tq_decode_attention) at the final context length."""
         wl = self.wl
@@ -248,6 +283,22 @@ class DecodeBench:
                 self.ctx.decode_attention(self.q[last, layer], cache, n_pages, self.btabs[layer], self.lens[last],
                                           wl.n_kv_heads, self.max_len, self.out[layer], self.ws)
         return self.capture(body, range(reps))
+
+
+def max_over_ranks(x, world, device):
+    """The largest of the ranks' values (every rank gets it); x itself when world == 1."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, seconds):
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / seconds
 
 
 def timed(torch, dev, fn):
@@ -379,18 +430,11 @@ def main():
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
-
     barrier()
     with ClockSampler(local) as clk:
         t_main = timed(torch, dev, g_main.replay)
     barrier()
-    t_main = max_over_ranks(t_main)
+    t_main = max_over_ranks(t_main, world, dev)
     clocks = clk.summary()
 
     # end-to-end arm: same K steps from host buffers (state rewinds: same slots rewritten)
@@ -398,7 +442,7 @@ def main():
     g_e2e_w = bench.capture(bench.step_e2e, range(W))
     g_e2e_w.replay()
     barrier()
-    t_e2e = max_over_ranks(timed(torch, dev, g_e2e.replay))
+    t_e2e = max_over_ranks(timed(torch, dev, g_e2e.replay), world, dev)
     barrier()
 
     # roofline: decode attention alone, back-to-back over the 32 layer caches
@@ -406,11 +450,13 @@ def main():
     g_dec = bench.decode_only_graph(reps)
     g_dec.replay()
     barrier()
-    t_dec = max_over_ranks(timed(torch, dev, g_dec.replay))
+    t_dec = max_over_ranks(timed(torch, dev, g_dec.replay), world, dev)
     n_dec = reps * bench.n_layers
     dec_s = t_dec / n_dec
     assert bench.ctx.device_error() == 0
 
+    quant = bench.quantize_timing()
+    quant["frac"] = quant["gbs"] / load_peaks()[0]
     peak, peak_kind = load_peaks()
     bpt = bench.ctx.block_bytes // 16                     # bytes per token-head (102 for 3/2 bits)
     ctx_len = bench.max_len
@@ -419,7 +465,7 @@ def main():
     traffic = recorded_traffic("bytes_per_launch")
 
     tokens = K * wl.batch * world
-    value = tokens / t_main
+    value = job_throughput(K * wl.batch, world, t_main)
     h2d, d2h = bench.e2e_bytes()
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -432,11 +478,12 @@ def main():
                    "l2": f"inputs larger than L2: {bench.n_layers} layer caches, "
                          f"{bench.n_layers * bench.caches[0][1] * bench.page_bytes / 1e9:.2f} GB per step",
                    "parallelism": f"replica x{world} (one sequence per GPU)"},
-        "e2e": {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": job_throughput(K * wl.batch, world, t_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                      "kernel": "decode_kernel via tq_decode_attention (query transform, split-K decode, merge)",
                      "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
+        "quantize": quant,
         "gpu_launches": K * bench.n_layers,
         "clocks": clocks,
     }
