@@ -199,7 +199,7 @@ struct tq_ctx {
   int sm_count = 0;                // streaming multiprocessors of the device (sizes decode grids)
   bool rot_ready = false, cb_ready = false;
   float* d_signs = nullptr;        // [2][128]: D_K then D_V
-  uint16_t* d_sketch_t = nullptr;  // [128][128] fp16 bits of S^T, then S in A-fragment order
+  uint16_t* d_sketch_t = nullptr;  // fp16 bits: S^T, S as decode A fragments, S as prefill B fragments
   unsigned* d_err = nullptr;
   tq::Tables tables;
 };
@@ -366,7 +366,7 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   cudaError_t e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, device);
   if (e == cudaSuccess && c->sm_count <= 0) e = cudaErrorInvalidDevice;
   if (e == cudaSuccess) e = cudaMalloc(&c->d_signs, 2 * tq::kHeadDim * sizeof(float));
-  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 2 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
+  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 3 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
   if (e == cudaSuccess) e = cudaMalloc(&c->d_err, sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(unsigned));
   if (e != cudaSuccess) {
@@ -377,6 +377,7 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   c->tables.signs_v = c->d_signs + tq::kHeadDim;
   c->tables.sketch_t = c->d_sketch_t;
   c->tables.sketch = c->d_sketch_t + tq::kQjlRows * tq::kHeadDim;
+  c->tables.sketch_qb = c->d_sketch_t + 2 * tq::kQjlRows * tq::kHeadDim;
   c->tables.err = c->d_err;
   *out = c;
   return TQ_OK;
@@ -399,7 +400,7 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
   if (tq_status st = check_device(ctx)) return st;
   const int d = tq::kHeadDim, m = tq::kQjlRows;
   std::vector<int8_t> sk(d), sv(d);
-  std::vector<uint16_t> s(m * d), st(2 * m * d);
+  std::vector<uint16_t> s(m * d), st(3 * m * d);
   tq_host_sign_vector(seed_k, d, sk.data());
   tq_host_sign_vector(seed_v, d, sv.data());
   tq_host_gaussian_sketch(seed_s, m, d, s.data());
@@ -414,6 +415,25 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
   // 16ks..16ks+15), lane (g, t), register j -> row 16w + g + 8(j&1), fp16 pair at
   // columns 16ks + 2t + 8(j>>1) (+0, +1). Stored [w][ks][lane][j], so one warp's
   // register set for one k-step is 512 contiguous bytes.
+  // S as m16n8k16 B fragments of the prefill product z = S u (tokens on rows):
+  // coordinates and sketch rows both follow a lane's layout chunk. Coordinate
+  // of k-step ks, k index kk: 16 ks + 4 tk + slot (tk = kk >> 1 mod 4, slot =
+  // kk & 1, + 2 when kk >= 8); sketch row of n-tile nt, column c:
+  // 32 (nt >> 2) + 16 ((nt >> 1) & 1) + 4 (c >> 1) + 2 (nt & 1) + (c & 1).
+  // Stored [ks][nt][lane][2 regs], lane (g, t): reg 0 = k 2t, 2t+1, reg 1 = k
+  // 2t+8, 2t+9, column g.
+  uint16_t* qb = st.data() + 2 * m * d;
+  for (int ks = 0; ks < d / 16; ++ks)
+    for (int nt = 0; nt < m / 8; ++nt)
+      for (int lane = 0; lane < 32; ++lane)
+        for (int r = 0; r < 2; ++r)
+          for (int h = 0; h < 2; ++h) {
+            const int kk = 2 * (lane & 3) + 8 * r + h, c = lane >> 2;
+            const int tk = (kk & 7) >> 1, slot = (kk & 1) + 2 * (kk >> 3);
+            const int coord = 16 * ks + 4 * tk + slot;
+            const int row = 32 * (nt >> 2) + 16 * ((nt >> 1) & 1) + 4 * (c >> 1) + 2 * (nt & 1) + (c & 1);
+            qb[(((ks * (m / 8) + nt) * 32 + lane) * 2 + r) * 2 + h] = s[row * d + coord];
+          }
   uint16_t* frag = st.data() + m * d;
   for (int w = 0; w < m / 16; ++w)
     for (int ks = 0; ks < d / 16; ++ks)
@@ -495,6 +515,8 @@ tq_status tq_quantize_prefill(tq_ctx* ctx, const void* k, const void* v, tq_dtyp
                                          cache, n_cache_pages))
     return st;
   if (n_tokens == 0) return TQ_OK;
+  // rows are staged by bulk copies, which need 16-byte aligned sources
+  if (reinterpret_cast<uintptr_t>(k) % 16 || reinterpret_cast<uintptr_t>(v) % 16) return TQ_ERR_INVALID_ARG;
   return from_cuda(tq::launch_quantize_prefill(ctx->tables, k, v, dtype, n_tokens, n_kv_heads,
                                                block_table, start_pos, cache, n_cache_pages,
                                                static_cast<cudaStream_t>(stream)));

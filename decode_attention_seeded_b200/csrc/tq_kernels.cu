@@ -341,57 +341,435 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(Tables T, const vo
   }
 }
 
-// One CTA per (page, KV head) of a contiguous run: the block is assembled in
-// shared memory (merged with the page's previous contents if the run covers it
-// only partly) and written back with 16-byte stores.
-__global__ void __launch_bounds__(256) quantize_prefill_kernel(Tables T, const void* k, const void* v,
-                                                               int dtype, int n_tokens, int n_kv,
-                                                               const int32_t* block_table, int start_pos,
-                                                               uint8_t* cache, int64_t n_pages) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __half* s_sk = reinterpret_cast<__half*>(smem);
-  uint8_t* sblk = smem + kHeadDim * kQjlRows * 2;
-  __shared__ float s_tab[64];     // thr_k, cen_k, thr_v, cen_v
-  stage_tables(T, s_sk, s_tab);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-  const int first_page = start_pos / kPage;
-  const int last_page = (start_pos + n_tokens - 1) / kPage;
-  const int n_run_pages = last_page - first_page + 1;
-  const int bb = T.block_bytes;
-  for (int job = blockIdx.x; job < n_run_pages * n_kv; job += gridDim.x) {
-    const int lp = first_page + job / n_kv, h = job % n_kv;
-    const int phys = block_table[lp];
-    const bool bad = phys < 0 || phys >= n_pages;
-    if (bad) {
-      if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_SLOT);
-      continue;     // uniform across the CTA
+// ---- shared-memory barriers and 1-D bulk copies ---------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: gives up after ~2^31 clock cycles (about a second).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > (1ll << 31)) return false;
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_1d(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ===================================================================== prefill
+// Quantize a contiguous run of one sequence, one warp per (page, KV head) tile.
+//
+// Lane (g, t) holds tokens g and g + 8 of the page at the 32 coordinates of its
+// layout chunk, coordinate pf_coord(i, t) = 16 (i >> 2) + 4 t + (i & 3) for
+// i = 0..31. Coordinate bits 0, 1, 4, 5, 6 are then bits of i and bits 2, 3 are
+// bits of t, so the Walsh-Hadamard transform runs five stages in registers and
+// two across the lanes of a quad. The same registers are the m16n8k16 A
+// fragments of z = S u (k-step ks = coordinates 16 ks .. 16 ks + 15, tokens on
+// the rows), and with S stored in a matching B-fragment order (sketch_qb) the
+// accumulator of n-tile nt holds exactly the sketch rows of the lane's sign
+// chunk, so codes and sign bits are packed without data exchange. Value codes
+// are moved to the value chunks (coordinates x 4 tokens) through a 2 KB
+// shared-memory tile per warp.
+__device__ __forceinline__ int pf_coord(int i, int t) { return 16 * (i >> 2) + 4 * t + (i & 3); }
+
+// Cell of y in a symmetric b-bit codebook: code = #{j : y > t_j} (a value on a
+// threshold may land in either neighbour; such values lie inside the tolerance
+// band) and the centroid c[code]. thr / cen: the 2^b - 1 thresholds and 2^b
+// centroids in ascending order; the middle threshold is 0.
+template <int B, typename TA, typename CA>
+__device__ __forceinline__ int cell_of(float y, const TA& thr, const CA& cen, float& chat) {
+  constexpr int H = 1 << (B - 1);
+  const float a = fabsf(y);
+  int k;
+  float cp;
+  if constexpr (B == 2) {
+    const bool p = a > thr[H];
+    k = p;
+    cp = p ? cen[H + 1] : cen[H];
+  } else if constexpr (B == 3) {
+    const bool p2 = a > thr[H + 1];
+    const bool p1 = a > (p2 ? thr[H + 2] : thr[H]);
+    k = 2 * p2 + p1;
+    cp = p2 ? (p1 ? cen[H + 3] : cen[H + 2]) : (p1 ? cen[H + 1] : cen[H]);
+  } else {
+    const bool p4 = a > thr[H + 3];
+    const bool p2 = a > (p4 ? thr[H + 5] : thr[H + 1]);
+    const bool p1 = a > (p4 ? (p2 ? thr[H + 6] : thr[H + 4]) : (p2 ? thr[H + 2] : thr[H]));
+    k = 4 * p4 + 2 * p2 + p1;
+    const float lo = p2 ? (p1 ? cen[H + 3] : cen[H + 2]) : (p1 ? cen[H + 1] : cen[H]);
+    const float hi = p2 ? (p1 ? cen[H + 7] : cen[H + 6]) : (p1 ? cen[H + 5] : cen[H + 4]);
+    cp = p4 ? hi : lo;
+  }
+  const bool pos = y > 0.0f;
+  chat = pos ? cp : -cp;
+  return pos ? H + k : H - 1 - k;
+}
+
+// Add code `c` of lane-local coordinate i (selector i >> 2, nibble i & 3) to the
+// b words of one token half of a key lane chunk.
+template <int B>
+__device__ __forceinline__ void put_key_code(uint32_t (&w)[4], int i, uint32_t c) {
+  const int j = i >> 2, q = i & 3;
+  if constexpr (B == 2) {
+    w[j >> 2] |= c << (16 * (j & 1) + 4 * q + 2 * ((j >> 1) & 1));
+  } else if constexpr (B == 3) {
+    if (j < 6) {
+      w[j >> 1] |= c << (16 * (j & 1) + 4 * q);
+    } else {
+      const int bit = 4 * (4 * (j - 6) + q) + 3;
+      w[0] |= (c & 1u) << bit;
+      w[1] |= ((c >> 1) & 1u) << bit;
+      w[2] |= ((c >> 2) & 1u) << bit;
     }
-    uint8_t* gblk = cache + (static_cast<int64_t>(phys) * n_kv + h) * bb;
-    const int t0 = max(start_pos, lp * kPage), t1 = min(start_pos + n_tokens, (lp + 1) * kPage);
-    const bool full = (t0 == lp * kPage) && (t1 == (lp + 1) * kPage);
-    __syncthreads();
-    for (int i = threadIdx.x; i < bb / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(sblk)[i] = full ? make_uint4(0, 0, 0, 0) : reinterpret_cast<const uint4*>(gblk)[i];
-    __syncthreads();
-    for (int pos = t0 + warp; pos < t1; pos += nwarp) {
-      const int tok = pos - start_pos, tau = pos % kPage;
-      float x[4];
-      VecOut o;
-      load_row4(k, static_cast<size_t>(tok) * n_kv + h, dtype, lane, x);
-      quantize_vector(x, T.signs_k, s_tab, s_tab + 16, T.key_bits, s_sk, true, lane, o);
-      store_key_token(sblk, tau, T.key_bits, o, lane);
-      if (lane == 0) {
-        store_norm(sblk, T.key_bits, T.value_bits, 0, tau, o.norm);
-        store_norm(sblk, T.key_bits, T.value_bits, 1, tau, o.gamma);
+  } else {
+    w[j >> 1] |= c << (16 * (j & 1) + 4 * q);
+  }
+}
+
+// Add the four codes of value coordinate (mt, hf) of a lane chunk to its 2b
+// words. x holds one code per byte: byte 2e + tg = token 2t + e + 8 tg.
+template <int B>
+__device__ __forceinline__ void put_value_codes(uint32_t (&w)[8], int mt, int hf, uint32_t x) {
+  if constexpr (B == 2) {
+    // selector s = 2 mt + tg -> word mt >> 1, bits 16 tg + 4 (2 hf + e) + 2 (mt & 1)
+    const uint32_t y = prmt(x, 0u, 0x3120u);                 // byte e + 2 tg
+    const uint32_t z = (y & 0x00030003u) | ((y >> 4) & 0x00300030u);
+    w[mt >> 1] |= z << (8 * hf + 2 * (mt & 1));
+  } else {
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int tg = 0; tg < 2; ++tg) {
+        const uint32_t c = (x >> (8 * (2 * e + tg))) & 0xFFu;
+        const int sel = 2 * mt + tg, n = 2 * hf + e;
+        if constexpr (B == 4) {
+          w[sel >> 1] |= (c & 0xFu) << (16 * (sel & 1) + 4 * n);
+        } else {
+          const int G = sel >> 3, j = sel & 7;
+          if (j < 6) {
+            w[3 * G + (j >> 1)] |= (c & 7u) << (16 * (j & 1) + 4 * n);
+          } else {
+            const int bit = 4 * (4 * (j - 6) + n) + 3;
+            w[3 * G + 0] |= (c & 1u) << bit;
+            w[3 * G + 1] |= ((c >> 1) & 1u) << bit;
+            w[3 * G + 2] |= ((c >> 2) & 1u) << bit;
+          }
+        }
       }
-      load_row4(v, static_cast<size_t>(tok) * n_kv + h, dtype, lane, x);
-      quantize_vector(x, T.signs_v, s_tab + 32, s_tab + 48, T.value_bits, nullptr, false, lane, o);
-      store_value_token(sblk, tau, T.key_bits, T.value_bits, o, lane);
-      if (lane == 0) store_norm(sblk, T.key_bits, T.value_bits, 2, tau, o.norm);
+  }
+}
+
+// The lane's 32 coordinates of tokens g, g + 8 from the staged rows (zeros where
+// invalid), multiplied by the rotation signs; returns both tokens' squared
+// norms over all 128 coordinates. rows: the tile's 16 staged rows of K or V,
+// `pitch` bytes apart, elements of `dtype`.
+__device__ __forceinline__ void pf_load(const uint8_t* rows, int pitch, int dtype, int g, int t, bool ok0,
+                                        bool ok1, uint32_t dmask, float (&v)[2][32], float (&ss)[2]) {
+#pragma unroll
+  for (int th = 0; th < 2; ++th) {
+    const bool ok = th ? ok1 : ok0;
+    const uint8_t* row = rows + (g + 8 * th) * pitch;
+    float acc = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      float x[4];
+      if (dtype == TQ_F32) {
+        const float4 f = *reinterpret_cast<const float4*>(row + (16 * ks + 4 * t) * 4);
+        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+      } else {
+        const uint2 raw = *reinterpret_cast<const uint2*>(row + (16 * ks + 4 * t) * 2);
+        if (dtype == TQ_BF16) {
+          x[0] = __uint_as_float(raw.x << 16); x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+          x[2] = __uint_as_float(raw.y << 16); x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+        } else {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+          x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * ks + e;
+        const float xe = ok ? x[e] : 0.0f;
+        acc = fmaf(xe, xe, acc);
+        v[th][i] = __uint_as_float(__float_as_uint(xe) ^ (((dmask >> i) & 1u) << 31));
+      }
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < bb / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(gblk)[i] = reinterpret_cast<const uint4*>(sblk)[i];
+    acc += __shfl_xor_sync(kFull, acc, 1);
+    acc += __shfl_xor_sync(kFull, acc, 2);
+    ss[th] = acc;
+  }
+}
+
+// In-place natural-order Walsh-Hadamard transform of both tokens (unnormalised).
+__device__ __forceinline__ void pf_fwht(float (&v)[2][32], int lane) {
+#pragma unroll
+  for (int th = 0; th < 2; ++th)
+#pragma unroll
+    for (int bit = 0; bit < 5; ++bit)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (!(i & (1 << bit))) {
+          const float a = v[th][i], b = v[th][i | (1 << bit)];
+          v[th][i] = a + b;
+          v[th][i | (1 << bit)] = a - b;
+        }
+#pragma unroll
+  for (int m = 1; m <= 2; m <<= 1) {
+    const float sg = (lane & m) ? -1.0f : 1.0f;
+#pragma unroll
+    for (int th = 0; th < 2; ++th)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[th][i] = fmaf(v[th][i], sg, __shfl_xor_sync(kFull, v[th][i], m));
+  }
+}
+
+// Shared memory of the prefill kernel, per CTA of W warps: W value-transpose
+// tiles (2 KB), W x 2 half-stages (16 staged K rows, 16 staged V rows, pf_pitch
+// bytes apart), W x 2 barriers. A half-stage is refilled with the next tile's
+// rows as soon as its rows have been read, so copies overlap the arithmetic.
+__host__ __device__ constexpr int pf_pitch(int elem) { return 128 * elem + 32; }
+__host__ __device__ constexpr size_t pf_smem(int warps, int elem) {
+  return size_t(warps) * 2048 + size_t(warps) * 32 * pf_pitch(elem) + size_t(warps) * 2 * 8;
+}
+
+template <int BK, int BV>
+__global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, const void* k, const void* v,
+                                                                  int dtype, int n_tokens, int n_kv,
+                                                                  const int32_t* block_table, int start_pos,
+                                                                  uint8_t* cache, int64_t n_pages) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int W = blockDim.x >> 5;
+  const int elem = dtype == TQ_F32 ? 4 : 2;
+  const int pitch = pf_pitch(elem), rb = 128 * elem;
+  const uint2* qb = reinterpret_cast<const uint2*>(T.sketch_qb);            // [8 ks][16 nt][32 lane]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  uint8_t* vt = smem + warp * 2048;                                          // value transpose tile
+  uint8_t* stage0 = smem + W * 2048 + warp * 32 * pitch;                     // K rows, then V rows
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + W * 2048 + W * 32 * pitch) + warp * 2;
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  uint32_t dmk = 0u, dmv = 0u;                  // rotation sign bits of the lane's coordinates
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    dmk |= (T.signs_k[pf_coord(i, t)] < 0.0f ? 1u : 0u) << i;
+    dmv |= (T.signs_v[pf_coord(i, t)] < 0.0f ? 1u : 0u) << i;
+  }
+  float thk[16], cnk[16], thv[16], cnv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    thk[i] = T.thr_k[i]; cnk[i] = T.cen_k[i]; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
+  }
+  __syncwarp();
+  const int first_page = start_pos / kPage;
+  const int n_tiles = ((start_pos + n_tokens - 1) / kPage - first_page + 1) * n_kv;
+  const int bb = T.block_bytes;
+  const float kInvRootD = 0.08838834764831845f;   // 1 / sqrt(128)
+  const int stride = gridDim.x * W;
+
+  // Stage the 16 rows of K (kv = 0) or V (kv = 1) of `tile`: lane tau copies token
+  // tau's row when the token is in the run and the tile's page id is in range.
+  auto stage_rows = [&](int tile, int kv) {
+    const int lp = first_page + tile / n_kv, h = tile % n_kv;
+    const int phys = block_table[lp];
+    const bool good = phys >= 0 && phys < n_pages;
+    const int tau0 = max(start_pos - lp * kPage, 0), tau1 = min(start_pos + n_tokens - lp * kPage, kPage);
+    if (lane == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");    // earlier reads of these rows
+      mbar_expect_tx(bar + kv, good ? static_cast<unsigned>((tau1 - tau0) * rb) : 0u);
+    }
+    __syncwarp();
+    if (good && lane >= tau0 && lane < tau1) {
+      const int64_t row = static_cast<int64_t>(lp * kPage + lane - start_pos) * n_kv + h;
+      const uint8_t* src = static_cast<const uint8_t*>(kv ? v : k) + row * rb;
+      tma_load_1d(stage0 + (kv * 16 + lane) * pitch, src, rb, bar + kv);
+    }
+  };
+
+  int tile = blockIdx.x * W + warp;
+  if (tile < n_tiles) {
+    stage_rows(tile, 0);
+    stage_rows(tile, 1);
+  }
+  unsigned ph = 0;
+  bool alive = true;
+  for (; tile < n_tiles && alive; tile += stride, ph ^= 1u) {
+    const int next = tile + stride;
+    const int lp = first_page + tile / n_kv, h = tile % n_kv;
+    const int phys = block_table[lp];
+    const bool good = phys >= 0 && phys < n_pages;
+    if (!good && lane == 0) set_error(T.err, TQ_DEV_BAD_SLOT);
+    uint8_t* blk = cache + (static_cast<int64_t>(good ? phys : 0) * n_kv + h) * bb;
+    const int tau0 = max(start_pos - lp * kPage, 0), tau1 = min(start_pos + n_tokens - lp * kPage, kPage);
+    const bool full = tau0 == 0 && tau1 == kPage;
+    const bool ok0 = g >= tau0 && g < tau1, ok1 = g + 8 >= tau0 && g + 8 < tau1;
+
+#pragma unroll 1
+    for (int kv = 0; kv < 2; ++kv) {               // 0: keys, 1: values (one copy of the rotation code)
+    if (!mbar_wait(bar + kv, ph)) {
+      if (lane == 0) set_error(T.err, TQ_DEV_TIMEOUT);
+      // bounded: let the copies still in flight land before the rows are reused
+      // (kv = 0: this tile's K and V rows; kv = 1: its V rows and the next tile's K rows)
+      mbar_wait(bar + kv, ph);
+      if (kv == 0) mbar_wait(bar + 1, ph);
+      else if (next < n_tiles) mbar_wait(bar, ph ^ 1u);
+      alive = false;
+      break;
+    }
+    float vv[2][32], ss[2];
+    pf_load(stage0 + kv * 16 * pitch, pitch, dtype, g, t, ok0, ok1, kv ? dmv : dmk, vv, ss);
+    __syncwarp();                                  // the rows are read: refill with the next tile's
+    if (next < n_tiles) stage_rows(next, kv);
+    if (!good) continue;
+    pf_fwht(vv, lane);
+    if (kv == 0) {
+    // ---------------- keys: norm, codes, residual, z = S u, signs
+    float nk[2], uu[2] = {0.f, 0.f};
+    uint32_t kw[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+#pragma unroll
+    for (int th = 0; th < 2; ++th) {
+      nk[th] = sqrtf(ss[th]);
+      const float inv = nk[th] > 0.0f ? kInvRootD / nk[th] : 0.0f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float y = vv[th][i] * inv;
+        float chat;
+        const int c = cell_of<BK>(y, thk, cnk, chat);
+        put_key_code<BK>(kw[th], i, static_cast<uint32_t>(c));
+        const float u = y - chat;
+        uu[th] = fmaf(u, u, uu[th]);
+        vv[th][i] = u * 1024.0f;                  // u 2^10: well inside the fp16 range
+      }
+      uu[th] += __shfl_xor_sync(kFull, uu[th], 1);
+      uu[th] += __shfl_xor_sync(kFull, uu[th], 2);
+    }
+    // A fragments (fp16 high and low parts) of the residual tile
+    uint32_t ah[8][4], al[8][4];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int th = r & 1, i = 4 * ks + 2 * (r >> 1);
+        const float x0 = vv[th][i], x1 = vv[th][i + 1];
+        const __half2 hi = __floats2half2_rn(x0, x1);
+        const float2 hf = __half22float2(hi);
+        ah[ks][r] = *reinterpret_cast<const uint32_t*>(&hi);
+        al[ks][r] = pack_half2(x0 - hf.x, x1 - hf.y);
+      }
+    uint32_t sw[2] = {0u, 0u};
+#pragma unroll 1
+    for (int nt = 0; nt < 16; nt += 2) {             // two independent accumulator chains
+      float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint2 b0 = __ldg(qb + (ks * 16 + nt) * 32 + lane), b1 = __ldg(qb + (ks * 16 + nt + 1) * 32 + lane);
+        mma_f16(z0, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], b0.x, b0.y);
+        mma_f16(z1, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], b1.x, b1.y);
+        mma_f16(z0, al[ks][0], al[ks][1], al[ks][2], al[ks][3], b0.x, b0.y);
+        mma_f16(z1, al[ks][0], al[ks][1], al[ks][2], al[ks][3], b1.x, b1.y);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int th = r >> 1, j0 = 2 * nt + (r & 1), j1 = j0 + 2;   // lane-local sketch rows
+        sw[th] |= (z0[r] >= 0.0f ? 1u : 0u) << (8 * (j0 & 3) + (j0 >> 2));
+        sw[th] |= (z1[r] >= 0.0f ? 1u : 0u) << (8 * (j1 & 3) + (j1 >> 2));
+      }
+    }
+    {
+      uint32_t* kwd = reinterpret_cast<uint32_t*>(blk) + lane * 2 * BK;
+      uint32_t* swd = reinterpret_cast<uint32_t*>(blk + 256 * BK) + lane * 2;
+#pragma unroll
+      for (int th = 0; th < 2; ++th) {
+        if (!(th ? ok1 : ok0)) continue;
+#pragma unroll
+        for (int w = 0; w < BK; ++w) kwd[th * BK + w] = kw[th][w];
+        swd[th] = sw[th];
+      }
+      if (t == 0) {
+        __half* nrm = reinterpret_cast<__half*>(blk + 256 * (BK + BV + 1));
+        const float gk0 = nk[0] * sqrtf(uu[0]), gk1 = nk[1] * sqrtf(uu[1]);
+        if (ok0) { nrm[2 * g] = __float2half_rn(nk[0]); nrm[16 + 2 * g] = __float2half_rn(gk0); }
+        if (ok1) { nrm[2 * g + 1] = __float2half_rn(nk[1]); nrm[16 + 2 * g + 1] = __float2half_rn(gk1); }
+      }
+    }
+
+    } else {
+    // ---------------- values: norm, codes, transpose to value chunks
+    float nv[2];
+#pragma unroll
+    for (int th = 0; th < 2; ++th) nv[th] = sqrtf(ss[th]);
+    {
+      const float inv0 = nv[0] > 0.0f ? kInvRootD / nv[0] : 0.0f;
+      const float inv1 = nv[1] > 0.0f ? kInvRootD / nv[1] : 0.0f;
+      __syncwarp();                                            // the tile's previous readers are done
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float chat;
+        const int c0 = cell_of<BV>(vv[0][i] * inv0, thv, cnv, chat);
+        const int c1 = cell_of<BV>(vv[1][i] * inv1, thv, cnv, chat);
+        // tokens g, g + 8 sit at bytes 2g, 2g + 1 of the coordinate's 16-byte row
+        *reinterpret_cast<uint16_t*>(vt + pf_coord(i, t) * 16 + 2 * g) =
+            static_cast<uint16_t>(c0 | (c1 << 8));
+      }
+      __syncwarp();
+    }
+    {
+      // value chunk of this lane: coordinates g + 8 hf + 16 mt, tokens 2t + e + 8 tg
+      uint32_t vw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, vm[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      const bool tv[4] = {2 * t >= tau0 && 2 * t < tau1, 2 * t + 8 >= tau0 && 2 * t + 8 < tau1,
+                          2 * t + 1 >= tau0 && 2 * t + 1 < tau1, 2 * t + 9 >= tau0 && 2 * t + 9 < tau1};
+      const uint32_t maskx = (tv[0] ? 0xFFu : 0u) | (tv[1] ? 0xFF00u : 0u) | (tv[2] ? 0xFF0000u : 0u) |
+                             (tv[3] ? 0xFF000000u : 0u);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t x = *reinterpret_cast<const uint32_t*>(vt + (g + 8 * hf + 16 * mt) * 16 + 4 * t);
+          put_value_codes<BV>(vw, mt, hf, x & maskx);
+          if (!full) put_value_codes<BV>(vm, mt, hf, maskx);
+        }
+      uint32_t* vwd = reinterpret_cast<uint32_t*>(blk + 256 * (BK + 1)) + lane * 2 * BV;
+#pragma unroll
+      for (int w = 0; w < 2 * BV; ++w) vwd[w] = full ? vw[w] : ((vwd[w] & ~vm[w]) | vw[w]);
+      if (t == 0) {
+        __half* nrm = reinterpret_cast<__half*>(blk + 256 * (BK + BV + 1));
+        if (ok0) nrm[32 + 2 * g] = __float2half_rn(nv[0]);
+        if (ok1) nrm[32 + 2 * g + 1] = __float2half_rn(nv[1]);
+      }
+    }
+    }
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar + 1)) : "memory");
   }
 }
 
@@ -460,41 +838,6 @@ struct DecodeWarps { static constexpr int value = NH == 1 ? 16 : 8; };
 __host__ __device__ constexpr int decode_stages(int warps, int block) { return warps * 6 * block <= 160 * 1024 ? 6 : 4; }
 constexpr int kStatic = 2;       // pages per warp assigned before the block-table window is cached
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: gives up after ~2^31 clock cycles (about a second).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > (1ll << 31)) return false;
-  }
-  return true;
-}
-__device__ __forceinline__ void tma_load_1d(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
 
 // ---- code words -> mma operands --------------------------------------------
 // Key selectors: 8 selectors (one per B register of the 4 k-tiles), each four
@@ -1465,16 +1808,54 @@ cudaError_t launch_quantize_append(const Tables& t, const void* k, const void* v
   return cudaGetLastError();
 }
 
+template <int BK, int BV>
+cudaError_t launch_prefill_t(const Tables& t, const void* k, const void* v, int dtype, int n_tokens, int n_kv,
+                             const int32_t* block_table, int start_pos, void* cache, int64_t n_pages,
+                             cudaStream_t s) {
+  const int first = start_pos / kPage, last = (start_pos + n_tokens - 1) / kPage;
+  const int tiles = (last - first + 1) * n_kv;
+  const int elem = dtype == TQ_F32 ? 4 : 2;
+  const int warps = 8;
+  int blocks = (tiles + warps - 1) / warps;
+  const size_t smem = pf_smem(warps, elem);
+  auto fn = quantize_prefill_kernel<BK, BV>;
+  // grid limit = resident CTAs, worked out once per instantiation and shared-memory size
+  static size_t configured = 0;
+  static int max_blocks = 0;
+  if (configured != smem) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    max_blocks = sms * per_sm;
+    configured = smem;
+  }
+  if (blocks > max_blocks) blocks = max_blocks;
+  fn<<<blocks, warps * 32, smem, s>>>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos,
+                                      static_cast<uint8_t*>(cache), n_pages);
+  return cudaGetLastError();
+}
+
+template <int BK>
+cudaError_t prefill_bv(const Tables& t, const void* k, const void* v, int dtype, int n_tokens, int n_kv,
+                       const int32_t* bt, int start_pos, void* cache, int64_t n_pages, cudaStream_t s) {
+  switch (t.value_bits) {
+    case 2: return launch_prefill_t<BK, 2>(t, k, v, dtype, n_tokens, n_kv, bt, start_pos, cache, n_pages, s);
+    case 3: return launch_prefill_t<BK, 3>(t, k, v, dtype, n_tokens, n_kv, bt, start_pos, cache, n_pages, s);
+    default: return launch_prefill_t<BK, 4>(t, k, v, dtype, n_tokens, n_kv, bt, start_pos, cache, n_pages, s);
+  }
+}
+
 cudaError_t launch_quantize_prefill(const Tables& t, const void* k, const void* v, int dtype, int n_tokens,
                                     int n_kv, const int32_t* block_table, int start_pos, void* cache,
                                     int64_t n_pages, cudaStream_t s) {
-  const int first = start_pos / kPage, last = (start_pos + n_tokens - 1) / kPage;
-  const int jobs = (last - first + 1) * n_kv;
-  const int blocks = jobs < 148 * 2 ? jobs : 148 * 2;
-  const size_t smem = kHeadDim * kQjlRows * 2 + t.block_bytes;
-  quantize_prefill_kernel<<<blocks, 256, smem, s>>>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos,
-                                                    static_cast<uint8_t*>(cache), n_pages);
-  return cudaGetLastError();
+  switch (t.key_bits) {
+    case 2: return prefill_bv<2>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
+    case 3: return prefill_bv<3>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
+    default: return prefill_bv<4>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
+  }
 }
 
 cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype,

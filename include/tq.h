@@ -114,7 +114,9 @@ tq_status tq_quantize_append(tq_ctx* ctx, const void* k, const void* v, tq_dtype
  * one): logical positions [start_pos, start_pos + n_tokens) go to the pages
  * named by block_table (device int32 [>= ceil((start_pos+n_tokens)/16)]).
  * Same arithmetic as tq_quantize_append; whole pages are written with full-width
- * stores, partial pages are merged with what they already hold.
+ * stores, partial pages are merged with what they already hold. k and v must be
+ * 16-byte aligned (their rows are staged in shared memory by bulk copies);
+ * otherwise TQ_ERR_INVALID_ARG.
  */
 tq_status tq_quantize_prefill(tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
                               int n_tokens, int n_kv_heads, const int32_t* block_table,
