@@ -131,6 +131,8 @@ class ClockSampler:
 
 # ------------------------------------------------------------- GPU workload
 class DecodeBench:
+    L2_BYTES = 126e6
+
     def __init__(self, wl, steps, warmup, device, rank):
         import torch
         from decode_attention_seeded_b200 import binding, synth
@@ -140,49 +142,50 @@ class DecodeBench:
         gen0 = synth.Generator(wl, layer=0)
         self.seeds = gen0.method_seeds()
         self.ctx = binding.Context(wl.key_bits, wl.value_bits, self.seeds, device=device.index)
-        self.n_layers = wl.n_layers
-        self.T0 = wl.context
-        self.total_steps = warmup + steps
-        self.max_len = self.T0 + self.total_steps
-        self.pages = (self.max_len + 15) // 16
         n_kv, nq, B = wl.n_kv_heads, wl.n_q_heads, wl.batch
-        assert B == 1
+        self.lens0 = gen0.seq_lens().astype(np.int64)            # cached tokens per sequence before step 0
+        self.T0 = int(self.lens0[0])
+        self.total_steps = warmup + steps
+        self.max_len = int(self.lens0.max()) + self.total_steps
+        pages = (self.lens0 + self.total_steps + 15) // 16
+        bpt = self.ctx.block_bytes // 16
+        per_layer = int(np.sum(self.lens0)) * n_kv * bpt
+        # rotate through enough layer caches that they exceed the L2 several times over
+        self.n_layers = max(wl.n_layers, min(64, int(np.ceil(4 * self.L2_BYTES / per_layer))))
         self.page_bytes = self.ctx.page_bytes(n_kv)
-        self.caches, self.btabs, self.slots = [], [], []
+        self.caches, self.btabs = [], []
         g = torch.Generator(device=device)
+        self.newk = torch.empty((self.n_layers, self.total_steps, B, n_kv, 128), dtype=torch.bfloat16,
+                                device=device)
+        self.newv = torch.empty_like(self.newk)
         for layer in range(self.n_layers):
             gen = synth.Generator(wl, layer=layer)
-            bt, n_pages = gen.page_pool(np.array([self.pages]))
+            bt, n_pages = gen.page_pool(pages)
             cache = torch.empty(n_pages * self.page_bytes, dtype=torch.uint8, device=device)
             btt = torch.from_numpy(bt).to(device)
             g.manual_seed(wl.seed * 1000 + layer + 7919 * rank)
-            for which, name in (("k", "k"), ("v", "v")):
-                sc = torch.from_numpy(gen.scales[which]).float().to(device)
-                x = (torch.randn((self.T0 + self.total_steps, n_kv, 128), generator=g, device=device) * sc)
-                x = x.to(torch.bfloat16)
-                setattr(self, "_" + name, x)
-            self.ctx.quantize_prefill(self._k[:self.T0], self._v[:self.T0], btt[0], 0, cache, n_pages)
-            sl = synth.slots_for(bt[0], self.T0, self.total_steps)
-            self.slots.append(torch.from_numpy(sl).to(device))
-            if layer == 0:
-                self.newk = torch.empty((self.n_layers, self.total_steps, n_kv, 128), dtype=torch.bfloat16,
-                                        device=device)
-                self.newv = torch.empty_like(self.newk)
-            self.newk[layer] = self._k[self.T0:]
-            self.newv[layer] = self._v[self.T0:]
-            del self._k, self._v
+            sk = torch.from_numpy(gen.scales["k"]).float().to(device)
+            sv = torch.from_numpy(gen.scales["v"]).float().to(device)
+            for b in range(B):
+                L = int(self.lens0[b])
+                k = (torch.randn((L + self.total_steps, n_kv, 128), generator=g, device=device) * sk).to(torch.bfloat16)
+                v = (torch.randn((L + self.total_steps, n_kv, 128), generator=g, device=device) * sv).to(torch.bfloat16)
+                self.ctx.quantize_prefill(k[:L], v[:L], btt[b], 0, cache, n_pages)
+                self.newk[layer, :, b] = k[L:]
+                self.newv[layer, :, b] = v[L:]
+                del k, v
             self.caches.append((cache, n_pages))
             self.btabs.append(btt)
         torch.cuda.synchronize(device)
         self.q = (torch.randn((self.total_steps, self.n_layers, B, nq, 128), generator=g, device=device)
                   .to(torch.bfloat16))
-        self.lens = torch.arange(self.T0 + 1, self.T0 + self.total_steps + 1, dtype=torch.int32,
-                                 device=device).reshape(-1, 1)
+        steps_ar = torch.arange(1, self.total_steps + 1, dtype=torch.int64).reshape(-1, 1)
+        self.lens = (torch.from_numpy(self.lens0).reshape(1, -1) + steps_ar).to(torch.int32).to(device)
         self.out = torch.zeros((self.n_layers, B, nq, 128), dtype=torch.float32, device=device)
         self.ws_bytes = self.ctx.decode_workspace_bytes(B, nq, n_kv, self.max_len)
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=device)
         # host-side buffers for the end-to-end arm
-        self.h_newk = torch.empty((self.total_steps, self.n_layers, n_kv, 128), dtype=torch.bfloat16,
+        self.h_newk = torch.empty((self.total_steps, self.n_layers, B, n_kv, 128), dtype=torch.bfloat16,
                                   pin_memory=True)
         self.h_newv = torch.empty_like(self.h_newk, pin_memory=True)
         self.h_q = torch.empty((self.total_steps, self.n_layers, B, nq, 128), dtype=torch.bfloat16,
@@ -192,16 +195,21 @@ class DecodeBench:
         self.h_q.copy_(self.q.cpu())
         self.h_out = torch.empty((self.total_steps, self.n_layers, B, nq, 128), dtype=torch.float32,
                                  pin_memory=True)
-        self.d_stepk = torch.empty((self.n_layers, n_kv, 128), dtype=torch.bfloat16, device=device)
+        self.d_stepk = torch.empty((self.n_layers, B, n_kv, 128), dtype=torch.bfloat16, device=device)
         self.d_stepv = torch.empty_like(self.d_stepk)
         self.d_stepq = torch.empty((self.n_layers, B, nq, 128), dtype=torch.bfloat16, device=device)
+
+    @property
+    def cache_tokens(self):
+        """Cached tokens read by one decode call at the final step (all sequences)."""
+        return int(np.sum(self.lens0)) + self.wl.batch * self.total_steps
 
     # one decode step (all layers) with inputs already on the device
     def step(self, s):
         wl = self.wl
         for layer in range(self.n_layers):
             cache, n_pages = self.caches[layer]
-            self.ctx.decode_step(self.newk[layer, s:s + 1], self.newv[layer, s:s + 1], self.q[s, layer], cache,
+            self.ctx.decode_step(self.newk[layer, s], self.newv[layer, s], self.q[s, layer], cache,
                                  n_pages, self.btabs[layer], self.lens[s], wl.n_kv_heads, self.max_len,
                                  self.out[layer], self.ws)
 
@@ -213,7 +221,7 @@ class DecodeBench:
         self.d_stepq.copy_(self.h_q[s], non_blocking=True)
         for layer in range(self.n_layers):
             cache, n_pages = self.caches[layer]
-            self.ctx.decode_step(self.d_stepk[layer:layer + 1], self.d_stepv[layer:layer + 1], self.d_stepq[layer],
+            self.ctx.decode_step(self.d_stepk[layer], self.d_stepv[layer], self.d_stepq[layer],
                                  cache, n_pages, self.btabs[layer], self.lens[s], wl.n_kv_heads, self.max_len,
                                  self.out[layer], self.ws)
         self.h_out[s].copy_(self.out, non_blocking=True)
@@ -221,7 +229,7 @@ class DecodeBench:
     def e2e_bytes(self):
         e = 2
         wl = self.wl
-        h2d = self.n_layers * (2 * wl.n_kv_heads * 128 * e + wl.batch * wl.n_q_heads * 128 * e)
+        h2d = self.n_layers * wl.batch * (2 * wl.n_kv_heads * 128 * e + wl.n_q_heads * 128 * e)
         d2h = self.n_layers * wl.batch * wl.n_q_heads * 128 * 4
         return h2d, d2h
 
@@ -271,6 +279,65 @@ class DecodeBench:
         return {"gbs": (bytes_in + bytes_out) / secs / 1e9, "us_per_call": secs * 1e6,
                 "tokens": self.T0, "kv_heads": n_kv, "bytes_in": bytes_in, "bytes_out": bytes_out,
                 "kernel": "quantize_prefill_kernel via tq_quantize_prefill (bf16 K/V, one layer)"}
+
+    def bf16_baseline(self, reps=3):
+        """Decode attention over an uncompressed bf16 KV cache of the same shape (context only).
+
+        The faster of flash-attention's KV-cache decode and PyTorch SDPA (GQA), timed
+        over the same number of layer caches as the compressed path, so that the
+        caches stream from HBM. Library kernels: a comparison point, not this path."""
+        torch, wl = self.torch, self.wl
+        n_kv, nq, T, B = wl.n_kv_heads, wl.n_q_heads, self.max_len, wl.batch
+        g = torch.Generator(device=self.dev)
+        g.manual_seed(99)
+        layers = self.n_layers
+        kc = [torch.randn((B, T, n_kv, 128), generator=g, device=self.dev).to(torch.bfloat16) for _ in range(layers)]
+        vc = [torch.randn((B, T, n_kv, 128), generator=g, device=self.dev).to(torch.bfloat16) for _ in range(layers)]
+        q = torch.randn((B, 1, nq, 128), generator=g, device=self.dev).to(torch.bfloat16)
+        lens = self.lens[-1]                          # final step's lengths (int32, per sequence)
+        ragged = bool((lens != lens[0]).any())
+        st = torch.cuda.current_stream(self.dev)
+        results, errors = {}, {}
+
+        def time_it(fn):
+            fn(0)
+            torch.cuda.synchronize(self.dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            for _ in range(reps):
+                for layer in range(layers):
+                    fn(layer)
+            b.record(st)
+            b.synchronize()
+            return a.elapsed_time(b) / 1e3 / (reps * layers)
+
+        try:
+            from flash_attn import __version__ as fav
+            from flash_attn import flash_attn_with_kvcache
+            results[f"flash_attn {fav} flash_attn_with_kvcache"] = time_it(
+                lambda l: flash_attn_with_kvcache(q, kc[l], vc[l], cache_seqlens=lens))
+        except Exception as e:                       # library kernel unavailable on this build
+            errors["flash_attn"] = repr(e)[:200]
+        try:
+            if ragged:
+                raise ValueError("ragged lengths: SDPA would attend the padding")
+            import torch.nn.functional as F
+            qs = q.transpose(1, 2)                   # [B, nq, 1, 128]
+            kt = [k.transpose(1, 2) for k in kc]
+            vt = [v.transpose(1, 2) for v in vc]
+            results[f"torch {torch.__version__} scaled_dot_product_attention (enable_gqa)"] = time_it(
+                lambda l: F.scaled_dot_product_attention(qs, kt[l], vt[l], enable_gqa=True))
+        except Exception as e:
+            errors["sdpa"] = repr(e)[:200]
+        del kc, vc
+        torch.cuda.empty_cache()
+        if not results:
+            return {"unavailable": errors}
+        name, secs = min(results.items(), key=lambda kv: kv[1])
+        nbytes = 2 * int(lens.sum().item()) * n_kv * 128 * 2
+        return {"kernel": name, "us_per_layer": secs * 1e6, "bytes_per_layer": nbytes,
+                "gbs": nbytes / secs / 1e9, "all_us": {k: v * 1e6 for k, v in results.items()},
+                "errors": errors or None}
 
     def decode_only_graph(self, reps):
         """reps x (32 layers of tq_decode_attention) at the final context length."""
@@ -455,12 +522,12 @@ def main():
     dec_s = t_dec / n_dec
     assert bench.ctx.device_error() == 0
 
+    base16 = bench.bf16_baseline()
     quant = bench.quantize_timing()
     quant["frac"] = quant["gbs"] / load_peaks()[0]
     peak, peak_kind = load_peaks()
     bpt = bench.ctx.block_bytes // 16                     # bytes per token-head (102 for 3/2 bits)
-    ctx_len = bench.max_len
-    alg_bytes = bpt * ctx_len * wl.n_kv_heads * wl.batch
+    alg_bytes = bpt * bench.cache_tokens * wl.n_kv_heads
     achieved = alg_bytes / dec_s / 1e9
     traffic = recorded_traffic("bytes_per_launch")
 
@@ -470,20 +537,25 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": t_main / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8/fp16 tensor-core, fp32 accumulate (3-bit keys + QJL, 2-bit values)",
+        "dtype": f"int8/fp16 tensor-core, fp32 accumulate ({wl.key_bits}-bit keys + QJL, {wl.value_bits}-bit values)",
         "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
-                   "head_dim": 128, "context": wl.context, "layers": wl.n_layers, "key_bits": wl.key_bits,
+                   "head_dim": 128, "context": wl.context, "context_lens": [int(x) for x in bench.lens0[:16]],
+                   "layers": bench.n_layers, "key_bits": wl.key_bits,
                    "value_bits": wl.value_bits, "qjl_rows": 128, "page_tokens": 16,
                    "l2": f"inputs larger than L2: {bench.n_layers} layer caches, "
                          f"{bench.n_layers * bench.caches[0][1] * bench.page_bytes / 1e9:.2f} GB per step",
-                   "parallelism": f"replica x{world} (one sequence per GPU)"},
+                   "parallelism": f"replica x{world} (each GPU serves its own batch)"},
         "e2e": {"value": job_throughput(K * wl.batch, world, t_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                      "kernel": "decode_kernel via tq_decode_attention (query transform, split-K decode, merge)",
                      "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
         "quantize": quant,
+        "bf16_baseline": dict(base16, **({"compressed_us_per_layer": dec_s * 1e6,
+                                          "speedup_vs_bf16": base16["us_per_layer"] / (dec_s * 1e6),
+                                          "cache_bytes_ratio": base16["bytes_per_layer"] / alg_bytes}
+                                         if "us_per_layer" in base16 else {})),
         "gpu_launches": K * bench.n_layers,
         "clocks": clocks,
     }
