@@ -1592,15 +1592,17 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       part[hh * 132 + 129] = l;
     }
   }
-  __threadfence();
+  // Publish the record: the barrier orders every thread's stores before thread 0's
+  // acquire-release increment at GPU scope (release is cumulative over what
+  // happens before it), and the CTA that takes the last ticket acquires all records.
   __syncthreads();
   if (threadIdx.x == 0) {
-    const unsigned ticket = atomicAdd(A.counters + pair, 1u);
+    unsigned ticket;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(A.counters + pair) : "memory");
     s_last = (ticket == static_cast<unsigned>(A.chunks - 1)) ? 1 : 0;
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   if (threadIdx.x == 0) A.counters[pair] = 0u;    // every CTA has counted: ready for the next call
 
   // ---- last CTA of this (sequence, KV head): merge the chunks, de-rotate, store.
