@@ -133,7 +133,7 @@ class ClockSampler:
 class DecodeBench:
     L2_BYTES = 126e6
 
-    def __init__(self, wl, steps, warmup, device, rank):
+    def __init__(self, wl, steps, warmup, device, rank, sparse_v=0.0, peaked=False):
         import torch
         from decode_attention_seeded_b200 import binding, synth
         self.torch, self.binding, self.synth = torch, binding, synth
@@ -142,6 +142,7 @@ class DecodeBench:
         gen0 = synth.Generator(wl, layer=0)
         self.seeds = gen0.method_seeds()
         self.ctx = binding.Context(wl.key_bits, wl.value_bits, self.seeds, device=device.index)
+        self.ctx.set_sparse_v(sparse_v)
         n_kv, nq, B = wl.n_kv_heads, wl.n_q_heads, wl.batch
         self.lens0 = gen0.seq_lens().astype(np.int64)            # cached tokens per sequence before step 0
         self.T0 = int(self.lens0[0])
@@ -158,6 +159,8 @@ class DecodeBench:
         self.newk = torch.empty((self.n_layers, self.total_steps, B, n_kv, 128), dtype=torch.bfloat16,
                                 device=device)
         self.newv = torch.empty_like(self.newk)
+        self.q = (torch.randn((self.total_steps, self.n_layers, B, nq, 128), generator=g, device=device)
+                  .to(torch.bfloat16))
         for layer in range(self.n_layers):
             gen = synth.Generator(wl, layer=layer)
             bt, n_pages = gen.page_pool(pages)
@@ -173,12 +176,18 @@ class DecodeBench:
                 self.ctx.quantize_prefill(k[:L], v[:L], btt[b], 0, cache, n_pages)
                 self.newk[layer, :, b] = k[L:]
                 self.newv[layer, :, b] = v[L:]
+                if peaked:
+                    # concentrated attention: each query is 5 x the sum of the unit
+                    # directions of 3 cached keys of its KV head
+                    idx = torch.randint(0, L, (self.total_steps, nq, 3), generator=g, device=device)
+                    hk = (torch.arange(nq, device=device) // (nq // n_kv)).view(1, nq, 1).expand_as(idx)
+                    kk = k[idx, hk].float()
+                    kk = kk / kk.norm(dim=-1, keepdim=True)
+                    self.q[:, layer, b] = (5.0 * kk.sum(dim=2)).to(torch.bfloat16)
                 del k, v
             self.caches.append((cache, n_pages))
             self.btabs.append(btt)
         torch.cuda.synchronize(device)
-        self.q = (torch.randn((self.total_steps, self.n_layers, B, nq, 128), generator=g, device=device)
-                  .to(torch.bfloat16))
         steps_ar = torch.arange(1, self.total_steps + 1, dtype=torch.int64).reshape(-1, 1)
         self.lens = (torch.from_numpy(self.lens0).reshape(1, -1) + steps_ar).to(torch.int32).to(device)
         self.out = torch.zeros((self.n_layers, B, nq, 128), dtype=torch.float32, device=device)
@@ -445,6 +454,10 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-budget", type=float, default=12.0)
+    ap.add_argument("--sparse-v", type=float, default=0.0,
+                    help="Sparse V threshold (relative attention weight; 0 = dense)")
+    ap.add_argument("--peaked", action="store_true",
+                    help="queries built from a few cached keys each (concentrated attention)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -484,7 +497,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
-    bench = DecodeBench(wl, args.steps, args.warmup, dev, rank)
+    bench = DecodeBench(wl, args.steps, args.warmup, dev, rank, sparse_v=args.sparse_v, peaked=args.peaked)
     W, K = args.warmup, args.steps
     g_warm = bench.capture(bench.step, range(W))
     g_main = bench.capture(bench.step, range(W, W + K))
@@ -545,7 +558,9 @@ def main():
                    "value_bits": wl.value_bits, "qjl_rows": 128, "page_tokens": 16,
                    "l2": f"inputs larger than L2: {bench.n_layers} layer caches, "
                          f"{bench.n_layers * bench.caches[0][1] * bench.page_bytes / 1e9:.2f} GB per step",
-                   "parallelism": f"replica x{world} (each GPU serves its own batch)"},
+                   "parallelism": f"replica x{world} (each GPU serves its own batch)",
+                   "sparse_v": args.sparse_v, "queries": "peaked (5 x 3 cached key directions)" if args.peaked
+                   else "N(0,1)"},
         "e2e": {"value": job_throughput(K * wl.batch, world, t_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,

@@ -48,6 +48,7 @@ _SIGS = {
     "tq_decode_attention_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int64,
                                                _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int,
                                                _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p]),
+    "tq_set_sparse_v": (_c.c_int, [_c.c_void_p, _c.c_float]),
     "tq_get_device_error": (_c.c_int, [_c.c_void_p, _c.POINTER(_c.c_uint32), _c.c_void_p]),
     "tq_host_sign_vector": (_c.c_int, [_c.c_uint64, _c.c_int, _c.c_void_p]),
     "tq_host_gaussian_sketch": (_c.c_int, [_c.c_uint64, _c.c_int, _c.c_int, _c.c_void_p]),
@@ -192,6 +193,10 @@ class Context:
             self._h, _ptr(q), _dtype_code(q), _ptr(cache), n_cache_pages, _ptr(block_tables),
             block_tables.shape[1], _ptr(seq_lens), batch, n_q, n_kv_heads, max_seq_len, scale, _ptr(out),
             _stream(stream)))
+
+    def set_sparse_v(self, tau: float):
+        """Sparse V threshold of later decode calls (0: dense attention)."""
+        _check("tq_set_sparse_v", lib().tq_set_sparse_v(self._h, tau))
 
     def device_error(self, stream=None) -> int:
         code = ctypes.c_uint32(0)

@@ -197,6 +197,7 @@ StoredCodebook make_codebook(int bits, int d) {
 struct tq_ctx {
   int device = 0;
   int sm_count = 0;                // streaming multiprocessors of the device (sizes decode grids)
+  float sparse_tau = 0.0f;         // Sparse V threshold of the decode calls (0: dense)
   bool rot_ready = false, cb_ready = false;
   float* d_signs = nullptr;        // [2][128]: D_K then D_V
   uint16_t* d_sketch_t = nullptr;  // fp16 bits: S^T, S as decode A fragments, S as prefill B fragments
@@ -567,7 +568,8 @@ tq_status tq_decode_attention(tq_ctx* ctx, const void* q, tq_dtype q_dtype, cons
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
   return from_cuda(tq::launch_decode(ctx->tables, plan, q, q_dtype, cache, n_cache_pages,
                                      block_tables, max_pages_per_seq, seq_lens, max_seq_len,
-                                     scale, out, workspace, static_cast<cudaStream_t>(stream)));
+                                     scale, out, workspace, ctx->sparse_tau,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_dtype kv_dtype,
@@ -588,7 +590,8 @@ tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_d
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
   return from_cuda(tq::launch_decode_step(ctx->tables, plan, k_new, v_new, kv_dtype, q, q_dtype, cache,
                                           n_cache_pages, block_tables, max_pages_per_seq, seq_lens, max_seq_len,
-                                          scale, out, workspace, static_cast<cudaStream_t>(stream)));
+                                          scale, out, workspace, ctx->sparse_tau,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
@@ -620,7 +623,14 @@ tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dty
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
   return from_cuda(tq::launch_decode(ctx->tables, plan, q, q_dtype, cache, n_cache_pages,
                                      block_tables, max_pages_per_seq, seq_lens, max_seq_len,
-                                     scale, out, scratch, static_cast<cudaStream_t>(stream)));
+                                     scale, out, scratch, ctx->sparse_tau,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+tq_status tq_set_sparse_v(tq_ctx* ctx, float tau) {
+  if (!ctx || !(tau >= 0.0f) || !(tau <= 1.0f)) return TQ_ERR_INVALID_ARG;
+  ctx->sparse_tau = tau;
+  return TQ_OK;
 }
 
 tq_status tq_get_device_error(tq_ctx* ctx, uint32_t* code, tq_stream stream) {

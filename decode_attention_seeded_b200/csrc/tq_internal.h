@@ -57,12 +57,13 @@ cudaError_t launch_quantize_prefill(const Tables& t, const void* k, const void* 
 cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype,
                           const void* cache, int64_t n_pages, const int32_t* block_tables,
                           int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len,
-                          float scale, float* out, void* workspace, cudaStream_t s);
+                          float scale, float* out, void* workspace, float sparse_tau, cudaStream_t s);
 
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, const void* q, int q_dtype, void* cache, int64_t n_pages,
                                const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
-                               int max_seq_len, float scale, float* out, void* workspace, cudaStream_t s);
+                               int max_seq_len, float scale, float* out, void* workspace, float sparse_tau,
+                               cudaStream_t s);
 
 // Device address (current device) of the fixed decode scratch used by
 // tq_decode_attention_noalloc; kNoAllocScratchBytes bytes, 256-byte aligned.

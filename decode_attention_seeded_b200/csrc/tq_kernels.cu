@@ -973,6 +973,8 @@ struct DecodeArgs {
   float* out;                    // [batch][n_q][128]
   int n_kv, n_q, group, n_hg, chunks, ppc, n_pairs;
   int merge_cap;                 // chunk records that fit in shared memory for the final merge
+  int sparse;                    // Sparse V on: values of positions below the threshold are skipped
+  float sparse_log2;             // log2 of the Sparse V threshold (relative attention weight)
 };
 
 // Shared-memory scratch of the prologue (after the stages and barriers).
@@ -1373,9 +1375,9 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[h][mt][c] = 0.0f;
-  float lsum[NH], mp2[NH];
+  float lsum[NH], mp2[NH], smx[NH];           // smx: running maximum of l2 (Sparse V only)
 #pragma unroll
-  for (int h = 0; h < NH; ++h) { lsum[h] = 0.0f; mp2[h] = kNegBig; }
+  for (int h = 0; h < NH; ++h) { lsum[h] = 0.0f; mp2[h] = kNegBig; smx[h] = kNegBig; }
 
   // transpose sources for the value-product B operand (see below)
   const int h4 = g & 3;
@@ -1456,6 +1458,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     const float lgv0 = lg2(fmaxf(nV.x, 5.9604645e-8f)), lgv1 = lg2(fmaxf(nV.y, 5.9604645e-8f));
     const float rnv0 = ex2(-lgv0), rnv1 = ex2(-lgv1);
     uint32_t pb[NH][2];
+    bool kept = false;                      // Sparse V: this lane keeps a (token, head) value
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
       float lp2[2];
@@ -1488,8 +1491,24 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
           acc[h][mt][0] *= f0; acc[h][mt][1] *= f1; acc[h][mt][2] *= f0; acc[h][mt][3] *= f1;
         }
       }
-      const float w0 = ex2(lp2[0] - mp2[h]), w1 = ex2(lp2[1] - mp2[h]);
+      float w0 = ex2(lp2[0] - mp2[h]), w1 = ex2(lp2[1] - mp2[h]);
       lsum[h] = fmaf(w0, rnv0, fmaf(w1, rnv1, lsum[h]));
+      if (A.sparse) {
+        // Sparse V: a value is skipped when its attention weight is below the
+        // threshold times the largest weight seen so far by this warp (never more
+        // than the largest overall); the denominator above still counts it.
+        const float l20 = lp2[0] - lgv0, l21 = lp2[1] - lgv1;
+        float ps = fmaxf(l20, l21);
+        ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 4));
+        ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 8));
+        ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 16));
+        smx[h] = fmaxf(smx[h], ps);
+        const float cut = smx[h] + A.sparse_log2;
+        const bool k0 = l20 >= cut, k1 = l21 >= cut;
+        w0 = k0 ? w0 : 0.0f;
+        w1 = k1 ? w1 : 0.0f;
+        kept = kept || k0 || k1;
+      }
       // weights of (token g, head t) and (token g+8, head t): high fp16 parts and residuals
       const __half2 whi = __floats2half2_rn(w0, w1);
       const float2 wr = __half22float2(whi);
@@ -1507,15 +1526,18 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     }
 
     // ---- weighted value sum in the rotated domain: fp16 tensor-core products
-    uint32_t vs[16];
-    value_selectors<BV>(vw, vs);
+    // (Sparse V: skipped for a page whose values are all below the threshold)
+    if (!A.sparse || __any_sync(kFull, kept)) {
+      uint32_t vs[16];
+      value_selectors<BV>(vw, vs);
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      uint32_t a0, a1, a2, a3;
-      value_regs<BV>(vs[2 * mt], vlo_, vhi_, a0, a1);
-      value_regs<BV>(vs[2 * mt + 1], vlo_, vhi_, a2, a3);
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        value_regs<BV>(vs[2 * mt], vlo_, vhi_, a0, a1);
+        value_regs<BV>(vs[2 * mt + 1], vlo_, vhi_, a2, a3);
 #pragma unroll
-      for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pb[h][0], pb[h][1]);
+        for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pb[h][0], pb[h][1]);
+      }
     }
 
     // ---- refill this stage with the pending claim (all its reads are consumed),
@@ -1768,7 +1790,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float scale, const void* cache,
                        int64_t n_pages, const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
-                       int max_seq_len, float* out, void* workspace) {
+                       int max_seq_len, float* out, void* workspace, float sparse_tau) {
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeArgs a{};
   a.q = q;
@@ -1790,6 +1812,8 @@ DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float
   a.chunks = plan.chunks;
   a.ppc = plan.pages_per_chunk;
   a.n_pairs = plan.n_pairs;
+  a.sparse = sparse_tau > 0.0f ? 1 : 0;
+  a.sparse_log2 = sparse_tau > 0.0f ? log2f(sparse_tau) : 0.0f;
   return a;
 }
 
@@ -1863,18 +1887,19 @@ cudaError_t launch_quantize_prefill(const Tables& t, const void* k, const void* 
 cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype,
                           const void* cache, int64_t n_pages, const int32_t* block_tables,
                           int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len, float scale,
-                          float* out, void* workspace, cudaStream_t s) {
+                          float* out, void* workspace, float sparse_tau, cudaStream_t s) {
   const DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq,
-                                   seq_lens, max_seq_len, out, workspace);
+                                   seq_lens, max_seq_len, out, workspace, sparse_tau);
   return dispatch_bk<false>(t, a, dim3(plan.chunks * plan.n_pairs), s);
 }
 
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, const void* q, int q_dtype, void* cache, int64_t n_pages,
                                const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,
-                               int max_seq_len, float scale, float* out, void* workspace, cudaStream_t s) {
+                               int max_seq_len, float scale, float* out, void* workspace, float sparse_tau,
+                               cudaStream_t s) {
   DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq, seq_lens,
-                             max_seq_len, out, workspace);
+                             max_seq_len, out, workspace, sparse_tau);
   a.k_new = k_new;
   a.v_new = v_new;
   a.kv_dtype = kv_dtype;

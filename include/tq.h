@@ -172,6 +172,22 @@ tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_d
                          void* workspace, size_t workspace_bytes, tq_stream stream);
 
 /*
+ * Sparse V (wis-web.com llama.cpp-fork post, third finding: decoding that skips
+ * the V positions with a low attention weight). With tau > 0, every later decode
+ * call of this context (tq_decode_attention, tq_decode_step and the no-alloc
+ * variant) gives no value contribution to a position whose softmax weight is
+ * below tau times the largest weight; the softmax denominator still covers every
+ * position, and a page whose values are all skipped costs no value work. The
+ * comparison is made against the largest weight seen so far by the warp that
+ * reads the page (never more than the largest overall), so a call skips a subset
+ * of the positions the definition allows; the output differs from the dense one
+ * by at most the sum over skipped positions of w_t ||v_t c_t||. The pages give no
+ * threshold. tau = 0 (the default) is dense attention; tau in [0, 1], else
+ * TQ_ERR_INVALID_ARG. Host-side setting; no device work.
+ */
+tq_status tq_set_sparse_v(tq_ctx* ctx, float tau);
+
+/*
  * tq_decode_attention without a caller workspace. The pages have no counterpart
  * to this call: it is a library convenience, computing exactly what
  * tq_decode_attention computes, with the same arguments minus the workspace.

@@ -15,6 +15,12 @@ Readings: scale = 1/sqrt(d) (the pages do not state one); values carry no QJL
 bits; all stored quantities (fp16 norms, fp16 centroids) are used as stored; a
 sequence with no cached tokens attends to nothing and returns 0. Query head h
 reads KV head floor(h / g) with g = n_q_heads / n_kv_heads.
+
+Sparse V (wis-web.com llama.cpp-fork post, third finding: decoding skips the V
+positions with a low attention weight): with a threshold tau > 0, position t
+contributes no value when its softmax weight is below tau times the largest
+weight; the softmax denominator still covers every position. The pages give no
+threshold; tau is a parameter and tau = 0 is dense attention.
 """
 
 import numpy as np
@@ -38,16 +44,34 @@ def logits(qt, p, k_codes, k_norm, gamma, sign_bits, centroids_k, scale, m):
     return scale * (main + qjl)
 
 
-def attend(lg, v_codes, v_norm, centroids_v, signs_v):
-    """Softmax over the logits and the de-rotated weighted value sum (float64, [d])."""
+def attend(lg, v_codes, v_norm, centroids_v, signs_v, sparse_tau=0.0):
+    """Softmax over the logits and the de-rotated weighted value sum (float64, [d]).
+
+    sparse_tau > 0: positions whose weight is below sparse_tau * max weight add no
+    value (Sparse V); the normalisation is unchanged."""
     d = len(signs_v)
     if len(lg) == 0:
         return np.zeros(d)
-    w = np.exp(lg - np.max(lg))
+    w = np.exp(lg - np.max(lg))                 # the largest weight is 1
     w = w / np.sum(w)
+    if sparse_tau > 0.0:
+        w = np.where(w >= sparse_tau * np.max(w), w, 0.0)
     cv = np.asarray(centroids_v, dtype=np.float64)[np.asarray(v_codes)]
     a = (w * np.asarray(v_norm, dtype=np.float64)) @ cv
     return unrotate(a, signs_v)
+
+
+def sparse_bound(lg, v_codes, v_norm, centroids_v, sparse_tau):
+    """Sum over the positions Sparse V drops of w_t ||v_t c_t||: an upper bound of the
+    2-norm change of the output (the inverse rotation preserves norms)."""
+    if len(lg) == 0 or sparse_tau <= 0.0:
+        return 0.0
+    w = np.exp(lg - np.max(lg))
+    w = w / np.sum(w)
+    drop = w < sparse_tau * np.max(w)
+    cv = np.asarray(centroids_v, dtype=np.float64)[np.asarray(v_codes)]
+    vn = np.asarray(v_norm, dtype=np.float64) * np.linalg.norm(cv, axis=1)
+    return float(np.sum(w[drop] * vn[drop]))
 
 
 def gather_sequence(cache, block_table, seq_len, kv_head, bk, bv):
@@ -62,12 +86,14 @@ def gather_sequence(cache, block_table, seq_len, kv_head, bk, bv):
     return tuple(cat)
 
 
-def decode_paged(cache, block_tables, seq_lens, q, tables, scale=None):
+def decode_paged(cache, block_tables, seq_lens, q, tables, scale=None, sparse_tau=0.0, bounds=None):
     """Reference decode over a paged cache.
 
     cache: uint8 [n_pages, n_kv, block_bytes]; block_tables: int [B, max_pages];
     seq_lens: int [B]; q: [B, Hq, d]; tables: dict with signs_k, signs_v, sketch,
-    centroids_k, centroids_v, bk, bv. Returns out [B, Hq, d] float64.
+    centroids_k, centroids_v, bk, bv. Returns out [B, Hq, d] float64. sparse_tau:
+    Sparse V threshold (0: dense); bounds, if given ([B, Hq]), receives each head's
+    sparse_bound.
     """
     q = np.asarray(q, dtype=np.float64)
     B, Hq, d = q.shape
@@ -85,5 +111,7 @@ def decode_paged(cache, block_tables, seq_lens, q, tables, scale=None):
                 h = hk * g + hh
                 qt, p = transform_query(q[b, h], tables["signs_k"], tables["sketch"])
                 lg = logits(qt, p, kc, nk, gm, sb, tables["centroids_k"], scale, m)
-                out[b, h] = attend(lg, vc, nv, tables["centroids_v"], tables["signs_v"])
+                out[b, h] = attend(lg, vc, nv, tables["centroids_v"], tables["signs_v"], sparse_tau)
+                if bounds is not None:
+                    bounds[b, h] = sparse_bound(lg, vc, nv, tables["centroids_v"], sparse_tau)
     return out

@@ -178,3 +178,56 @@ def test_paged_decode_equals_direct_decode():
         qt, p = dec.transform_query(q[0, h], tab["signs_k"], tab["sketch"])
         lg = dec.logits(qt, p, kc, nk, gm, sb, tab["centroids_k"], 1 / np.sqrt(D), D)
         np.testing.assert_allclose(out[0, h], dec.attend(lg, vc, nv, tab["centroids_v"], tab["signs_v"]))
+
+
+def _sparse_case(seed, T=200, spread=3.0):
+    book = cb.codebook(2)
+    dv = sign_vector(seed, D)
+    rng = np.random.default_rng(seed)
+    qv = quantize(rng.standard_normal((T, D)), dv, book.centroids, book.thresholds)
+    lg = rng.standard_normal(T) * spread
+    return lg, qv, book, dv
+
+
+def test_sparse_v_zero_threshold_is_dense_attention():
+    lg, qv, book, dv = _sparse_case(11)
+    dense = dec.attend(lg, qv.codes, qv.norm16, book.centroids, dv)
+    assert np.array_equal(dec.attend(lg, qv.codes, qv.norm16, book.centroids, dv, 0.0), dense)
+    assert dec.sparse_bound(lg, qv.codes, qv.norm16, book.centroids, 0.0) == 0.0
+
+
+def test_sparse_v_threshold_one_keeps_only_the_largest_weight():
+    # closed form: with tau = 1 only the argmax position adds its value, with its
+    # softmax weight (the normalisation still covers every position)
+    lg, qv, book, dv = _sparse_case(12)
+    j = int(np.argmax(lg))
+    p_max = 1.0 / np.sum(np.exp(lg - lg[j]))
+    vhat_j = qv.norm16[j] * unrotate(book.centroids[qv.codes[j]], dv)
+    got = dec.attend(lg, qv.codes, qv.norm16, book.centroids, dv, 1.0)
+    np.testing.assert_allclose(got, p_max * vhat_j, rtol=1e-12, atol=1e-15)
+
+
+def test_sparse_v_dropping_one_position_moves_the_output_by_its_contribution():
+    # exactly one position below the threshold: the output changes by w_t ||v_t||
+    # (the inverse rotation is orthogonal), which is what sparse_bound reports
+    lg, qv, book, dv = _sparse_case(13, T=50, spread=0.5)
+    lg[7] = lg.max() - 8.0                        # weight e^-8 of the largest; all others > e^-3
+    tau = 1e-3
+    w = np.exp(lg - lg.max())
+    assert np.sum(w < tau) == 1
+    dense = dec.attend(lg, qv.codes, qv.norm16, book.centroids, dv)
+    sparse = dec.attend(lg, qv.codes, qv.norm16, book.centroids, dv, tau)
+    bound = dec.sparse_bound(lg, qv.codes, qv.norm16, book.centroids, tau)
+    vhat7 = qv.norm16[7] * unrotate(book.centroids[qv.codes[7]], dv)
+    expect = (w[7] / w.sum()) * vhat7
+    np.testing.assert_allclose(dense - sparse, expect, rtol=1e-9, atol=1e-9 * np.linalg.norm(expect))
+    assert np.isclose(np.linalg.norm(dense - sparse), bound, rtol=1e-9)
+
+
+@pytest.mark.parametrize("tau", [1e-6, 1e-3, 1e-1])
+def test_sparse_v_change_is_within_the_dropped_mass(tau):
+    lg, qv, book, dv = _sparse_case(14, T=400, spread=4.0)
+    dense = dec.attend(lg, qv.codes, qv.norm16, book.centroids, dv)
+    sparse = dec.attend(lg, qv.codes, qv.norm16, book.centroids, dv, tau)
+    bound = dec.sparse_bound(lg, qv.codes, qv.norm16, book.centroids, tau)
+    assert np.linalg.norm(dense - sparse) <= bound * (1 + 1e-12) + 1e-300
