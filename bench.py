@@ -289,6 +289,62 @@ class DecodeBench:
                 "tokens": self.T0, "kv_heads": n_kv, "bytes_in": bytes_in, "bytes_out": bytes_out,
                 "kernel": "quantize_prefill_kernel via tq_quantize_prefill (bf16 K/V, one layer)"}
 
+    def logits_timing(self, reps=3):
+        """Logits only (tq_decode_logits) against logits from full-precision fp32 keys.
+
+        The pages compare attention-logit speed on compressed keys with 32-bit keys.
+        Ours reads the key codes, sign bits and norms of every cached token-head and
+        writes fp32 logits; the comparison is one cuBLAS batched product of the
+        queries with an fp32 key cache of the same shape. Both rotate over the layer
+        caches, so both stream from HBM."""
+        torch, wl = self.torch, self.wl
+        n_kv, nq, B, T = wl.n_kv_heads, wl.n_q_heads, wl.batch, self.max_len
+        g = nq // n_kv
+        last = self.total_steps - 1
+        out = torch.empty((B, nq, T), dtype=torch.float32, device=self.dev)
+        st = torch.cuda.current_stream(self.dev)
+
+        def run_ours(layer):
+            cache, n_pages = self.caches[layer]
+            self.ctx.decode_logits(self.q[last, layer], cache, n_pages, self.btabs[layer], self.lens[last], n_kv,
+                                   T, out)
+
+        def time_it(fn, layers):
+            fn(0)
+            torch.cuda.synchronize(self.dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            for _ in range(reps):
+                for layer in range(layers):
+                    fn(layer)
+            b.record(st)
+            b.synchronize()
+            return a.elapsed_time(b) / 1e3 / (reps * layers)
+
+        ours = time_it(run_ours, self.n_layers)
+        key_bytes = self.cache_tokens * n_kv * (16 * wl.key_bits + 16 + 4)
+        res = {"kernel": "decode_kernel (logits mode) via tq_decode_logits", "us_per_layer": ours * 1e6,
+               "key_bytes_per_layer": key_bytes, "gbs": key_bytes / ours / 1e9,
+               "logit_bytes_written": nq * int(self.lens[last].sum().item()) * 4}
+        try:
+            gen = torch.Generator(device=self.dev)
+            gen.manual_seed(5)
+            k32 = [torch.randn((B, n_kv, T, 128), generator=gen, device=self.dev) for _ in range(self.n_layers)]
+            q32 = self.q[last].float().view(self.n_layers, B, n_kv, g, 128)
+            o32 = torch.empty((B, n_kv, g, T), dtype=torch.float32, device=self.dev)
+            fp32 = time_it(lambda layer: torch.matmul(q32[layer], k32[layer].transpose(-1, -2), out=o32),
+                           self.n_layers)
+            b32 = B * n_kv * T * 128 * 4
+            res.update({"fp32_keys": f"torch {torch.__version__} matmul (cuBLAS), fp32 keys",
+                        "fp32_keys_us_per_layer": fp32 * 1e6, "fp32_key_bytes_per_layer": b32,
+                        "fp32_keys_gbs": b32 / fp32 / 1e9, "speedup_vs_fp32_keys": fp32 / ours,
+                        "key_bytes_ratio": b32 / key_bytes})
+            del k32
+            torch.cuda.empty_cache()
+        except Exception as e:                       # comparison unavailable
+            res["fp32_keys_error"] = repr(e)[:200]
+        return res
+
     def bf16_baseline(self, reps=3):
         """Decode attention over an uncompressed bf16 KV cache of the same shape (context only).
 
@@ -536,6 +592,7 @@ def main():
     assert bench.ctx.device_error() == 0
 
     base16 = bench.bf16_baseline()
+    logits_cmp = bench.logits_timing()
     quant = bench.quantize_timing()
     quant["frac"] = quant["gbs"] / load_peaks()[0]
     peak, peak_kind = load_peaks()
@@ -567,6 +624,7 @@ def main():
                      "kernel": "decode_kernel via tq_decode_attention (query transform, split-K decode, merge)",
                      "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
         "quantize": quant,
+        "logits": logits_cmp,
         "bf16_baseline": dict(base16, **({"compressed_us_per_layer": dec_s * 1e6,
                                           "speedup_vs_bf16": base16["us_per_layer"] / (dec_s * 1e6),
                                           "cache_bytes_ratio": base16["bytes_per_layer"] / alg_bytes}

@@ -49,6 +49,9 @@ _SIGS = {
                                                _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int,
                                                _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p]),
     "tq_set_sparse_v": (_c.c_int, [_c.c_void_p, _c.c_float]),
+    "tq_decode_logits": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int64, _c.c_void_p,
+                                    _c.c_int, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
+                                    _c.c_void_p, _c.c_int64, _c.c_void_p]),
     "tq_get_device_error": (_c.c_int, [_c.c_void_p, _c.POINTER(_c.c_uint32), _c.c_void_p]),
     "tq_host_sign_vector": (_c.c_int, [_c.c_uint64, _c.c_int, _c.c_void_p]),
     "tq_host_gaussian_sketch": (_c.c_int, [_c.c_uint64, _c.c_int, _c.c_int, _c.c_void_p]),
@@ -192,6 +195,15 @@ class Context:
         _check("tq_decode_attention_noalloc", lib().tq_decode_attention_noalloc(
             self._h, _ptr(q), _dtype_code(q), _ptr(cache), n_cache_pages, _ptr(block_tables),
             block_tables.shape[1], _ptr(seq_lens), batch, n_q, n_kv_heads, max_seq_len, scale, _ptr(out),
+            _stream(stream)))
+
+    def decode_logits(self, q, cache, n_cache_pages: int, block_tables, seq_lens, n_kv_heads: int,
+                      max_seq_len: int, logits, scale: float = 0.0, stream=None):
+        """logits: float32 [batch, n_q_heads, stride >= max_seq_len] CUDA tensor."""
+        batch, n_q = q.shape[0], q.shape[1]
+        _check("tq_decode_logits", lib().tq_decode_logits(
+            self._h, _ptr(q), _dtype_code(q), _ptr(cache), n_cache_pages, _ptr(block_tables), block_tables.shape[1],
+            _ptr(seq_lens), batch, n_q, n_kv_heads, max_seq_len, scale, _ptr(logits), logits.shape[-1],
             _stream(stream)))
 
     def set_sparse_v(self, tau: float):

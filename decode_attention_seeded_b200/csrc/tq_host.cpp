@@ -535,7 +535,7 @@ static tq_status check_decode_args(tq_ctx* ctx, const void* q, tq_dtype q_dtype,
                                    int64_t n_cache_pages, const int32_t* block_tables, int max_pages_per_seq,
                                    const int32_t* seq_lens, int batch, int n_q_heads, int n_kv_heads,
                                    int max_seq_len, float scale, const float* out, const void* workspace,
-                                   size_t workspace_bytes, tq::DecodePlan* plan) {
+                                   size_t workspace_bytes, tq::DecodePlan* plan, bool need_workspace = true) {
   if (!ctx) return TQ_ERR_INVALID_ARG;
   if (!ctx->rot_ready || !ctx->cb_ready) return TQ_ERR_NOT_INITIALIZED;
   if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads ||
@@ -543,14 +543,16 @@ static tq_status check_decode_args(tq_ctx* ctx, const void* q, tq_dtype q_dtype,
     return TQ_ERR_INVALID_ARG;
   if (n_q_heads / n_kv_heads > 16) return TQ_ERR_UNSUPPORTED;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16) return TQ_ERR_UNSUPPORTED;
-  if (!q || !cache || !block_tables || !seq_lens || !out || !workspace) return TQ_ERR_INVALID_ARG;
+  if (!q || !cache || !block_tables || !seq_lens || !out || (need_workspace && !workspace))
+    return TQ_ERR_INVALID_ARG;
   if (static_cast<int64_t>(max_pages_per_seq) * tq::kPage < max_seq_len) return TQ_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(cache) % 16) return TQ_ERR_INVALID_ARG;
   const size_t es = q_dtype == TQ_F32 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(q) % (4 * es)) return TQ_ERR_INVALID_ARG;
   if (!(scale >= 0.0f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
   *plan = tq::make_plan(batch, n_q_heads, n_kv_heads, max_seq_len, ctx->sm_count);
-  if (workspace_bytes < plan->total || reinterpret_cast<uintptr_t>(workspace) % 256) return TQ_ERR_WORKSPACE;
+  if (need_workspace && (workspace_bytes < plan->total || reinterpret_cast<uintptr_t>(workspace) % 256))
+    return TQ_ERR_WORKSPACE;
   return check_device(ctx);
 }
 
@@ -624,6 +626,22 @@ tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dty
   return from_cuda(tq::launch_decode(ctx->tables, plan, q, q_dtype, cache, n_cache_pages,
                                      block_tables, max_pages_per_seq, seq_lens, max_seq_len,
                                      scale, out, scratch, ctx->sparse_tau,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+tq_status tq_decode_logits(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
+                           int64_t n_cache_pages, const int32_t* block_tables, int max_pages_per_seq,
+                           const int32_t* seq_lens, int batch, int n_q_heads, int n_kv_heads, int max_seq_len,
+                           float scale, float* logits, int64_t logits_stride, tq_stream stream) {
+  tq::DecodePlan plan;
+  if (tq_status st = check_decode_args(ctx, q, q_dtype, cache, n_cache_pages, block_tables, max_pages_per_seq,
+                                       seq_lens, batch, n_q_heads, n_kv_heads, max_seq_len, scale, logits,
+                                       nullptr, 0, &plan, false))
+    return st;
+  if (logits_stride < max_seq_len) return TQ_ERR_INVALID_ARG;
+  if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
+  return from_cuda(tq::launch_logits(ctx->tables, plan, q, q_dtype, cache, n_cache_pages, block_tables,
+                                     max_pages_per_seq, seq_lens, max_seq_len, scale, logits, logits_stride,
                                      static_cast<cudaStream_t>(stream)));
 }
 

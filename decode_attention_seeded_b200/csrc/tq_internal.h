@@ -59,6 +59,11 @@ cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q
                           int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len,
                           float scale, float* out, void* workspace, float sparse_tau, cudaStream_t s);
 
+cudaError_t launch_logits(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype, const void* cache,
+                          int64_t n_pages, const int32_t* block_tables, int max_pages_per_seq,
+                          const int32_t* seq_lens, int max_seq_len, float scale, float* logits,
+                          int64_t logits_stride, cudaStream_t s);
+
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, const void* q, int q_dtype, void* cache, int64_t n_pages,
                                const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,

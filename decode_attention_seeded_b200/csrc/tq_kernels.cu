@@ -975,6 +975,8 @@ struct DecodeArgs {
   int merge_cap;                 // chunk records that fit in shared memory for the final merge
   int sparse;                    // Sparse V on: values of positions below the threshold are skipped
   float sparse_log2;             // log2 of the Sparse V threshold (relative attention weight)
+  float* logits;                 // logits-only mode: [batch][n_q][logits_stride] (natural log units)
+  int64_t logits_stride;
 };
 
 // Shared-memory scratch of the prologue (after the stages and barriers).
@@ -1043,8 +1045,10 @@ __device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float
 // APPEND: the CTA whose chunk holds a sequence's last page first quantizes
 // (k_new, v_new) of that sequence into position seq_len - 1; a warp that is
 // given that page before then holds its copy back until the token is written.
-template <int BK, int BV, int NH, bool APPEND>
+template <int BK, int BV, int NH, int MODE>
 __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
+  constexpr bool APPEND = MODE == 1;        // append the new token first (decode step)
+  constexpr bool LOGITS = MODE == 2;        // write the logits; no softmax, no value sum
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int W = DecodeWarps<NH>::value;
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
@@ -1135,6 +1139,11 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     if (!ok) {
       set_error(T.err, TQ_DEV_BAD_PAGE);
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mybar + s)) : "memory");
+    } else if constexpr (LOGITS) {          // key codes and signs, then the norms; no value codes
+      const uint8_t* src = A.cache + (static_cast<int64_t>(phys) * A.n_kv + hk) * kBlock;
+      mbar_expect_tx(mybar + s, kVOff + 96);
+      tma_load_1d(stage0 + s * kBlock, src, kVOff, mybar + s);
+      tma_load_1d(stage0 + s * kBlock + kNormOff, src + kNormOff, 96, mybar + s);
     } else {
       mbar_expect_tx(mybar + s, kBlock);
       tma_load_1d(stage0 + s * kBlock, A.cache + (static_cast<int64_t>(phys) * A.n_kv + hk) * kBlock, kBlock,
@@ -1403,7 +1412,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     lds_words<2 * BK>(reinterpret_cast<const uint32_t*>(blk) + lane * 2 * BK, kw);
     const uint2 sw = reinterpret_cast<const uint2*>(blk + kSignOff)[lane];
     uint32_t vw[2 * BV];
-    lds_words<2 * BV>(reinterpret_cast<const uint32_t*>(blk + kVOff) + lane * 2 * BV, vw);
+    if constexpr (!LOGITS) lds_words<2 * BV>(reinterpret_cast<const uint32_t*>(blk + kVOff) + lane * 2 * BV, vw);
     const uint32_t* nrm = reinterpret_cast<const uint32_t*>(blk + kNormOff);
     const uint32_t rk = nrm[g], rg = nrm[8 + g], rv = nrm[16 + g];
     const float2 nK = __half22float2(*reinterpret_cast<const __half2*>(&rk));
@@ -1471,9 +1480,16 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
         const float main = fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
         const int sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + ds[h][1][2 * r];
         const float nk = r ? nK.y : nK.x, gg = r ? gm.y : gm.x, lv = r ? lgv1 : lgv0;
-        const float v = fmaf(nk * ca[h], main, fmaf(gg * cb[h], static_cast<float>(2 * sj - csum[h]), lv));
-        lp2[r] = (g + 8 * r) < n_valid ? v : -INFINITY;
+        const float l2 = fmaf(nk * ca[h], main, gg * cb[h] * static_cast<float>(2 * sj - csum[h]));
+        if constexpr (LOGITS) {               // natural-log logit of (token g + 8r, head 4h + t)
+          const int qi = 4 * h + t;
+          if ((g + 8 * r) < n_valid && qi < A.group)
+            A.logits[(static_cast<int64_t>(b) * A.n_q + hk * A.group + qi) * A.logits_stride + lp * kPage + g +
+                     8 * r] = l2 * 0.6931471805599453f;
+        }
+        lp2[r] = (g + 8 * r) < n_valid ? l2 + lv : -INFINITY;
       }
+      if constexpr (LOGITS) continue;
       float pm = fmaxf(lp2[0], lp2[1]);
       pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 4));
       pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 8));
@@ -1527,7 +1543,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
 
     // ---- weighted value sum in the rotated domain: fp16 tensor-core products
     // (Sparse V: skipped for a page whose values are all below the threshold)
-    if (!A.sparse || __any_sync(kFull, kept)) {
+    if (!LOGITS && (!A.sparse || __any_sync(kFull, kept))) {
       uint32_t vs[16];
       value_selectors<BV>(vw, vs);
 #pragma unroll
@@ -1566,6 +1582,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   if (lane == 0)
     for (int s2 = 0; s2 < S; ++s2)
       asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(mybar + s2)) : "memory");
+  if constexpr (LOGITS) return;                   // logits are written; nothing to merge
 
   // ---- merge the warps of this CTA (the pipeline buffers are free now)
 #pragma unroll
@@ -1726,7 +1743,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   }
 }
 
-template <int BK, int BV, int NH, bool APPEND>
+template <int BK, int BV, int NH, int MODE>
 cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   constexpr int W = DecodeWarps<NH>::value;
   constexpr int kBlock = 256 * (BK + BV + 1) + 96;
@@ -1743,7 +1760,7 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
   if (smem > 227 * 1024 || smem < (groups + 1) * chunk_bytes + 16) return cudaErrorInvalidConfiguration;
   DecodeArgs args = a;
   args.merge_cap = static_cast<int>((smem - groups * chunk_bytes - 16) / chunk_bytes);
-  auto fn = decode_kernel<BK, BV, NH, APPEND>;
+  auto fn = decode_kernel<BK, BV, NH, MODE>;
   static size_t configured = 0;     // raise the shared-memory limit once per instantiation
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -1754,31 +1771,31 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
   return cudaGetLastError();
 }
 
-template <int BK, int BV, bool APPEND>
+template <int BK, int BV, int MODE>
 cudaError_t dispatch_nh(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   switch (a.n_hg) {
-    case 1: return launch_decode_t<BK, BV, 1, APPEND>(T, a, grid, s);
-    case 2: return launch_decode_t<BK, BV, 2, APPEND>(T, a, grid, s);
-    case 3: return launch_decode_t<BK, BV, 3, APPEND>(T, a, grid, s);
-    default: return launch_decode_t<BK, BV, 4, APPEND>(T, a, grid, s);
+    case 1: return launch_decode_t<BK, BV, 1, MODE>(T, a, grid, s);
+    case 2: return launch_decode_t<BK, BV, 2, MODE>(T, a, grid, s);
+    case 3: return launch_decode_t<BK, BV, 3, MODE>(T, a, grid, s);
+    default: return launch_decode_t<BK, BV, 4, MODE>(T, a, grid, s);
   }
 }
 
-template <int BK, bool APPEND>
+template <int BK, int MODE>
 cudaError_t dispatch_bv(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   switch (T.value_bits) {
-    case 2: return dispatch_nh<BK, 2, APPEND>(T, a, grid, s);
-    case 3: return dispatch_nh<BK, 3, APPEND>(T, a, grid, s);
-    default: return dispatch_nh<BK, 4, APPEND>(T, a, grid, s);
+    case 2: return dispatch_nh<BK, 2, MODE>(T, a, grid, s);
+    case 3: return dispatch_nh<BK, 3, MODE>(T, a, grid, s);
+    default: return dispatch_nh<BK, 4, MODE>(T, a, grid, s);
   }
 }
 
-template <bool APPEND>
+template <int MODE>
 cudaError_t dispatch_bk(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   switch (T.key_bits) {
-    case 2: return dispatch_bv<2, APPEND>(T, a, grid, s);
-    case 3: return dispatch_bv<3, APPEND>(T, a, grid, s);
-    default: return dispatch_bv<4, APPEND>(T, a, grid, s);
+    case 2: return dispatch_bv<2, MODE>(T, a, grid, s);
+    case 3: return dispatch_bv<3, MODE>(T, a, grid, s);
+    default: return dispatch_bv<4, MODE>(T, a, grid, s);
   }
 }
 
@@ -1802,8 +1819,8 @@ DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float
   a.max_pages_per_seq = max_pages_per_seq;
   a.seq_lens = seq_lens;
   a.max_seq_len = max_seq_len;
-  a.partial = reinterpret_cast<float*>(ws + plan.off_partial);
-  a.counters = reinterpret_cast<unsigned*>(ws + plan.off_counter);
+  a.partial = ws ? reinterpret_cast<float*>(ws + plan.off_partial) : nullptr;
+  a.counters = ws ? reinterpret_cast<unsigned*>(ws + plan.off_counter) : nullptr;
   a.out = out;
   a.n_kv = plan.n_kv;
   a.n_q = plan.n_q;
@@ -1890,7 +1907,18 @@ cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q
                           float* out, void* workspace, float sparse_tau, cudaStream_t s) {
   const DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq,
                                    seq_lens, max_seq_len, out, workspace, sparse_tau);
-  return dispatch_bk<false>(t, a, dim3(plan.chunks * plan.n_pairs), s);
+  return dispatch_bk<0>(t, a, dim3(plan.chunks * plan.n_pairs), s);
+}
+
+cudaError_t launch_logits(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype, const void* cache,
+                          int64_t n_pages, const int32_t* block_tables, int max_pages_per_seq,
+                          const int32_t* seq_lens, int max_seq_len, float scale, float* logits,
+                          int64_t logits_stride, cudaStream_t s) {
+  DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq, seq_lens,
+                             max_seq_len, nullptr, nullptr, 0.0f);
+  a.logits = logits;
+  a.logits_stride = logits_stride;
+  return dispatch_bk<2>(t, a, dim3(plan.chunks * plan.n_pairs), s);
 }
 
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
@@ -1903,7 +1931,7 @@ cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const vo
   a.k_new = k_new;
   a.v_new = v_new;
   a.kv_dtype = kv_dtype;
-  return dispatch_bk<true>(t, a, dim3(plan.chunks * plan.n_pairs), s);
+  return dispatch_bk<1>(t, a, dim3(plan.chunks * plan.n_pairs), s);
 }
 
 }  // namespace tq

@@ -172,6 +172,23 @@ tq_status tq_decode_step(tq_ctx* ctx, const void* k_new, const void* v_new, tq_d
                          void* workspace, size_t workspace_bytes, tq_stream stream);
 
 /*
+ * Attention logits only (leviatan.io page, sections "Accélération jusqu'à 8× du
+ * calcul d'attention" and "Comparaison 4-bit vs 32-bit": the logit computation on
+ * compressed keys against full-precision keys). Writes, for every sequence b,
+ * query head h and cached position t < seq_lens[b],
+ *   logits[(b * n_q_heads + h) * logits_stride + t]
+ *     = scale * ( |k_t| <R_K q, c[code_t]> + |r_t| sqrt(pi/2)/m <S R_K q, sign(S r_t)> )
+ * (natural-log units, float32), exactly the logits tq_decode_attention softmaxes.
+ * Positions >= seq_lens[b] are not written. Only the key codes, sign bits and
+ * norms of each block are read. logits: (device) float32, logits_stride >=
+ * max_seq_len. No workspace. Other arguments and errors as tq_decode_attention.
+ */
+tq_status tq_decode_logits(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
+                           int64_t n_cache_pages, const int32_t* block_tables, int max_pages_per_seq,
+                           const int32_t* seq_lens, int batch, int n_q_heads, int n_kv_heads, int max_seq_len,
+                           float scale, float* logits, int64_t logits_stride, tq_stream stream);
+
+/*
  * Sparse V (wis-web.com llama.cpp-fork post, third finding: decoding that skips
  * the V positions with a low attention weight). With tau > 0, every later decode
  * call of this context (tq_decode_attention, tq_decode_step and the no-alloc
