@@ -26,7 +26,8 @@ threshold; tau is a parameter and tau = 0 is dense attention.
 import numpy as np
 
 from .hadamard import rotate, unrotate
-from .layout import read_page, PAGE
+from .layout import read_page, read_page_q8, PAGE
+from .q8 import logits_q8
 
 
 def transform_query(q, signs_k, sketch):
@@ -86,12 +87,22 @@ def gather_sequence(cache, block_table, seq_len, kv_head, bk, bv):
     return tuple(cat)
 
 
+def gather_sequence_q8(cache, block_table, seq_len, kv_head, bv):
+    """q8_0-key cache: values [T, d], scales16 [T, 4], v_codes [T, d], v_norm [T]."""
+    n_pages = (seq_len + PAGE - 1) // PAGE
+    parts = [read_page_q8(cache[int(block_table[i]), kv_head], bv) for i in range(n_pages)]
+    if not parts:
+        z = np.zeros((0, 128), dtype=np.int64)
+        return z, np.zeros((0, 4)), z, np.zeros(0)
+    return tuple(np.concatenate([pp[f] for pp in parts])[:seq_len] for f in range(4))
+
+
 def decode_paged(cache, block_tables, seq_lens, q, tables, scale=None, sparse_tau=0.0, bounds=None):
     """Reference decode over a paged cache.
 
     cache: uint8 [n_pages, n_kv, block_bytes]; block_tables: int [B, max_pages];
     seq_lens: int [B]; q: [B, Hq, d]; tables: dict with signs_k, signs_v, sketch,
-    centroids_k, centroids_v, bk, bv. Returns out [B, Hq, d] float64. sparse_tau:
+    centroids_k, centroids_v, bk, bv (bk = 8: q8_0 keys). Returns out [B, Hq, d] float64. sparse_tau:
     Sparse V threshold (0: dense); bounds, if given ([B, Hq]), receives each head's
     sparse_bound.
     """
@@ -105,12 +116,18 @@ def decode_paged(cache, block_tables, seq_lens, q, tables, scale=None, sparse_ta
     out = np.zeros((B, Hq, d))
     for b in range(B):
         for hk in range(n_kv):
-            kc, sb, vc, nk, gm, nv = gather_sequence(cache, block_tables[b], int(seq_lens[b]), hk,
-                                                     tables["bk"], tables["bv"])
+            if tables["bk"] == 8:                  # q8_0 keys: raw query, block scales
+                k8, sc, vc, nv = gather_sequence_q8(cache, block_tables[b], int(seq_lens[b]), hk, tables["bv"])
+            else:
+                kc, sb, vc, nk, gm, nv = gather_sequence(cache, block_tables[b], int(seq_lens[b]), hk,
+                                                         tables["bk"], tables["bv"])
             for hh in range(g):
                 h = hk * g + hh
-                qt, p = transform_query(q[b, h], tables["signs_k"], tables["sketch"])
-                lg = logits(qt, p, kc, nk, gm, sb, tables["centroids_k"], scale, m)
+                if tables["bk"] == 8:
+                    lg = logits_q8(q[b, h], k8, sc, scale)
+                else:
+                    qt, p = transform_query(q[b, h], tables["signs_k"], tables["sketch"])
+                    lg = logits(qt, p, kc, nk, gm, sb, tables["centroids_k"], scale, m)
                 out[b, h] = attend(lg, vc, nv, tables["centroids_v"], tables["signs_v"], sparse_tau)
                 if bounds is not None:
                     bounds[b, h] = sparse_bound(lg, vc, nv, tables["centroids_v"], sparse_tau)

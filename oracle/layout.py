@@ -41,6 +41,17 @@ Value codes of token tau, coordinate i:
       b=4: word s>>1, bit 16*(s&1) + 4n + p
 
 Codes are stored as the ascending centroid index (0 = most negative centroid).
+
+q8_0 keys (b_k = 8; see q8.py) use the same block frame with other key sections:
+
+    offset 0                 K values  2048 bytes  = 32 lane chunks of 64 int8
+    offset 2048              K scales  128 bytes: fp16 [16 tokens x 4 blocks of 32 coordinates]
+    offset 2176              V codes   256*b_v bytes (as above)
+    offset 2176 + 256*b_v    norms     32 bytes: ||v|| fp16[16], token tau at entry 2*(tau & 7) + (tau >> 3)
+
+    int8 value of token tau, coordinate i (g, th, kt, sub, t, q, lane as for codes):
+        byte 64*lane + 32*th + 8*kt + 4*sub + q
+    scale of token tau, block kt = i >> 5: fp16 entry 8*(tau & 7) + 4*(tau >> 3) + kt
 """
 
 from functools import lru_cache
@@ -52,11 +63,16 @@ D = 128
 
 
 def section_offsets(bk: int, bv: int):
+    if bk == 8:                                   # q8_0 keys: values, scales
+        return {"k": 0, "sign": 2048, "v": 2176, "norm": 2176 + 256 * bv}
     return {"k": 0, "sign": 256 * bk, "v": 256 * (bk + 1), "norm": 256 * (bk + bv + 1)}
 
 
 def block_bytes(bk: int, bv: int) -> int:
-    """Bytes of one (page, KV head) block: 16 tokens x (16 b_k + 16 + 4 + 16 b_v + 2)."""
+    """Bytes of one (page, KV head) block: 16 tokens x (16 b_k + 16 + 4 + 16 b_v + 2);
+    q8_0 keys: 16 tokens x (128 + 8 + 16 b_v + 2)."""
+    if bk == 8:
+        return 2176 + 256 * bv + 32
     return 256 * (bk + bv + 1) + 96
 
 
@@ -174,3 +190,50 @@ def read_page(block, bk, bv):
     norms = block[no:no + 96].view(np.float16).astype(np.float64).reshape(3, PAGE)
     order = [norm_slot(tau) for tau in range(PAGE)]
     return k_codes, sign_bits, v_codes, norms[0][order], norms[1][order], norms[2][order]
+
+
+# ------------------------------------------------------------------ q8_0 keys
+@lru_cache(maxsize=None)
+def q8_byte_index() -> np.ndarray:
+    """[16, 128] byte of every int8 key value."""
+    out = np.zeros((PAGE, D), dtype=np.int64)
+    for tau in range(PAGE):
+        g, th = tau & 7, tau >> 3
+        for i in range(D):
+            kt, sub, t, q = i >> 5, (i >> 4) & 1, (i >> 2) & 3, i & 3
+            out[tau, i] = 64 * (4 * g + t) + 32 * th + 8 * kt + 4 * sub + q
+    return out
+
+
+def q8_scale_entry(tau: int, kt: int) -> int:
+    """fp16 entry (within the scale section) of token tau's block kt."""
+    return 8 * (tau & 7) + 4 * (tau >> 3) + kt
+
+
+def write_token_q8(block, tau, bv, values, scales16, v_codes, v_norm16):
+    """Store one token of a q8_0-key block (uint8 view), leaving other tokens alone."""
+    idx = q8_byte_index()[tau]
+    block[idx] = (np.asarray(values, dtype=np.int64) & 0xFF).astype(np.uint8)
+    off = section_offsets(8, bv)
+    for kt in range(4):
+        e = off["sign"] + 2 * q8_scale_entry(tau, kt)
+        block[e:e + 2] = np.array([scales16[kt]], dtype=np.float16).view(np.uint8)
+    vb = v_bit_index(8, bv)[tau]
+    vval = (np.asarray(v_codes)[:, None] >> np.arange(bv)) & 1
+    _set_bits(block, vb, vval)
+    e = off["norm"] + 2 * norm_slot(tau)
+    block[e:e + 2] = np.array([v_norm16], dtype=np.float16).view(np.uint8)
+
+
+def read_page_q8(block, bv):
+    """Unpack a q8_0-key block: values [16,128], scales16 [16,4], v_codes [16,128], v_norm [16]."""
+    block = np.asarray(block, dtype=np.uint8)
+    values = block[q8_byte_index()].view(np.int8).astype(np.int64)
+    off = section_offsets(8, bv)
+    sc = block[off["sign"]:off["sign"] + 128].view(np.float16).astype(np.float64)
+    scales = np.array([[sc[q8_scale_entry(tau, kt)] for kt in range(4)] for tau in range(PAGE)])
+    vb = v_bit_index(8, bv)
+    v_codes = np.sum(_get_bits(block, vb).astype(np.int64) << np.arange(bv), axis=-1)
+    nv = block[off["norm"]:off["norm"] + 32].view(np.float16).astype(np.float64)
+    v_norm = np.array([nv[norm_slot(tau)] for tau in range(PAGE)])
+    return values, scales, v_codes, v_norm
