@@ -221,10 +221,14 @@ class DeviceGuard {               // make ctx->device current for the scope
 };
 
 bool valid_bits(int b) { return b >= 2 && b <= 4; }
-size_t block_bytes_for(int bk, int bv) { return 256u * (bk + bv + 1) + 96u; }
+bool valid_key_bits(int b) { return valid_bits(b) || b == 8; }   // 8: q8_0 keys
+size_t block_bytes_for(int bk, int bv) {
+  return bk == 8 ? 2176u + 256u * bv + 32u : 256u * (bk + bv + 1) + 96u;
+}
 
 tq_status fill_codebook_tables(tq::Tables& t, int bk, int bv) {
-  StoredCodebook ck = make_codebook(bk, tq::kHeadDim), cv = make_codebook(bv, tq::kHeadDim);
+  const bool q8 = bk == 8;                  // q8_0 keys carry no key codebook
+  StoredCodebook ck = make_codebook(q8 ? 2 : bk, tq::kHeadDim), cv = make_codebook(bv, tq::kHeadDim);
   if (!ck.ok || !cv.ok) return TQ_ERR_UNSUPPORTED;
   std::memset(t.thr_k, 0, sizeof t.thr_k);
   std::memset(t.thr_v, 0, sizeof t.thr_v);
@@ -234,7 +238,7 @@ tq_status fill_codebook_tables(tq::Tables& t, int bk, int bv) {
   std::memset(t.kq_lo, 0, sizeof t.kq_lo);
   std::memset(t.v_lo, 0, sizeof t.v_lo);
   std::memset(t.v_hi, 0, sizeof t.v_hi);
-  const int nk = 1 << bk, nv = 1 << bv;
+  const int nk = q8 ? 0 : 1 << bk, nv = 1 << bv;
   double kmax = 0.0;
   for (int j = 0; j < nk; ++j) {
     t.cen_k[j] = static_cast<float>(half_bits_to_double(ck.half_bits[j]));
@@ -249,7 +253,7 @@ tq_status fill_codebook_tables(tq::Tables& t, int bk, int bv) {
     t.v_hi[j >> 2] |= static_cast<uint32_t>(h >> 8) << (8 * (j & 3));
   }
   // Key centroids as exact int16 values C = c * 2^E split C = 256*hi + lo.
-  int E = static_cast<int>(std::floor(std::log2(32639.0 / kmax)));
+  int E = q8 ? 0 : static_cast<int>(std::floor(std::log2(32639.0 / kmax)));
   for (int j = 0; j < nk; ++j) {
     const double C = std::ldexp(static_cast<double>(t.cen_k[j]), E);
     if (C != std::floor(C) || std::fabs(C) > 32639.0) return TQ_ERR_UNSUPPORTED;
@@ -462,7 +466,7 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
 tq_status tq_init_codebooks(tq_ctx* ctx, int key_bits, int value_bits, tq_stream stream) {
   (void)stream;
   if (!ctx) return TQ_ERR_INVALID_ARG;
-  if (!valid_bits(key_bits) || !valid_bits(value_bits)) return TQ_ERR_UNSUPPORTED;
+  if (!valid_key_bits(key_bits) || !valid_bits(value_bits)) return TQ_ERR_UNSUPPORTED;
   tq::Tables t = ctx->tables;
   if (tq_status st = fill_codebook_tables(t, key_bits, value_bits)) return st;
   ctx->tables = t;

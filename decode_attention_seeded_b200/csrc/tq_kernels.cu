@@ -225,6 +225,38 @@ __device__ __forceinline__ void stage_tables(const Tables& T, __half* s_sk, floa
   __syncthreads();
 }
 
+// Section offsets of a (page, KV head) block. TurboQuant keys (b_k = 2..4): key
+// codes, sign bits, value codes, norms (|k|, gamma, |v|: 3 x 16 fp16). q8_0 keys
+// (b_k = 8): int8 key values (2048 B), 64 fp16 block scales (128 B), value codes,
+// value norms (16 fp16).
+__host__ __device__ constexpr int sec_scale(int bk) { return bk == 8 ? 2048 : 256 * bk; }
+__host__ __device__ constexpr int sec_v(int bk) { return bk == 8 ? 2176 : 256 * (bk + 1); }
+__host__ __device__ constexpr int sec_norm(int bk, int bv) { return sec_v(bk) + 256 * bv; }
+__host__ __device__ constexpr int block_bytes_of(int bk, int bv) { return sec_norm(bk, bv) + (bk == 8 ? 32 : 96); }
+__host__ __device__ constexpr int vnorm_entry0(int bk) { return bk == 8 ? 0 : 32; }   // first |v| entry
+
+// q8_0 key of one token, 4 coordinates (4 lane .. 4 lane + 3) per lane: block
+// kt = lane >> 3 has scale d = max|x| / 127 (reduced over its 8 lanes) and values
+// rint(x / d). Stores the 4 int8 values as one word of lane chunk 4 (tau & 7) +
+// (lane & 3) and, from the block's first lane, the fp16 scale.
+__device__ __forceinline__ void store_key_q8(uint8_t* blk, int tau, const float (&x)[4], int lane) {
+  float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
+  const float d = amax / 127.0f;
+  uint32_t word = 0u;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int qv = d > 0.0f ? __float2int_rn(x[e] / d) : 0;
+    word |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * e);
+  }
+  const int kt = lane >> 3, sub = (lane >> 2) & 1, t = lane & 3, g = tau & 7, th = tau >> 3;
+  reinterpret_cast<uint32_t*>(blk)[(64 * (4 * g + t) + 32 * th + 8 * kt + 4 * sub) >> 2] = word;
+  if ((lane & 7) == 0)
+    reinterpret_cast<__half*>(blk + sec_scale(8))[8 * g + 4 * th + kt] = __float2half_rn(d);
+}
+
 // Word and bit of code bit p for nibble q of selector j within a group of b words.
 __device__ __forceinline__ void code_bit_pos(int b, int j, int q, int p, int& w, int& bit) {
   if (b == 2) {
@@ -274,7 +306,7 @@ __device__ void store_key_token(uint8_t* blk, int tau, int bk, const VecOut& o, 
 // Value codes share words between the four tokens 2t, 2t+1, 8+2t, 9+2t of a
 // lane chunk: clear-then-set with atomics (global or shared memory).
 __device__ void store_value_token(uint8_t* blk, int tau, int bk, int bv, const VecOut& o, int lane) {
-  uint32_t* vw = reinterpret_cast<uint32_t*>(blk + 256 * (bk + 1));
+  uint32_t* vw = reinterpret_cast<uint32_t*>(blk + sec_v(bk));
   const int tg = tau >> 3, t = (tau >> 1) & 3, et = tau & 1;
   const int mt = lane >> 2, hf = (lane >> 1) & 1;
   const int s = 2 * mt + tg, n = 2 * hf + et;
@@ -299,9 +331,10 @@ __device__ void store_value_token(uint8_t* blk, int tau, int bk, int bv, const V
 }
 
 // Norm arrays keep tokens g and g + 8 in one 32-bit word: entry 2 (tau & 7) + (tau >> 3).
+// which: 0 = |k|, 1 = gamma, 2 = |v| (q8_0 keys: |v| only, at entry 0).
 __device__ __forceinline__ void store_norm(uint8_t* blk, int bk, int bv, int which, int tau, float v) {
-  __half* nrm = reinterpret_cast<__half*>(blk + 256 * (bk + bv + 1));
-  nrm[16 * which + 2 * (tau & 7) + (tau >> 3)] = __float2half_rn(v);
+  __half* nrm = reinterpret_cast<__half*>(blk + sec_norm(bk, bv));
+  nrm[(bk == 8 ? 0 : 16 * which) + 2 * (tau & 7) + (tau >> 3)] = __float2half_rn(v);
 }
 
 // One warp per (token, KV head): quantize K and V and store them at the slot.
@@ -328,11 +361,15 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(Tables T, const vo
     float x[4];
     VecOut o;
     load_row4(k, static_cast<size_t>(tok) * n_kv + h, dtype, lane, x);
-    quantize_vector(x, T.signs_k, s_tab, s_tab + 16, T.key_bits, s_sk, true, lane, o);
-    store_key_token(blk, tau, T.key_bits, o, lane);
-    if (lane == 0) {
-      store_norm(blk, T.key_bits, T.value_bits, 0, tau, o.norm);
-      store_norm(blk, T.key_bits, T.value_bits, 1, tau, o.gamma);
+    if (T.key_bits == 8) {
+      store_key_q8(blk, tau, x, lane);
+    } else {
+      quantize_vector(x, T.signs_k, s_tab, s_tab + 16, T.key_bits, s_sk, true, lane, o);
+      store_key_token(blk, tau, T.key_bits, o, lane);
+      if (lane == 0) {
+        store_norm(blk, T.key_bits, T.value_bits, 0, tau, o.norm);
+        store_norm(blk, T.key_bits, T.value_bits, 1, tau, o.gamma);
+      }
     }
     load_row4(v, static_cast<size_t>(tok) * n_kv + h, dtype, lane, x);
     quantize_vector(x, T.signs_v, s_tab + 32, s_tab + 48, T.value_bits, nullptr, false, lane, o);
@@ -643,12 +680,56 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
       break;
     }
     float vv[2][32], ss[2];
-    pf_load(stage0 + kv * 16 * pitch, pitch, dtype, g, t, ok0, ok1, kv ? dmv : dmk, vv, ss);
+    pf_load(stage0 + kv * 16 * pitch, pitch, dtype, g, t, ok0, ok1, kv ? dmv : (BK == 8 ? 0u : dmk), vv, ss);
     __syncwarp();                                  // the rows are read: refill with the next tile's
     if (next < n_tiles) stage_rows(next, kv);
     if (!good) continue;
+    if (BK == 8 && kv == 0) {
+    // ---------------- q8_0 keys: the lane's coordinates i = 0..31 of token half th
+    // are bytes 32 th + i of its lane chunk; block kt = i >> 3 spans the quad
+      uint32_t w8[2][8];
+      float dsc[2][4];
+#pragma unroll
+      for (int th = 0; th < 2; ++th)
+#pragma unroll
+        for (int kt = 0; kt < 4; ++kt) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 8 * kt; i < 8 * kt + 8; ++i) amax = fmaxf(amax, fabsf(vv[th][i]));
+          amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+          amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+          const float d = amax / 127.0f;
+          dsc[th][kt] = d;
+#pragma unroll
+          for (int w = 2 * kt; w < 2 * kt + 2; ++w) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int qv = d > 0.0f ? __float2int_rn(vv[th][4 * w + e] / d) : 0;
+              word |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * e);
+            }
+            w8[th][w] = word;
+          }
+        }
+      uint4* kd = reinterpret_cast<uint4*>(blk + lane * 64);
+      __half* sd = reinterpret_cast<__half*>(blk + sec_scale(8)) + 8 * g;
+#pragma unroll
+      for (int th = 0; th < 2; ++th) {
+        if (!(th ? ok1 : ok0)) continue;
+        kd[2 * th] = make_uint4(w8[th][0], w8[th][1], w8[th][2], w8[th][3]);
+        kd[2 * th + 1] = make_uint4(w8[th][4], w8[th][5], w8[th][6], w8[th][7]);
+        if (t == 0) {
+          const __half2 s01 = __floats2half2_rn(dsc[th][0], dsc[th][1]);
+          const __half2 s23 = __floats2half2_rn(dsc[th][2], dsc[th][3]);
+          reinterpret_cast<uint2*>(sd + 4 * th)[0] =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&s01), *reinterpret_cast<const uint32_t*>(&s23));
+        }
+      }
+      continue;
+    }
     pf_fwht(vv, lane);
     if (kv == 0) {
+    if constexpr (BK != 8) {
     // ---------------- keys: norm, codes, residual, z = S u, signs
     float nk[2], uu[2] = {0.f, 0.f};
     uint32_t kw[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
@@ -703,7 +784,7 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
     }
     {
       uint32_t* kwd = reinterpret_cast<uint32_t*>(blk) + lane * 2 * BK;
-      uint32_t* swd = reinterpret_cast<uint32_t*>(blk + 256 * BK) + lane * 2;
+      uint32_t* swd = reinterpret_cast<uint32_t*>(blk + sec_scale(BK)) + lane * 2;
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
         if (!(th ? ok1 : ok0)) continue;
@@ -712,13 +793,14 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
         swd[th] = sw[th];
       }
       if (t == 0) {
-        __half* nrm = reinterpret_cast<__half*>(blk + 256 * (BK + BV + 1));
+        __half* nrm = reinterpret_cast<__half*>(blk + sec_norm(BK, BV));
         const float gk0 = nk[0] * sqrtf(uu[0]), gk1 = nk[1] * sqrtf(uu[1]);
         if (ok0) { nrm[2 * g] = __float2half_rn(nk[0]); nrm[16 + 2 * g] = __float2half_rn(gk0); }
         if (ok1) { nrm[2 * g + 1] = __float2half_rn(nk[1]); nrm[16 + 2 * g + 1] = __float2half_rn(gk1); }
       }
     }
 
+    }
     } else {
     // ---------------- values: norm, codes, transpose to value chunks
     float nv[2];
@@ -754,13 +836,13 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
           put_value_codes<BV>(vw, mt, hf, x & maskx);
           if (!full) put_value_codes<BV>(vm, mt, hf, maskx);
         }
-      uint32_t* vwd = reinterpret_cast<uint32_t*>(blk + 256 * (BK + 1)) + lane * 2 * BV;
+      uint32_t* vwd = reinterpret_cast<uint32_t*>(blk + sec_v(BK)) + lane * 2 * BV;
 #pragma unroll
       for (int w = 0; w < 2 * BV; ++w) vwd[w] = full ? vw[w] : ((vwd[w] & ~vm[w]) | vw[w]);
       if (t == 0) {
-        __half* nrm = reinterpret_cast<__half*>(blk + 256 * (BK + BV + 1));
-        if (ok0) nrm[32 + 2 * g] = __float2half_rn(nv[0]);
-        if (ok1) nrm[32 + 2 * g + 1] = __float2half_rn(nv[1]);
+        __half* nrm = reinterpret_cast<__half*>(blk + sec_norm(BK, BV)) + vnorm_entry0(BK);
+        if (ok0) nrm[2 * g] = __float2half_rn(nv[0]);
+        if (ok1) nrm[2 * g + 1] = __float2half_rn(nv[1]);
       }
     }
     }
@@ -835,7 +917,9 @@ __device__ __forceinline__ int warp_isum(int v) {
 template <int NH>
 struct DecodeWarps { static constexpr int value = NH == 1 ? 16 : 8; };
 // TMA stages per warp: six when they fit in 160 KB of shared memory, else four.
-__host__ __device__ constexpr int decode_stages(int warps, int block) { return warps * 6 * block <= 160 * 1024 ? 6 : 4; }
+__host__ __device__ constexpr int decode_stages(int warps, int block) {
+  return warps * 6 * block <= 160 * 1024 ? 6 : warps * 4 * block <= 160 * 1024 ? 4 : 3;
+}
 constexpr int kStatic = 2;       // pages per warp assigned before the block-table window is cached
 
 
@@ -1049,11 +1133,13 @@ template <int BK, int BV, int NH, int MODE>
 __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
   constexpr bool APPEND = MODE == 1;        // append the new token first (decode step)
   constexpr bool LOGITS = MODE == 2;        // write the logits; no softmax, no value sum
+  constexpr bool KQ8 = BK == 8;              // q8_0 keys (raw query, block scales, no QJL)
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int W = DecodeWarps<NH>::value;
-  constexpr int kBlock = 256 * (BK + BV + 1) + 96;
+  constexpr int kBlock = block_bytes_of(BK, BV);
   constexpr int S = decode_stages(W, kBlock);
-  constexpr int kSignOff = 256 * BK, kVOff = 256 * (BK + 1), kNormOff = 256 * (BK + BV + 1);
+  constexpr int kSignOff = sec_scale(BK), kVOff = sec_v(BK), kNormOff = sec_norm(BK, BV);
+  constexpr int kNormBytes = KQ8 ? 32 : 96;
   constexpr int kHeads = NH * kGroupHeads;
   constexpr bool kRegQ = NH <= 2;              // query fragments in registers (else shared memory)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1077,7 +1163,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   // do not queue behind it: this warp's sketch rows as m16n8k16 A fragments and
   // the input of its first job (query head `warp`, or the new key / value).
   uint4 afv[8];
-  if (warp < kQjlRows / 16) {
+  if (!KQ8 && warp < kQjlRows / 16) {
     const uint4* F = reinterpret_cast<const uint4*>(T.sketch) + warp * 8 * 32 + lane;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) afv[ks] = __ldg(F + ks * 32);
@@ -1141,9 +1227,9 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mybar + s)) : "memory");
     } else if constexpr (LOGITS) {          // key codes and signs, then the norms; no value codes
       const uint8_t* src = A.cache + (static_cast<int64_t>(phys) * A.n_kv + hk) * kBlock;
-      mbar_expect_tx(mybar + s, kVOff + 96);
+      mbar_expect_tx(mybar + s, kVOff + kNormBytes);
       tma_load_1d(stage0 + s * kBlock, src, kVOff, mybar + s);
-      tma_load_1d(stage0 + s * kBlock + kNormOff, src + kNormOff, 96, mybar + s);
+      tma_load_1d(stage0 + s * kBlock + kNormOff, src + kNormOff, kNormBytes, mybar + s);
     } else {
       mbar_expect_tx(mybar + s, kBlock);
       tma_load_1d(stage0 + s * kBlock, A.cache + (static_cast<int64_t>(phys) * A.n_kv + hk) * kBlock, kBlock,
@@ -1226,13 +1312,16 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       job_input(j, x);
     }
     if (j < kHeads) {
+      if constexpr (!KQ8) {                  // q~ = H D_K q / sqrt(d); q8_0 keys use q itself
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] *= (&sgk.x)[e];
-      fwht128(x, lane);
+        for (int e = 0; e < 4; ++e) x[e] *= (&sgk.x)[e];
+        fwht128(x, lane);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] *= kInvSqrtD;
+      }
       float mx = 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        x[e] *= kInvSqrtD;
         P.qt[j][4 * lane + e] = x[e];
         mx = fmaxf(mx, fabsf(x[e]));
       }
@@ -1240,6 +1329,8 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       int E = 0;
       if (mx > 0.0f) E = max(exp_above(mx), -115);   // 2^(10-E) stays a normal float
       if (lane == 0) P.sig[j] = 10 - E;      // fp16 high/low split near 2^10
+    } else if (j == kHeads && KQ8) {
+      store_key_q8(ablk, pos % kPage, x, lane);
     } else if (j == kHeads) {
       float u[4];
       VecOut o;
@@ -1297,14 +1388,27 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       out4[t * 128 + 16 * warp + g + 8] = (c[2] + c[3]) * inv;
     }
   };
-  if (warp < kQjlRows / 16) {             // warp-uniform: eight warps own the 128 sketch rows
+  if (!KQ8 && warp < kQjlRows / 16) {     // warp-uniform: eight warps own the 128 sketch rows
 #pragma unroll
     for (int h = 0; h < NH; ++h) sketch_product(&P.qt[4 * h][0], &P.sig[4 * h], 8, &P.pp[4 * h][0]);
     if (ablk) sketch_product(P.u, &P.sig[kHeads], 2, P.z);
   }
   __syncthreads();
-  for (int j = warp; j < kHeads + (ablk ? 1 : 0); j += W) {
-    if (j < kHeads) {
+  for (int j = warp; j < kHeads + (!KQ8 && ablk ? 1 : 0); j += W) {
+    if (j < kHeads && KQ8) {                         // q8_0 keys: query limbs only
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] = P.qt[j][4 * lane + e];
+      const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
+      const Limbs lq = split3(x, eq);
+      uint32_t* lm = P.limb[j];
+      lm[0 * 32 + lane] = lq.w0;  lm[1 * 32 + lane] = lq.w1;  lm[2 * 32 + lane] = lq.w2;
+      if (lane == 0) {
+        P.cst[j][0] = j < A.group ? A.scale * kLog2e * pow2i(-eq) : 0.0f;
+        P.cst[j][1] = 0.0f;
+        P.cst[j][2] = __int_as_float(0);
+      }
+    } else if (j < kHeads) {
       float x[4], pv[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -1408,16 +1512,26 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     const uint8_t* blk = stage0 + s * kBlock;
 
     // ---- this lane's operands from the staged block (tokens g and g + 8)
+    // (q8_0 keys: 16 words of int8 key values, the same count as 2 * 8 code words)
     uint32_t kw[2 * BK];
     lds_words<2 * BK>(reinterpret_cast<const uint32_t*>(blk) + lane * 2 * BK, kw);
-    const uint2 sw = reinterpret_cast<const uint2*>(blk + kSignOff)[lane];
+    uint2 sw = make_uint2(0u, 0u);
+    uint4 sc4 = make_uint4(0u, 0u, 0u, 0u);   // q8_0: fp16 block scales 4 th + kt of tokens g, g + 8
+    if constexpr (KQ8) sc4 = *reinterpret_cast<const uint4*>(blk + kSignOff + 16 * g);
+    else sw = reinterpret_cast<const uint2*>(blk + kSignOff)[lane];
     uint32_t vw[2 * BV];
     if constexpr (!LOGITS) lds_words<2 * BV>(reinterpret_cast<const uint32_t*>(blk + kVOff) + lane * 2 * BV, vw);
     const uint32_t* nrm = reinterpret_cast<const uint32_t*>(blk + kNormOff);
-    const uint32_t rk = nrm[g], rg = nrm[8 + g], rv = nrm[16 + g];
-    const float2 nK = __half22float2(*reinterpret_cast<const __half2*>(&rk));
-    const float2 gm = __half22float2(*reinterpret_cast<const __half2*>(&rg));
-    const float2 nV = __half22float2(*reinterpret_cast<const __half2*>(&rv));
+    float2 nK = make_float2(0.0f, 0.0f), gm = make_float2(0.0f, 0.0f), nV;
+    if constexpr (KQ8) {
+      const uint32_t rv = nrm[g];
+      nV = __half22float2(*reinterpret_cast<const __half2*>(&rv));
+    } else {
+      const uint32_t rk = nrm[g], rg = nrm[8 + g], rv = nrm[16 + g];
+      nK = __half22float2(*reinterpret_cast<const __half2*>(&rk));
+      gm = __half22float2(*reinterpret_cast<const __half2*>(&rg));
+      nV = __half22float2(*reinterpret_cast<const __half2*>(&rv));
+    }
 
     // ---- logits: int8 tensor-core products, tokens on the rows
     int dh[NH][2][4], dl[NH][2][4], ds[NH][2][4];
@@ -1427,6 +1541,44 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) dh[h][nt][c] = dl[h][nt][c] = ds[h][nt][c] = 0;
+    float lq8[NH][2];                        // q8_0: sum over blocks of d_b <Q_b, k8_b>
+    if constexpr (KQ8) {
+      float dsc[2][4];
+      {
+        const uint32_t sw4[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&sw4[i]));
+          dsc[i >> 1][2 * (i & 1)] = f.x;
+          dsc[i >> 1][2 * (i & 1) + 1] = f.y;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < NH; ++h) lq8[h][0] = lq8[h][1] = 0.0f;
+#pragma unroll
+      for (int kt = 0; kt < 4; ++kt) {
+        // A fragment of block kt: tokens g, g + 8 (rows), coordinates 4t.. and 16+4t.. (columns)
+        const uint32_t ak[4] = {kw[2 * kt], kw[8 + 2 * kt], kw[2 * kt + 1], kw[8 + 2 * kt + 1]};
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+          if constexpr (kRegQ) {
+            mma_s8(d0, ak, bq[h][kt][0][0], bq[h][kt][0][1]);
+            mma_s8(d1, ak, bq[h][kt][1][0], bq[h][kt][1][1]);
+          } else {
+            mma_s8(d0, ak, qword(h, 0, kt, 0, 0), qword(h, 0, kt, 0, 1));
+            mma_s8(d1, ak, qword(h, 0, kt, 1, 0), qword(h, 0, kt, 1, 1));
+          }
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            // columns: (Q2, Q1) of head t in d0, Q0 in d1; |Q2 . k| 2^16 can pass 2^31, so in fp32
+            const float m = fmaf(65536.0f, static_cast<float>(d0[2 * r]),
+                                 fmaf(256.0f, static_cast<float>(d0[2 * r + 1]), static_cast<float>(d1[2 * r])));
+            lq8[h][r] = fmaf(dsc[r][kt], m, lq8[h][r]);
+          }
+        }
+      }
+    } else {
     uint32_t sel0[8], sel1[8];
     key_selectors<BK>(kw, sel0);
     key_selectors<BK>(kw + BK, sel1);
@@ -1457,6 +1609,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
           mma_s8(ds[h][nt], as, r0, r1);
         }
     }
+    }
 
     // ---- softmax: one running maximum of l2 + log2|v| per head. The fp16 weight
     // of token t is w_t = 2^(l2_t + log2|v_t| - m) <= 2^8 (the maximum is only
@@ -1475,12 +1628,18 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       for (int r = 0; r < 2; ++r) {
         // accumulator columns: n-tile 0 -> (Q2, Q1) of head t, n-tile 1 -> (Q0, 0)
         //   <Q,C> = 2^16 (256 Q2.Chi + Q2.Clo + Q1.Chi) + 256 (Q1.Clo + Q0.Chi) + Q0.Clo
-        const int hiw = 256 * dh[h][0][2 * r] + dl[h][0][2 * r] + dh[h][0][2 * r + 1];
-        const int low = 256 * (dl[h][0][2 * r + 1] + dh[h][1][2 * r]) + dl[h][1][2 * r];
-        const float main = fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
-        const int sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + ds[h][1][2 * r];
-        const float nk = r ? nK.y : nK.x, gg = r ? gm.y : gm.x, lv = r ? lgv1 : lgv0;
-        const float l2 = fmaf(nk * ca[h], main, gg * cb[h] * static_cast<float>(2 * sj - csum[h]));
+        const float lv = r ? lgv1 : lgv0;
+        float l2;
+        if constexpr (KQ8) {
+          l2 = ca[h] * lq8[h][r];
+        } else {
+          const int hiw = 256 * dh[h][0][2 * r] + dl[h][0][2 * r] + dh[h][0][2 * r + 1];
+          const int low = 256 * (dl[h][0][2 * r + 1] + dh[h][1][2 * r]) + dl[h][1][2 * r];
+          const float main = fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
+          const int sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + ds[h][1][2 * r];
+          const float nk = r ? nK.y : nK.x, gg = r ? gm.y : gm.x;
+          l2 = fmaf(nk * ca[h], main, gg * cb[h] * static_cast<float>(2 * sj - csum[h]));
+        }
         if constexpr (LOGITS) {               // natural-log logit of (token g + 8r, head 4h + t)
           const int qi = 4 * h + t;
           if ((g + 8 * r) < n_valid && qi < A.group)
@@ -1746,7 +1905,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
 template <int BK, int BV, int NH, int MODE>
 cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
   constexpr int W = DecodeWarps<NH>::value;
-  constexpr int kBlock = 256 * (BK + BV + 1) + 96;
+  constexpr int kBlock = block_bytes_of(BK, BV);
   constexpr int S = decode_stages(W, kBlock);
   // main loop: stages, barriers, prologue scratch, the chunk's block-table window
   const size_t pipe = static_cast<size_t>(W) * S * kBlock + W * S * sizeof(uint64_t) + sizeof(Prologue<NH>) +
@@ -1795,7 +1954,9 @@ cudaError_t dispatch_bk(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStr
   switch (T.key_bits) {
     case 2: return dispatch_bv<2, MODE>(T, a, grid, s);
     case 3: return dispatch_bv<3, MODE>(T, a, grid, s);
-    default: return dispatch_bv<4, MODE>(T, a, grid, s);
+    case 4: return dispatch_bv<4, MODE>(T, a, grid, s);
+    case 8: return dispatch_bv<8, MODE>(T, a, grid, s);
+    default: return cudaErrorNotSupported;
   }
 }
 
@@ -1897,7 +2058,8 @@ cudaError_t launch_quantize_prefill(const Tables& t, const void* k, const void* 
   switch (t.key_bits) {
     case 2: return prefill_bv<2>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
     case 3: return prefill_bv<3>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
-    default: return prefill_bv<4>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
+    case 4: return prefill_bv<4>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
+    default: return prefill_bv<8>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos, cache, n_pages, s);
   }
 }
 
