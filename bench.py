@@ -322,7 +322,7 @@ class DecodeBench:
             return a.elapsed_time(b) / 1e3 / (reps * layers)
 
         ours = time_it(run_ours, self.n_layers)
-        key_bytes = self.cache_tokens * n_kv * (16 * wl.key_bits + 16 + 4)
+        key_bytes = self.cache_tokens * n_kv * key_bytes_per_token(wl.key_bits)
         res = {"kernel": "decode_kernel (logits mode) via tq_decode_logits", "us_per_layer": ours * 1e6,
                "key_bytes_per_layer": key_bytes, "gbs": key_bytes / ours / 1e9,
                "logit_bytes_written": nq * int(self.lens[last].sum().item()) * 4}
@@ -417,6 +417,16 @@ class DecodeBench:
         return self.capture(body, range(reps))
 
 
+def key_bytes_per_token(key_bits):
+    """Key bytes one token-head contributes to its logits: q8_0 = 128 int8 values + 4 fp16
+    block scales; TurboQuant = b-bit codes + 128 sign bits + fp16 norm and residual norm."""
+    return 136 if key_bits == 8 else 16 * key_bits + 16 + 4
+
+
+def key_format(key_bits):
+    return "q8_0 keys" if key_bits == 8 else f"{key_bits}-bit keys + QJL"
+
+
 def max_over_ranks(x, world, device):
     """The largest of the ranks' values (every rank gets it); x itself when world == 1."""
     if world == 1:
@@ -454,11 +464,12 @@ def oracle_sample(wl, budget_s=12.0, gpu_cache=None):
     step time is extrapolated to all KV heads and layers.
     """
     import threadpoolctl
-    from oracle import decode as odec, layout as lay, quantize as oq, codebook as ocb, rng as orng
+    from oracle import decode as odec, layout as lay, quantize as oq, codebook as ocb, rng as orng, q8 as oq8
     from decode_attention_seeded_b200 import synth
     gen = synth.Generator(wl, layer=0)
     seeds = gen.method_seeds()
-    kb, vb = ocb.codebook(wl.key_bits), ocb.codebook(wl.value_bits)
+    q8k = wl.key_bits == 8
+    kb, vb = ocb.codebook(2 if q8k else wl.key_bits), ocb.codebook(wl.value_bits)
     tab = dict(signs_k=orng.sign_vector(seeds[0], 128), signs_v=orng.sign_vector(seeds[1], 128),
                sketch=orng.gaussian_sketch(seeds[2], 128, 128), centroids_k=kb.centroids,
                centroids_v=vb.centroids, bk=wl.key_bits, bv=wl.value_bits)
@@ -469,9 +480,14 @@ def oracle_sample(wl, budget_s=12.0, gpu_cache=None):
         # packed bytes of a synthetic cache (random bits: the oracle's cost does not depend on them)
         npg = (T + 15) // 16
         blocks = rng.integers(0, 256, size=(npg, lay.block_bytes(wl.key_bits, wl.value_bits)), dtype=np.uint8)
-        no = lay.section_offsets(wl.key_bits, wl.value_bits)["norm"]
-        blocks[:, no:no + 96] = np.frombuffer(
-            np.abs(rng.standard_normal((npg, 48))).astype(np.float16).tobytes(), dtype=np.uint8).reshape(npg, 96)
+        off = lay.section_offsets(wl.key_bits, wl.value_bits)
+        no, nn = off["norm"], blocks.shape[1] - off["norm"]
+        blocks[:, no:] = np.frombuffer(np.abs(rng.standard_normal((npg, nn // 2))).astype(np.float16).tobytes(),
+                                       dtype=np.uint8).reshape(npg, nn)
+        if q8k:                                    # finite fp16 block scales
+            so = off["sign"]                       # the scale section
+            blocks[:, so:so + 128] = np.frombuffer(np.abs(rng.standard_normal((npg, 64))).astype(np.float16)
+                                                   .tobytes(), dtype=np.uint8).reshape(npg, 128)
     else:
         blocks = gpu_cache
     bt = np.arange(blocks.shape[0])
@@ -480,12 +496,22 @@ def oracle_sample(wl, budget_s=12.0, gpu_cache=None):
     with threadpoolctl.threadpool_limits(1):
         while True:
             x = rng.standard_normal((1, 128))
-            oq.quantize(x, tab["signs_k"], kb.centroids, kb.thresholds, tab["sketch"])
+            if q8k:
+                oq8.quantize_q8(x)
+            else:
+                oq.quantize(x, tab["signs_k"], kb.centroids, kb.thresholds, tab["sketch"])
             oq.quantize(x, tab["signs_v"], vb.centroids, vb.thresholds)
-            kc, sb, vc, nk, gm, nv = odec.gather_sequence(blocks[:, None, :], bt, T, 0, wl.key_bits, wl.value_bits)
+            if q8k:
+                k8, sc, vc, nv = odec.gather_sequence_q8(blocks[:, None, :], bt, T, 0, wl.value_bits)
+            else:
+                kc, sb, vc, nk, gm, nv = odec.gather_sequence(blocks[:, None, :], bt, T, 0, wl.key_bits,
+                                                              wl.value_bits)
             for hh in range(g):
-                qt, p = odec.transform_query(rng.standard_normal(128), tab["signs_k"], tab["sketch"])
-                lg = odec.logits(qt, p, kc, nk, gm, sb, kb.centroids, 1 / np.sqrt(128), 128)
+                if q8k:
+                    lg = oq8.logits_q8(rng.standard_normal(128), k8, sc, 1 / np.sqrt(128))
+                else:
+                    qt, p = odec.transform_query(rng.standard_normal(128), tab["signs_k"], tab["sketch"])
+                    lg = odec.logits(qt, p, kc, nk, gm, sb, kb.centroids, 1 / np.sqrt(128), 128)
                 odec.attend(lg, vc, nv, vb.centroids, tab["signs_v"])
             heads_done += 1
             el = time.perf_counter() - t0
@@ -607,12 +633,12 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": t_main / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": f"int8/fp16 tensor-core, fp32 accumulate ({wl.key_bits}-bit keys + QJL, {wl.value_bits}-bit values)",
+        "dtype": f"int8/fp16 tensor-core, fp32 accumulate ({key_format(wl.key_bits)}, {wl.value_bits}-bit values)",
         "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
                    "head_dim": 128, "context": wl.context, "context_lens": [int(x) for x in bench.lens0[:16]],
                    "layers": bench.n_layers, "key_bits": wl.key_bits,
-                   "value_bits": wl.value_bits, "qjl_rows": 128, "page_tokens": 16,
+                   "value_bits": wl.value_bits, "qjl_rows": 0 if wl.key_bits == 8 else 128, "page_tokens": 16,
                    "l2": f"inputs larger than L2: {bench.n_layers} layer caches, "
                          f"{bench.n_layers * bench.caches[0][1] * bench.page_bytes / 1e9:.2f} GB per step",
                    "parallelism": f"replica x{world} (each GPU serves its own batch)",

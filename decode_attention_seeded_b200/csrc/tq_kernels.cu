@@ -1579,36 +1579,36 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
         }
       }
     } else {
-    uint32_t sel0[8], sel1[8];
-    key_selectors<BK>(kw, sel0);
-    key_selectors<BK>(kw + BK, sel1);
+      uint32_t sel0[8], sel1[8];
+      key_selectors<BK>(kw, sel0);
+      key_selectors<BK>(kw + BK, sel1);
 #pragma unroll
-    for (int kt = 0; kt < 4; ++kt) {
-      uint32_t ah[4], al[4], as[4];
-      key_limbs<BK>(sel0[2 * kt], kth_, ktl_, ah[0], al[0]);          // token g,     k 4t..
-      key_limbs<BK>(sel1[2 * kt], kth_, ktl_, ah[1], al[1]);          // token g + 8, k 4t..
-      key_limbs<BK>(sel0[2 * kt + 1], kth_, ktl_, ah[2], al[2]);      // token g,     k 16+4t..
-      key_limbs<BK>(sel1[2 * kt + 1], kth_, ktl_, ah[3], al[3]);      // token g + 8, k 16+4t..
-      as[0] = (kt == 0 ? sw.x : __umulhi(sw.x, 1u << (32 - 2 * kt))) & 0x01010101u;
-      as[1] = (kt == 0 ? sw.y : __umulhi(sw.y, 1u << (32 - 2 * kt))) & 0x01010101u;
-      as[2] = __umulhi(sw.x, 1u << (31 - 2 * kt)) & 0x01010101u;
-      as[3] = __umulhi(sw.y, 1u << (31 - 2 * kt)) & 0x01010101u;
+      for (int kt = 0; kt < 4; ++kt) {
+        uint32_t ah[4], al[4], as[4];
+        key_limbs<BK>(sel0[2 * kt], kth_, ktl_, ah[0], al[0]);          // token g,     k 4t..
+        key_limbs<BK>(sel1[2 * kt], kth_, ktl_, ah[1], al[1]);          // token g + 8, k 4t..
+        key_limbs<BK>(sel0[2 * kt + 1], kth_, ktl_, ah[2], al[2]);      // token g,     k 16+4t..
+        key_limbs<BK>(sel1[2 * kt + 1], kth_, ktl_, ah[3], al[3]);      // token g + 8, k 16+4t..
+        as[0] = (kt == 0 ? sw.x : __umulhi(sw.x, 1u << (32 - 2 * kt))) & 0x01010101u;
+        as[1] = (kt == 0 ? sw.y : __umulhi(sw.y, 1u << (32 - 2 * kt))) & 0x01010101u;
+        as[2] = __umulhi(sw.x, 1u << (31 - 2 * kt)) & 0x01010101u;
+        as[3] = __umulhi(sw.y, 1u << (31 - 2 * kt)) & 0x01010101u;
 #pragma unroll
-      for (int h = 0; h < NH; ++h)
+        for (int h = 0; h < NH; ++h)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          uint32_t q0, q1, r0, r1;
-          if constexpr (kRegQ) {
-            q0 = bq[h][kt][nt][0]; q1 = bq[h][kt][nt][1]; r0 = bp[h][kt][nt][0]; r1 = bp[h][kt][nt][1];
-          } else {
-            q0 = qword(h, 0, kt, nt, 0); q1 = qword(h, 0, kt, nt, 1);
-            r0 = qword(h, 1, kt, nt, 0); r1 = qword(h, 1, kt, nt, 1);
+          for (int nt = 0; nt < 2; ++nt) {
+            uint32_t q0, q1, r0, r1;
+            if constexpr (kRegQ) {
+              q0 = bq[h][kt][nt][0]; q1 = bq[h][kt][nt][1]; r0 = bp[h][kt][nt][0]; r1 = bp[h][kt][nt][1];
+            } else {
+              q0 = qword(h, 0, kt, nt, 0); q1 = qword(h, 0, kt, nt, 1);
+              r0 = qword(h, 1, kt, nt, 0); r1 = qword(h, 1, kt, nt, 1);
+            }
+            mma_s8(dh[h][nt], ah, q0, q1);
+            mma_s8(dl[h][nt], al, q0, q1);
+            mma_s8(ds[h][nt], as, r0, r1);
           }
-          mma_s8(dh[h][nt], ah, q0, q1);
-          mma_s8(dl[h][nt], al, q0, q1);
-          mma_s8(ds[h][nt], as, r0, r1);
-        }
-    }
+      }
     }
 
     // ---- softmax: one running maximum of l2 + log2|v| per head. The fp16 weight

@@ -67,6 +67,9 @@ WORKLOADS = {
     "llama70b": Workload("llama70b", 3, 1, 64, 8, 131072, 3, 2, "bf16", True, 0.0, 0, 1.0,
                          decode_steps=32),
     "cmdr104b": Workload("cmdr104b", 4, 4, 96, 8, 131072, 4, 2, "bf16", False, 0.01, 0, 20.0),
+    # the llama8b cache with q8_0 keys and 3-bit TurboQuant values (the asymmetric setting)
+    "llama8b_q8k": Workload("llama8b_q8k", 1, 1, 32, 8, 32768, 8, 3, "bf16", True, 0.02, 0, 10.0,
+                            n_layers=32, decode_steps=128),
 }
 
 

@@ -212,3 +212,62 @@ def test_q8_decode_step_appends_and_attends():
         want = odec.decode_paged(host, bt, lens, q.astype(np.float64), tab)
         print("worst rel err", assert_outputs_close(out.cpu().numpy().astype(np.float64), want))
     assert ctx.device_error() == 0
+
+
+def test_q8_full_size_sampled_parity():
+    """Llama-8B 32K with q8_0 keys and 3-bit values, in the launch configuration bench.py times:
+    prefill of the whole context, one decode step; sampled rows and one KV head's decode
+    against the oracle."""
+    wl = synth.WORKLOADS["llama8b_q8k"]
+    gen = synth.Generator(wl)
+    seeds = gen.method_seeds()
+    tab = dict(oracle_tables(seeds, 2, wl.value_bits), bk=8)
+    ctx = binding.Context(8, wl.value_bits, seeds, device=0)
+    L = int(gen.seq_lens()[0])
+    bt, n_pages = gen.page_pool(np.array([(L + 1 + 15) // 16]))
+    n_kv = wl.n_kv_heads
+    cache = torch.zeros(n_pages * ctx.page_bytes(n_kv), dtype=torch.uint8, device=DEV)
+    btt = torch.from_numpy(bt).to(DEV)
+    tg = torch.Generator(device=DEV)
+    tg.manual_seed(4242)
+    sk = torch.from_numpy(gen.scales["k"]).float().to(DEV)
+    sv = torch.from_numpy(gen.scales["v"]).float().to(DEV)
+    k = (torch.randn((L, n_kv, 128), generator=tg, device=DEV) * sk).to(torch.bfloat16)
+    v = (torch.randn((L, n_kv, 128), generator=tg, device=DEV) * sv).to(torch.bfloat16)
+    ctx.quantize_prefill(k, v, btt[0], 0, cache, n_pages)
+    k_new = (torch.randn((1, n_kv, 128), generator=tg, device=DEV) * sk).to(torch.bfloat16)
+    v_new = (torch.randn((1, n_kv, 128), generator=tg, device=DEV) * sv).to(torch.bfloat16)
+    q = torch.randn((1, wl.n_q_heads, 128), generator=tg, device=DEV).to(torch.bfloat16)
+    ws = torch.zeros(ctx.decode_workspace_bytes(1, wl.n_q_heads, n_kv, L + 1), dtype=torch.uint8, device=DEV)
+    out = torch.full((1, wl.n_q_heads, 128), float("nan"), device=DEV)
+    ctx.decode_step(k_new, v_new, q, cache, n_pages, btt, torch.tensor([L + 1], dtype=torch.int32, device=DEV),
+                    n_kv, L + 1, out, ws)
+    torch.cuda.synchronize()
+    assert ctx.device_error() == 0
+    cache3 = cache.view(n_pages, n_kv, ctx.block_bytes)
+    rng = np.random.default_rng(5)
+    pos = np.append(rng.choice(L, size=200, replace=False), L)
+    heads = rng.integers(0, n_kv, size=len(pos))
+    kn, vn_ = k.float().cpu().numpy(), v.float().cpu().numpy()
+    knew, vnew = k_new.float().cpu().numpy()[0], v_new.float().cpu().numpy()[0]
+    bad = 0
+    for p, h in zip(pos, heads):
+        kr = (knew[h] if p == L else kn[p, h]).astype(np.float64)
+        vr = (vnew[h] if p == L else vn_[p, h]).astype(np.float64)
+        vals, sc, vc, vnorm = lay.read_page_q8(cache3[int(bt[0, p // 16]), int(h)].cpu().numpy(), wl.value_bits)
+        kq = q8.quantize_q8(kr)
+        near = np.abs(np.abs(kq.ratio) % 1.0 - 0.5) < 1e-5
+        bad += int(np.sum((vals[p % 16] != kq.values) & ~near))
+        assert np.all(half_ulps_apart(sc[p % 16], kq.scales16) <= 1)
+        _, qv = oracle_quantize(kr[None], vr[None], tab)
+        bad += int(np.sum((vc[p % 16] != qv.codes[0]) & ~near_boundary(qv.y[0], tab["thresholds_v"])))
+        assert half_ulps_apart(np.array([vnorm[p % 16]]), np.array([qv.norm16[0]]))[0] <= 1
+    assert bad == 0
+    g = wl.group
+    h = int(rng.integers(0, n_kv))
+    pg = bt[0, :(L + 1 + 15) // 16]
+    sub = cache3[torch.from_numpy(pg.astype(np.int64)).to(DEV), h].cpu().numpy()[:, None, :]
+    qn = q.float().cpu().numpy().astype(np.float64)
+    want = odec.decode_paged(sub, np.arange(len(pg))[None], [L + 1], qn[:, h * g:(h + 1) * g], tab)
+    got = out.cpu().numpy().astype(np.float64)[:, h * g:(h + 1) * g]
+    print("q8 full size: decode worst rel err", assert_outputs_close(got, want))
