@@ -25,6 +25,13 @@
  *     reads (and clears) it.
  *   - Fixed geometry in this version: head_dim d = 128, QJL rows m = 128,
  *     16 tokens per page, key/value code widths 2, 3 or 4 bits.
+ *   - Asymmetric cache (key_bits = 8): keys are kept in q8_0 blocks instead of
+ *     TurboQuant codes (wis-web.com llama.cpp-fork post, first finding: values
+ *     tolerate 2-3 bits when keys stay in q8_0). Each key is cut into 4 blocks of
+ *     32 coordinates; a block stores d = max|x| / 127 as fp16 and rint(x / d) as
+ *     int8 (0 for an all-zero block); no rotation and no QJL bits. Values are
+ *     TurboQuant codes as above. Decode uses the raw query against the int8
+ *     values, scaled per block.
  */
 #ifndef TQ_H_
 #define TQ_H_
@@ -85,12 +92,14 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
  * advance, so no quantisation constants are stored; turbo2/3/4 = 2/3/4 bits).
  * Law: one coordinate of a uniform point on the unit sphere, density
  * proportional to (1-t^2)^((d-3)/2). Centroids are rounded to fp16; thresholds
- * are midpoints of adjacent stored centroids. key_bits, value_bits in {2,3,4}.
+ * are midpoints of adjacent stored centroids. key_bits in {2,3,4,8} (8: q8_0
+ * keys, no key codebook), value_bits in {2,3,4}.
  */
 tq_status tq_init_codebooks(tq_ctx* ctx, int key_bits, int value_bits, tq_stream stream);
 
 /* Bytes of one (page, KV head) block and of one physical page (all KV heads):
- * block = 16 * (16*key_bits + 16 + 4 + 16*value_bits + 2). 0 if not initialised. */
+ * block = 16 * (16*key_bits + 16 + 4 + 16*value_bits + 2); with q8_0 keys
+ * block = 16 * (128 + 8 + 16*value_bits + 2). 0 if not initialised. */
 size_t tq_block_bytes(const tq_ctx* ctx);
 size_t tq_page_bytes(const tq_ctx* ctx, int n_kv_heads);
 
