@@ -7,6 +7,7 @@
 #include "tq.h"
 #include "tq_internal.h"
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -200,7 +201,7 @@ struct tq_ctx {
   float sparse_tau = 0.0f;         // Sparse V threshold of the decode calls (0: dense)
   bool rot_ready = false, cb_ready = false;
   float* d_signs = nullptr;        // [2][128]: D_K then D_V
-  uint16_t* d_sketch_t = nullptr;  // fp16 bits: S^T, S as decode A fragments, S as prefill B fragments
+  uint16_t* d_sketch_t = nullptr;  // fp16 bits: S^T, M = S R_K (high, low) as decode A fragments, S as prefill B fragments
   unsigned* d_err = nullptr;
   tq::Tables tables;
 };
@@ -371,7 +372,7 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   cudaError_t e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, device);
   if (e == cudaSuccess && c->sm_count <= 0) e = cudaErrorInvalidDevice;
   if (e == cudaSuccess) e = cudaMalloc(&c->d_signs, 2 * tq::kHeadDim * sizeof(float));
-  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 3 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
+  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 4 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
   if (e == cudaSuccess) e = cudaMalloc(&c->d_err, sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(unsigned));
   if (e != cudaSuccess) {
@@ -381,8 +382,8 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   c->tables.signs_k = c->d_signs;
   c->tables.signs_v = c->d_signs + tq::kHeadDim;
   c->tables.sketch_t = c->d_sketch_t;
-  c->tables.sketch = c->d_sketch_t + tq::kQjlRows * tq::kHeadDim;
-  c->tables.sketch_qb = c->d_sketch_t + 2 * tq::kQjlRows * tq::kHeadDim;
+  c->tables.sketch_m = c->d_sketch_t + tq::kQjlRows * tq::kHeadDim;
+  c->tables.sketch_qb = c->d_sketch_t + 3 * tq::kQjlRows * tq::kHeadDim;
   c->tables.err = c->d_err;
   *out = c;
   return TQ_OK;
@@ -405,7 +406,7 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
   if (tq_status st = check_device(ctx)) return st;
   const int d = tq::kHeadDim, m = tq::kQjlRows;
   std::vector<int8_t> sk(d), sv(d);
-  std::vector<uint16_t> s(m * d), st(3 * m * d);
+  std::vector<uint16_t> s(m * d), st(4 * m * d);
   tq_host_sign_vector(seed_k, d, sk.data());
   tq_host_sign_vector(seed_v, d, sv.data());
   tq_host_gaussian_sketch(seed_s, m, d, s.data());
@@ -416,9 +417,12 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
   }
   for (int r = 0; r < m; ++r)
     for (int c = 0; c < d; ++c) st[c * m + r] = s[r * d + c];   // S^T
-  // S as m16n8k16 A fragments: warp w (rows 16w..16w+15), k-step ks (columns
-  // 16ks..16ks+15), lane (g, t), register j -> row 16w + g + 8(j&1), fp16 pair at
-  // columns 16ks + 2t + 8(j>>1) (+0, +1). Stored [w][ks][lane][j], so one warp's
+  // M = S R_K with R_K = H D_K / sqrt(d), so that p = S q~ = M q needs no rotated
+  // query: row r of S H is the Walsh-Hadamard transform of row r of S. M is kept
+  // as fp16 high and low parts (M ~ hi + lo to about 22 bits) in m16n8k16 A
+  // fragment order: warp w (rows 16w..16w+15), k-step ks (columns 16ks..16ks+15),
+  // lane (g, t), register j -> row 16w + g + 8(j&1), fp16 pair at columns
+  // 16ks + 2t + 8(j>>1) (+0, +1). Stored [hi/lo][w][ks][lane][j], so one warp's
   // register set for one k-step is 512 contiguous bytes.
   // S as m16n8k16 B fragments of the prefill product z = S u (tokens on rows):
   // coordinates and sketch rows both follow a lane's layout chunk. Coordinate
@@ -427,7 +431,7 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
   // 32 (nt >> 2) + 16 ((nt >> 1) & 1) + 4 (c >> 1) + 2 (nt & 1) + (c & 1).
   // Stored [ks][nt][lane][2 regs], lane (g, t): reg 0 = k 2t, 2t+1, reg 1 = k
   // 2t+8, 2t+9, column g.
-  uint16_t* qb = st.data() + 2 * m * d;
+  uint16_t* qb = st.data() + 3 * m * d;
   for (int ks = 0; ks < d / 16; ++ks)
     for (int nt = 0; nt < m / 8; ++nt)
       for (int lane = 0; lane < 32; ++lane)
@@ -439,17 +443,43 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
             const int row = 32 * (nt >> 2) + 16 * ((nt >> 1) & 1) + 4 * (c >> 1) + 2 * (nt & 1) + (c & 1);
             qb[(((ks * (m / 8) + nt) * 32 + lane) * 2 + r) * 2 + h] = s[row * d + coord];
           }
-  uint16_t* frag = st.data() + m * d;
-  for (int w = 0; w < m / 16; ++w)
-    for (int ks = 0; ks < d / 16; ++ks)
-      for (int lane = 0; lane < 32; ++lane)
-        for (int j = 0; j < 4; ++j) {
-          const int row = 16 * w + (lane >> 2) + 8 * (j & 1);
-          const int col = 16 * ks + 2 * (lane & 3) + 8 * (j >> 1);
-          const int o = (((w * (d / 16) + ks) * 32 + lane) * 4 + j) * 2;
-          frag[o] = s[row * d + col];
-          frag[o + 1] = s[row * d + col + 1];
+  std::vector<uint16_t> mhi(m * d), mlo(m * d);
+  double rownorm = 0.0;
+  for (int r = 0; r < m; ++r) {
+    std::vector<double> row(d);
+    for (int c = 0; c < d; ++c) row[c] = half_bits_to_double(s[r * d + c]);
+    for (int len = 1; len < d; len <<= 1)            // row H (H symmetric, unnormalised)
+      for (int i = 0; i < d; i += 2 * len)
+        for (int k = i; k < i + len; ++k) {
+          const double a = row[k], bb = row[k + len];
+          row[k] = a + bb;
+          row[k + len] = a - bb;
         }
+    double nn = 0.0;
+    for (int c = 0; c < d; ++c) {
+      const double v = row[c] * sk[c] / std::sqrt(static_cast<double>(d));
+      mhi[r * d + c] = to_half_bits(v);
+      mlo[r * d + c] = to_half_bits(v - half_bits_to_double(mhi[r * d + c]));
+      const double kept = half_bits_to_double(mhi[r * d + c]) + half_bits_to_double(mlo[r * d + c]);
+      nn += kept * kept;
+    }
+    rownorm = std::max(rownorm, std::sqrt(nn));
+  }
+  for (int hl = 0; hl < 2; ++hl) {
+    const std::vector<uint16_t>& src = hl ? mlo : mhi;
+    uint16_t* frag = st.data() + m * d + hl * m * d;
+    for (int w = 0; w < m / 16; ++w)
+      for (int ks = 0; ks < d / 16; ++ks)
+        for (int lane = 0; lane < 32; ++lane)
+          for (int j = 0; j < 4; ++j) {
+            const int row = 16 * w + (lane >> 2) + 8 * (j & 1);
+            const int col = 16 * ks + 2 * (lane & 3) + 8 * (j >> 1);
+            const int o = (((w * (d / 16) + ks) * 32 + lane) * 4 + j) * 2;
+            frag[o] = src[row * d + col];
+            frag[o + 1] = src[row * d + col + 1];
+          }
+  }
+  ctx->tables.m_rownorm = static_cast<float>(rownorm * (1.0 + 1e-6));
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // Synchronous copies from pageable memory: this is the cold set-up path.
   cudaError_t e = cudaMemcpyAsync(ctx->d_signs, signs.data(), 2 * d * sizeof(float),

@@ -29,7 +29,9 @@ struct Tables {
   const float* signs_k = nullptr;     // device [128], +-1
   const float* signs_v = nullptr;     // device [128], +-1
   const uint16_t* sketch_t = nullptr; // device fp16 bits of S^T, [128 (d)][128 (m)]
-  const uint16_t* sketch = nullptr;   // device fp16 bits of S as m16n8k16 A fragments [8 w][8 ks][32 lane][4 reg][2]
+  const uint16_t* sketch_m = nullptr;  // device fp16 bits of M = S R_K, high then low parts, as m16n8k16 A
+                                       //   fragments [2][8 w][8 ks][32 lane][4 reg][2]
+  float m_rownorm = 0.0f;             // max over rows r of |M_r| (bounds |p_r| <= |M_r| |q|)
   const uint16_t* sketch_qb = nullptr;  // device fp16 bits of S as prefill B fragments [8 ks][16 nt][32 lane][2 reg][2]
   unsigned* err = nullptr;            // device error word
 };

@@ -917,6 +917,8 @@ __device__ __forceinline__ int warp_isum(int v) {
 template <int NH>
 struct DecodeWarps { static constexpr int value = NH == 1 ? 16 : 8; };
 // TMA stages per warp: six when they fit in 160 KB of shared memory, else four.
+constexpr int kAccPitch = 132;      // floats per accumulator column in the CTA merge
+
 __host__ __device__ constexpr int decode_stages(int warps, int block) {
   return warps * 6 * block <= 160 * 1024 ? 6 : warps * 4 * block <= 160 * 1024 ? 4 : 3;
 }
@@ -1065,13 +1067,15 @@ struct DecodeArgs {
 
 // Shared-memory scratch of the prologue (after the stages and barriers).
 // Every member starts on a 16-byte boundary (vector loads read qt and u).
+constexpr int kQrawPitch = 136;     // floats per raw query row: the sketch's B loads avoid bank conflicts
+
 template <int NH>
 struct alignas(16) Prologue {
-  alignas(16) float qt[NH * kGroupHeads][128];     // rotated queries q~
-  alignas(16) float pp[NH * kGroupHeads][128];     // sketch products S q~
+  alignas(16) float qraw[NH * kGroupHeads][kQrawPitch];   // queries as given (fp32)
   alignas(16) uint32_t limb[NH * kGroupHeads][192];  // [which (q, p)][limb 0..2][32 words of 4 int8]
   alignas(16) float cst[NH * kGroupHeads][4];      // a, b, sum P (int bits)
-  alignas(16) float u[128];                        // residual of the appended key
+  alignas(16) float qn[NH * kGroupHeads];          // |q|
+  alignas(16) float u[128];                        // appended key: R_K^T u (original domain)
   alignas(16) float z[128];                        // S u
   alignas(16) float tab[64];                       // key / value thresholds and centroids
   alignas(16) VecOut key[32];                      // appended key: codes and norms per lane
@@ -1160,25 +1164,33 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   int* mylp = s_lp + warp * S;
 
   // The prologue's own loads go out first, ahead of the page stream, so that they
-  // do not queue behind it: this warp's sketch rows as m16n8k16 A fragments and
-  // the input of its first job (query head `warp`, or the new key / value).
-  uint4 afv[8];
-  if (!KQ8 && warp < kQjlRows / 16) {
-    const uint4* F = reinterpret_cast<const uint4*>(T.sketch) + warp * 8 * 32 + lane;
+  // do not queue behind it: the last eight warps' rows of M = S R_K (fp16 high
+  // and low parts as m16n8k16 A fragments) and the inputs of this warp's jobs
+  // (query heads warp, warp + W, ...; with APPEND the new key or value).
+  constexpr int kSkW = W - kQjlRows / 16;          // warps kSkW.. own sketch rows 16 (warp - kSkW) + 0..15
+  const int skw = warp - kSkW;
+  uint4 amh[8], aml[8];
+  if (!KQ8 && skw >= 0) {
+    const uint4* F = reinterpret_cast<const uint4*>(T.sketch_m) + skw * 8 * 32 + lane;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) afv[ks] = __ldg(F + ks * 32);
+    for (int ks = 0; ks < 8; ++ks) {
+      amh[ks] = __ldg(F + ks * 32);
+      aml[ks] = __ldg(F + kQjlRows / 16 * 8 * 32 + ks * 32);
+    }
   }
   const size_t kv_row = static_cast<size_t>(b) * A.n_kv + hk;
-  auto job_input = [&](int j, float (&x)[4]) {
-    x[0] = x[1] = x[2] = x[3] = 0.0f;
-    if (j < kHeads) {
-      if (j < A.group) load_row4(A.q, static_cast<size_t>(b) * A.n_q + hk * A.group + j, A.q_dtype, lane, x);
-    } else if (APPEND && j < kHeads + 2) {
-      load_row4(j == kHeads ? A.k_new : A.v_new, kv_row, A.kv_dtype, lane, x);
-    }
-  };
-  float xin[4];
-  job_input(warp, xin);
+  constexpr int kQJobs = (kHeads + W - 1) / W;     // query heads per warp (at most)
+  float xq[kQJobs][4];
+#pragma unroll
+  for (int i = 0; i < kQJobs; ++i) {
+    const int j = warp + W * i;
+    xq[i][0] = xq[i][1] = xq[i][2] = xq[i][3] = 0.0f;
+    if (j < A.group) load_row4(A.q, static_cast<size_t>(b) * A.n_q + hk * A.group + j, A.q_dtype, lane, xq[i]);
+  }
+  // the append jobs: key (job kHeads) and value (kHeads + 1), on warps kHeads % W, (kHeads + 1) % W
+  const int ajob = warp == kHeads % W ? kHeads : (warp == (kHeads + 1) % W ? kHeads + 1 : -1);
+  float xa[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (APPEND && ajob >= 0) load_row4(ajob == kHeads ? A.k_new : A.v_new, kv_row, A.kv_dtype, lane, xa);
   const float4 sgk = __ldg(reinterpret_cast<const float4*>(T.signs_k) + lane);
   const float4 sgv = __ldg(reinterpret_cast<const float4*>(T.signs_v) + lane);
   // this warp's static pages (lane k holds page p0 + warp + W k), fetched before
@@ -1254,6 +1266,26 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   }
 
   // ---- prologue, while the first pages are in flight
+  // Raw queries for the sketch product, with their fp16 scaling exponents and
+  // norms; the QJL limb sums start at zero.
+  if constexpr (!KQ8) {
+#pragma unroll
+    for (int i = 0; i < kQJobs; ++i) {
+      const int j = warp + W * i;
+      if (j >= kHeads) continue;                   // warp-uniform
+      const float* x = xq[i];
+      const float mx = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+      const float ss = warp_sum(fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], x[3] * x[3]))));
+      reinterpret_cast<float4*>(&P.qraw[j][0])[lane] = make_float4(x[0], x[1], x[2], x[3]);
+      if (lane == 0) {
+        int E = 0;
+        if (mx > 0.0f) E = max(exp_above(mx), -115);   // 2^(10-E) stays a normal float
+        P.sig[j] = 10 - E;                             // fp16 high/low split near 2^10
+        P.qn[j] = sqrtf(ss);
+        P.cst[j][2] = __int_as_float(0);
+      }
+    }
+  }
   if (threadIdx.x < 16) {
     P.tab[threadIdx.x] = T.thr_k[threadIdx.x];
     P.tab[16 + threadIdx.x] = T.cen_k[threadIdx.x];
@@ -1301,75 +1333,80 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     if (phys >= 0 && phys < A.n_pages) ablk = A.cache + (static_cast<int64_t>(phys) * A.n_kv + hk) * kBlock;
     else if (threadIdx.x == 0) set_error(T.err, TQ_DEV_BAD_SLOT);
   }
-  // jobs: kHeads query rotations, then (appender) the key and the value of the new token
-  const int n_jobs = kHeads + (ablk ? 2 : 0);
-  for (int j = warp; j < n_jobs; j += W) {
-    float x[4];
-    if (j == warp) {
+  // Jobs: the query limbs, and (appender) the quantization of the new key and
+  // value. The sketch warps meanwhile form p = M q = S q~ for every query head.
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = xin[e];
-    } else {
-      job_input(j, x);
+  for (int i = 0; i < kQJobs; ++i) {
+    const int j = warp + W * i;
+    if (j >= kHeads) continue;                     // warp-uniform
+    float x[4] = {xq[i][0], xq[i][1], xq[i][2], xq[i][3]};
+    if constexpr (!KQ8) {                          // q~ = H D_K q / sqrt(d); q8_0 keys use q itself
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] *= (&sgk.x)[e];
+      fwht128(x, lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] *= kInvSqrtD;
     }
-    if (j < kHeads) {
-      if constexpr (!KQ8) {                  // q~ = H D_K q / sqrt(d); q8_0 keys use q itself
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] *= (&sgk.x)[e];
-        fwht128(x, lane);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] *= kInvSqrtD;
+    const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
+    const Limbs lq = split3(x, eq);
+    uint32_t* lm = P.limb[j];                      // [which (q, p)][limb 0..2][32 words of 4 int8]
+    lm[0 * 32 + lane] = lq.w0;  lm[1 * 32 + lane] = lq.w1;  lm[2 * 32 + lane] = lq.w2;
+    if (lane == 0) {
+      const bool real = j < A.group;
+      P.cst[j][0] = real ? A.scale * kLog2e * pow2i(-eq - (KQ8 ? 0 : T.k_exp)) : 0.0f;
+      if (KQ8) {
+        P.cst[j][1] = 0.0f;
+        P.cst[j][2] = __int_as_float(0);
       }
-      float mx = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        P.qt[j][4 * lane + e] = x[e];
-        mx = fmaxf(mx, fabsf(x[e]));
-      }
-      mx = warp_max(mx);
-      int E = 0;
-      if (mx > 0.0f) E = max(exp_above(mx), -115);   // 2^(10-E) stays a normal float
-      if (lane == 0) P.sig[j] = 10 - E;      // fp16 high/low split near 2^10
-    } else if (j == kHeads && KQ8) {
-      store_key_q8(ablk, pos % kPage, x, lane);
-    } else if (j == kHeads) {
+    }
+  }
+  if (ablk && ajob == kHeads) {                    // the appended key
+    if constexpr (KQ8) {
+      store_key_q8(ablk, pos % kPage, xa, lane);
+    } else {
       float u[4];
       VecOut o;
-      rotate_and_code(x, sgk, P.tab, P.tab + 16, BK, lane, o, u);
+      rotate_and_code(xa, sgk, P.tab, P.tab + 16, BK, lane, o, u);
+      // S u = M R_K^T u with R_K^T u = D_K H u / sqrt(d)
+      fwht128(u, lane);
       float mx = 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
+        u[e] *= (&sgk.x)[e] * kInvSqrtD;
         P.u[4 * lane + e] = u[e];
         mx = fmaxf(mx, fabsf(u[e]));
       }
       mx = warp_max(mx);
       int E = 0;
-      if (mx > 0.0f) E = max(exp_above(mx), -115);   // 2^(10-E) stays a normal float
+      if (mx > 0.0f) E = max(exp_above(mx), -115);
       if (lane == 0) P.sig[kHeads] = 10 - E;
       P.key[lane] = o;
-    } else {
-      float u[4];
-      VecOut o;
-      rotate_and_code(x, sgv, P.tab + 32, P.tab + 48, BV, lane, o, u);
-      store_value_token(ablk, pos % kPage, BK, BV, o, lane);
-      if (lane == 0) store_norm(ablk, BK, BV, 2, pos % kPage, o.norm);
     }
+  } else if (ablk && ajob == kHeads + 1) {         // the appended value
+    float u[4];
+    VecOut o;
+    rotate_and_code(xa, sgv, P.tab + 32, P.tab + 48, BV, lane, o, u);
+    store_value_token(ablk, pos % kPage, BK, BV, o, lane);
+    if (lane == 0) store_norm(ablk, BK, BV, 2, pos % kPage, o.norm);
   }
-  __syncthreads();
-  // sketch products on the tensor cores: warp w owns sketch rows 16w .. 16w+15; the B
-  // columns are (head h, fp16 high part) and (head h, fp16 low part) of x * 2^sig
-  auto sketch_product = [&](const float* vec4, const int* sig4, int cols, float* out4) {
-    // vec4: column-pair sources (cols/2 vectors of 128); out4: destinations [cols/2][128]
+  // Sketch products on the tensor cores: warp kSkW + w owns rows 16w .. 16w+15 of
+  // M = S R_K, as fp16 high and low parts. The B columns are (source s, fp16 high
+  // part) and (source s, fp16 low part) of x_s * 2^sig_s. On return, lane (g, t)
+  // holds rows 16w + g (c[0] + c[1]) and 16w + g + 8 (c[2] + c[3]) of source t,
+  // still scaled by 2^sig_t.
+  auto sketch_m = [&](const float* vec, int pitch, const int* sig, int sources, float (&c)[4]) {
     const int src = g >> 1;
-    const bool has = src < cols / 2;
-    const float sc = has ? pow2i(sig4[src]) : 0.0f;
+    const bool has = src < sources;
+    const float sc = has ? pow2i(sig[src]) : 0.0f;
     const bool lo_col = g & 1;
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    c[0] = c[1] = c[2] = c[3] = 0.0f;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
       if (has) {
-        u0 = *reinterpret_cast<const float2*>(vec4 + src * 128 + 16 * ks + 2 * t);
-        u1 = *reinterpret_cast<const float2*>(vec4 + src * 128 + 16 * ks + 2 * t + 8);
+        u0 = *reinterpret_cast<const float2*>(vec + src * pitch + 16 * ks + 2 * t);
+        u1 = *reinterpret_cast<const float2*>(vec + src * pitch + 16 * ks + 2 * t + 8);
       }
       const float2 v0 = make_float2(u0.x * sc, u0.y * sc), v1 = make_float2(u1.x * sc, u1.y * sc);
       const __half2 h0 = __floats2half2_rn(v0.x, v0.y), h1 = __floats2half2_rn(v1.x, v1.y);
@@ -1379,57 +1416,77 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
         b0 = __floats2half2_rn(v0.x - r0.x, v0.y - r0.y);
         b1 = __floats2half2_rn(v1.x - r1.x, v1.y - r1.y);
       }
-      mma_f16(c, afv[ks].x, afv[ks].y, afv[ks].z, afv[ks].w, *reinterpret_cast<uint32_t*>(&b0),
-              *reinterpret_cast<uint32_t*>(&b1));
+      const uint32_t ub0 = *reinterpret_cast<uint32_t*>(&b0), ub1 = *reinterpret_cast<uint32_t*>(&b1);
+      mma_f16(c, amh[ks].x, amh[ks].y, amh[ks].z, amh[ks].w, ub0, ub1);
+      mma_f16(d, aml[ks].x, aml[ks].y, aml[ks].z, aml[ks].w, ub0, ub1);
     }
-    if (t < cols / 2) {                     // columns 2t (high) and 2t+1 (low) of source t
-      const float inv = pow2i(-sig4[t]);
-      out4[t * 128 + 16 * warp + g] = (c[0] + c[1]) * inv;
-      out4[t * 128 + 16 * warp + g + 8] = (c[2] + c[3]) * inv;
-    }
-  };
-  if (!KQ8 && warp < kQjlRows / 16) {     // warp-uniform: eight warps own the 128 sketch rows
 #pragma unroll
-    for (int h = 0; h < NH; ++h) sketch_product(&P.qt[4 * h][0], &P.sig[4 * h], 8, &P.pp[4 * h][0]);
-    if (ablk) sketch_product(P.u, &P.sig[kHeads], 2, P.z);
+    for (int e = 0; e < 4; ++e) c[e] += d[e];
+  };
+  if (!KQ8 && skw >= 0) {
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      float c[4];
+      sketch_m(&P.qraw[4 * h][0], kQrawPitch, &P.sig[4 * h], 4, c);
+      // int8 limbs of P = p 2^ep for head j = 4h + t, rows 16 skw + g (+8). The
+      // exponent comes from the bound |p_r| <= |M_r| |q|, the same in every warp.
+      const int j = 4 * h + t;
+      const float inv = pow2i(-P.sig[j]);
+      const float p0 = (c[0] + c[1]) * inv, p1 = (c[2] + c[3]) * inv;
+      const int ep = pick_exponent24(T.m_rownorm * P.qn[j] * 1.0001f);
+      const float f = pow2i(ep);
+      const int Q0 = __float2int_rn(p0 * f), Q1 = __float2int_rn(p1 * f);
+      // limbs of row 16 skw + g go to byte g & 3 of word 4 skw + (g >> 2); row +8 to word + 2
+      const int sh = 8 * (g & 3);
+      uint32_t w[6];
+      {
+        const int a0 = ((Q0 + 128) & 255) - 128, r0 = (Q0 - a0) >> 8, a1 = ((r0 + 128) & 255) - 128;
+        const int b0 = ((Q1 + 128) & 255) - 128, r1 = (Q1 - b0) >> 8, b1 = ((r1 + 128) & 255) - 128;
+        w[0] = static_cast<uint32_t>(a0 & 0xFF) << sh;
+        w[1] = static_cast<uint32_t>(a1 & 0xFF) << sh;
+        w[2] = static_cast<uint32_t>(((r0 - a1) >> 8) & 0xFF) << sh;
+        w[3] = static_cast<uint32_t>(b0 & 0xFF) << sh;
+        w[4] = static_cast<uint32_t>(b1 & 0xFF) << sh;
+        w[5] = static_cast<uint32_t>(((r1 - b1) >> 8) & 0xFF) << sh;
+      }
+#pragma unroll
+      for (int k = 0; k < 6; ++k) {
+        w[k] |= __shfl_xor_sync(kFull, w[k], 4);
+        w[k] |= __shfl_xor_sync(kFull, w[k], 8);
+      }
+      int ps = Q0 + Q1;
+      ps += __shfl_xor_sync(kFull, ps, 4);
+      ps += __shfl_xor_sync(kFull, ps, 8);
+      ps += __shfl_xor_sync(kFull, ps, 16);
+      uint32_t* lm = P.limb[j] + 96;
+      if ((g & 3) == 0) {
+        const int wd = 4 * skw + (g >> 2);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          lm[k * 32 + wd] = w[k];
+          lm[k * 32 + wd + 2] = w[3 + k];
+        }
+      }
+      if (g == 0) {
+        atomicAdd(reinterpret_cast<int*>(&P.cst[j][2]), j < A.group ? ps : 0);
+        if (skw == 0)
+          P.cst[j][1] = j < A.group ? A.scale * kLog2e * kSqrtPiOver2 / kQjlRows * pow2i(-ep) : 0.0f;
+      }
+    }
   }
   __syncthreads();
-  for (int j = warp; j < kHeads + (!KQ8 && ablk ? 1 : 0); j += W) {
-    if (j < kHeads && KQ8) {                         // q8_0 keys: query limbs only
-      float x[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = P.qt[j][4 * lane + e];
-      const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
-      const Limbs lq = split3(x, eq);
-      uint32_t* lm = P.limb[j];
-      lm[0 * 32 + lane] = lq.w0;  lm[1 * 32 + lane] = lq.w1;  lm[2 * 32 + lane] = lq.w2;
-      if (lane == 0) {
-        P.cst[j][0] = j < A.group ? A.scale * kLog2e * pow2i(-eq) : 0.0f;
-        P.cst[j][1] = 0.0f;
-        P.cst[j][2] = __int_as_float(0);
+  if (!KQ8 && ablk) {                              // CTA-uniform: the appended key's sign bits
+    if (skw >= 0) {
+      float c[4];
+      sketch_m(P.u, 128, &P.sig[kHeads], 1, c);
+      if (t == 0) {
+        const float inv = pow2i(-P.sig[kHeads]);
+        P.z[16 * skw + g] = (c[0] + c[1]) * inv;
+        P.z[16 * skw + g + 8] = (c[2] + c[3]) * inv;
       }
-    } else if (j < kHeads) {
-      float x[4], pv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[e] = P.qt[j][4 * lane + e];
-        pv[e] = P.pp[j][4 * lane + e];
-      }
-      const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
-      const int ep = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(pv[0]), fabsf(pv[1])), fmaxf(fabsf(pv[2]), fabsf(pv[3])))));
-      const Limbs lq = split3(x, eq);
-      const Limbs lp = split3(pv, ep);
-      const int psum = warp_isum(lp.sum);            // |sum| < 2^29
-      uint32_t* lm = P.limb[j];                      // [which][limb][32]
-      lm[0 * 32 + lane] = lq.w0;  lm[1 * 32 + lane] = lq.w1;  lm[2 * 32 + lane] = lq.w2;
-      lm[96 + 0 * 32 + lane] = lp.w0; lm[96 + 1 * 32 + lane] = lp.w1; lm[96 + 2 * 32 + lane] = lp.w2;
-      if (lane == 0) {
-        const bool real = j < A.group;
-        P.cst[j][0] = real ? A.scale * kLog2e * pow2i(-eq - T.k_exp) : 0.0f;
-        P.cst[j][1] = real ? A.scale * kLog2e * kSqrtPiOver2 / kQjlRows * pow2i(-ep) : 0.0f;
-        P.cst[j][2] = __int_as_float(real ? psum : 0);
-      }
-    } else {                                         // the appended key: sign bits, store
+    }
+    __syncthreads();
+    if (ajob == kHeads) {
       VecOut o = P.key[lane];
 #pragma unroll
       for (int e = 0; e < 4; ++e) o.sgn[e] = P.z[4 * lane + e] >= 0.0f ? 1 : 0;
@@ -1440,8 +1497,10 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       }
     }
   }
-  if (ablk) asm volatile("fence.proxy.async.global;" ::: "memory");   // the page is next read by the TMA unit
-  __syncthreads();
+  if (ablk) {                                      // CTA-uniform
+    asm volatile("fence.proxy.async.global;" ::: "memory");   // the page is next read by the TMA unit
+    __syncthreads();
+  }
   if (lane == 0 && def_stage >= 0) issue(s_def[warp], held, def_stage);   // the appended page
   __syncwarp();
   __syncwarp();                           // lane 0's stage records are visible to the warp
@@ -1751,8 +1810,10 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     lsum[h] += __shfl_xor_sync(kFull, lsum[h], 16);
   }
   __syncthreads();
-  float* s_acc = reinterpret_cast<float*>(smem);                       // [warp][NH][8 columns][128]
-  float* s_st = s_acc + W * NH * 8 * 128;                                // [warp][NH][4 heads][3]
+  // [warp][NH][8 columns][kAccPitch]: the pitch of 132 floats puts the four
+  // column pairs a quad stores at once in different banks
+  float* s_acc = reinterpret_cast<float*>(smem);
+  float* s_st = s_acc + W * NH * 8 * kAccPitch;                          // [warp][NH][4 heads][3]
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
 #pragma unroll
@@ -1760,7 +1821,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int coord = 16 * mt + g + 8 * (c >> 1), col = 2 * t + (c & 1);
-        s_acc[((warp * NH + h) * 8 + col) * 128 + coord] = acc[h][mt][c];
+        s_acc[((warp * NH + h) * 8 + col) * kAccPitch + coord] = acc[h][mt][c];
       }
     if (g == 0) {
       float* st = s_st + ((warp * NH + h) * kGroupHeads + t) * 3;
@@ -1779,9 +1840,9 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
 #pragma unroll
     for (int w = 0; w < W; ++w) {
       const float* st = s_st + ((w * NH + h) * kGroupHeads + h4) * 3;
-      const float* ac = s_acc + ((w * NH + h) * 8) * 128;
+      const float* ac = s_acc + ((w * NH + h) * 8) * kAccPitch;
       const float f = ex2(st[0] - M);
-      a = fmaf(ac[h4 * 128 + coord] + ac[(h4 + 4) * 128 + coord], f, a);
+      a = fmaf(ac[h4 * kAccPitch + coord] + ac[(h4 + 4) * kAccPitch + coord], f, a);
       l = fmaf(st[1], f, l);
     }
     part[hh * 132 + coord] = a;
@@ -1911,7 +1972,7 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
   const size_t pipe = static_cast<size_t>(W) * S * kBlock + W * S * sizeof(uint64_t) + sizeof(Prologue<NH>) +
                       ((static_cast<size_t>(a.ppc) * 4 + 15) & ~static_cast<size_t>(15));
   // CTA merge: every warp's accumulators and softmax state
-  const size_t merge = static_cast<size_t>(W) * NH * 8 * 128 * 4 + W * NH * kGroupHeads * 3 * 4;
+  const size_t merge = static_cast<size_t>(W) * NH * 8 * kAccPitch * 4 + W * NH * kGroupHeads * 3 * 4;
   const size_t smem = pipe > merge ? pipe : merge;
   // final merge: merge_cap chunk records, then [W / 4][slots][132] floats and one barrier
   const size_t chunk_bytes = static_cast<size_t>(NH) * kGroupHeads * 132 * 4;
