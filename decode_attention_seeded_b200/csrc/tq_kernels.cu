@@ -1146,6 +1146,10 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   constexpr int kNormBytes = KQ8 ? 32 : 96;
   constexpr int kHeads = NH * kGroupHeads;
   constexpr bool kRegQ = NH <= 2;              // query fragments in registers (else shared memory)
+  // Launched as a programmatic dependent of the previous kernel in the stream: its
+  // memory operations are complete and visible once this wait returns, so nothing
+  // of the previous kernel's output is touched before it.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int pair = static_cast<int>(blockIdx.x % static_cast<unsigned>(A.n_pairs));
@@ -1800,6 +1804,9 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   if (lane == 0)
     for (int s2 = 0; s2 < S; ++s2)
       asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(mybar + s2)) : "memory");
+  // the page stream is done: the next kernel in the stream may be scheduled on SMs
+  // this grid frees (it waits for this grid's completion before touching memory)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if constexpr (LOGITS) return;                   // logits are written; nothing to merge
 
   // ---- merge the warps of this CTA (the pipeline buffers are free now)
@@ -1987,8 +1994,18 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  fn<<<grid, W * 32, smem, s>>>(T, args);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(W * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the launch with the previous kernel's tail
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, T, args);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int BK, int BV, int MODE>
