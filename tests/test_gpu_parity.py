@@ -275,3 +275,46 @@ def test_decode_step_api_matches_oracle():
         want = odec.decode_paged(host, bt, lens, q.astype(np.float64), tab)
         assert_outputs_close(out.cpu().numpy().astype(np.float64), want)
     assert ctx.device_error() == 0
+
+
+@pytest.mark.parametrize("path", ["prefill", "append"])
+def test_zero_vectors_and_zero_query(path):
+    """Zero key / value rows quantize to norm 0 (and gamma 0) with no NaN, and a zero
+    query head attends uniformly; both against the oracle from the GPU-written bytes."""
+    bk, bv, n_kv, g, L = 3, 2, 2, 4, 53
+    seeds = (61, 62, 63)
+    tab = oracle_tables(seeds, bk, bv)
+    rng = np.random.default_rng(17)
+    k, v = _rand_kv(rng, L, n_kv, "bf16")
+    k[[5, 17, 40]] = 0.0
+    v[[9, 17]] = 0.0
+    k[30, 1] = 0.0
+    bt, n_pages = _pool([L], 23)
+    ctx = _ctx(bk, bv, seeds)
+    cache = torch.zeros(n_pages * ctx.page_bytes(n_kv), dtype=torch.uint8, device=DEV)
+    btt = torch.from_numpy(bt).to(DEV)
+    if path == "prefill":
+        ctx.quantize_prefill(_t(k, "bf16"), _t(v, "bf16"), btt[0], 0, cache, n_pages)
+    else:
+        slots = torch.from_numpy(synth.slots_for(bt[0], 0, L)).to(DEV)
+        ctx.quantize_append(_t(k, "bf16"), _t(v, "bf16"), slots, cache, n_pages)
+    host = cache.cpu().numpy().reshape(n_pages, n_kv, -1)
+    for h in range(n_kv):
+        qk, qv = oracle_quantize(k[:, h].astype(np.float64), v[:, h].astype(np.float64), tab)
+        fields = unpack_tokens(host, bt[0], 0, L, h, bk, bv)
+        rep = compare_tokens(fields, qk, qv, tab)
+        assert all(val == 0 for key, val in rep.items() if key.startswith("bad")), rep
+        zk = np.all(k[:, h] == 0, axis=1)
+        assert np.all(fields[3][zk] == 0) and np.all(fields[4][zk] == 0)      # key norm, gamma
+        assert np.all(fields[5][np.all(v[:, h] == 0, axis=1)] == 0)           # value norm
+    q = synth.round_to_bf16(rng.standard_normal((1, n_kv * g, 128)).astype(np.float32))
+    q[0, 2] = 0.0
+    ws = torch.zeros(ctx.decode_workspace_bytes(1, n_kv * g, n_kv, L), dtype=torch.uint8, device=DEV)
+    out = torch.full((1, n_kv * g, 128), float("nan"), device=DEV)
+    ctx.decode_attention(_t(q, "bf16"), cache, n_pages, btt, torch.tensor([L], dtype=torch.int32, device=DEV),
+                         n_kv, L, out, ws)
+    assert ctx.device_error() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    want = odec.decode_paged(host, bt, [L], q.astype(np.float64), tab)
+    print("worst rel err", assert_outputs_close(got, want))

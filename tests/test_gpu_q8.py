@@ -271,3 +271,40 @@ def test_q8_full_size_sampled_parity():
     want = odec.decode_paged(sub, np.arange(len(pg))[None], [L + 1], qn[:, h * g:(h + 1) * g], tab)
     got = out.cpu().numpy().astype(np.float64)[:, h * g:(h + 1) * g]
     print("q8 full size: decode worst rel err", assert_outputs_close(got, want))
+
+
+@pytest.mark.parametrize("path", ["prefill", "append"])
+def test_q8_zero_blocks(path):
+    """All-zero 32-coordinate key blocks store scale 0 and values 0; a zero key row and
+    zero value rows decode without NaN; decode matches the oracle on the GPU-written bytes."""
+    bv, n_kv, g, L = 3, 2, 4, 41
+    seeds = (91, 92, 93)
+    tab = dict(oracle_tables(seeds, 2, bv), bk=8)
+    rng = np.random.default_rng(44)
+    k, v = _rows(rng, L, n_kv)
+    k[3, 0, 32:64] = 0.0
+    k[7, 1, 96:] = 0.0
+    k[11] = 0.0
+    v[[11, 20]] = 0.0
+    ctx, cache, bt, n_pages = _gpu_cache(bv, seeds, k, v, path)
+    for t in range(L):
+        for h in range(n_kv):
+            vals, sc, vc, vn = lay.read_page_q8(cache[bt[t // 16], h], bv)
+            kq = q8.quantize_q8(k[t, h])
+            zero = np.all(k[t, h].reshape(4, 32) == 0, axis=1)
+            assert np.all(sc[t % 16][zero] == 0) and np.all(vals[t % 16].reshape(4, 32)[zero] == 0)
+            near = np.abs(np.abs(kq.ratio) % 1.0 - 0.5) < 1e-5
+            assert np.all((vals[t % 16] == kq.values) | near)
+            if np.all(v[t, h] == 0):
+                assert vn[t % 16] == 0
+    q = synth.round_to_bf16(rng.standard_normal((1, n_kv * g, 128)).astype(np.float32))
+    ws = torch.zeros(ctx.decode_workspace_bytes(1, n_kv * g, n_kv, L), dtype=torch.uint8, device=DEV)
+    out = torch.full((1, n_kv * g, 128), float("nan"), device=DEV)
+    dc = torch.from_numpy(cache.reshape(-1)).to(DEV)
+    ctx.decode_attention(torch.from_numpy(q).to(DEV).to(torch.bfloat16), dc, n_pages, torch.from_numpy(bt[None]).to(DEV),
+                         torch.tensor([L], dtype=torch.int32, device=DEV), n_kv, L, out, ws)
+    assert ctx.device_error() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    want = odec.decode_paged(cache, bt[None], [L], q.astype(np.float64), tab)
+    print("worst rel err", assert_outputs_close(got, want))
