@@ -301,10 +301,35 @@ DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int sm_count
   ppc = std::min(std::max(ppc, kMinChunkPages), kMaxChunkPages);
   p.pages_per_chunk = ppc;
   p.chunks = (p.max_pages + ppc - 1) / ppc;
+  p.grid = p.chunks * pairs;
+  // Balanced mode when the uniform split is SM-limited and leaves more than 5 % of
+  // the SMs idle, or needs more than one wave: the split then follows the actual
+  // (ragged) lengths, read on the device.
+  const int sm_chunks = std::max(1, sm_count / pairs);
+  const bool sm_limited = p.chunks == sm_chunks && pairs <= sm_count;
+  const bool idle = sm_limited && (sm_count - p.chunks * pairs) * 20 > sm_count;
+  p.balanced = 0;
+  // (8-warp instantiations only: groups of more than 4 query heads per KV head)
+  if ((idle || pairs > sm_count) && p.n_hg >= 2 && batch <= kMaxBalancedBatch) {
+    const int seg_w = std::max(8, 36 / p.n_hg);
+    const int64_t all = static_cast<int64_t>(pairs) * (p.max_pages + seg_w);
+    const int64_t share = std::max<int64_t>(kMinShare, (all + sm_count - 1) / sm_count) + 2;
+    if (share <= kMaxChunkPages) {
+      p.balanced = 1;
+      p.shares = sm_count;
+      p.grid = sm_count;                           // one CTA per share
+      p.seg_w = seg_w;
+      p.min_share = kMinShare;
+      p.pages_per_chunk = static_cast<int>(share);
+    }
+  }
+  // records: uniform, one per (pair, chunk); balanced, one per segment, at slot
+  // share + pair ordinal (below shares + pairs)
+  const size_t records = p.balanced ? static_cast<size_t>(p.shares) + pairs : static_cast<size_t>(pairs) * p.chunks;
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   size_t off = 0;
   p.off_partial = off;
-  off = al(off + static_cast<size_t>(pairs) * p.chunks * p.n_hg * 4 * 132 * sizeof(float));
+  off = al(off + records * p.n_hg * 4 * 132 * sizeof(float));
   p.off_counter = off;
   off = al(off + static_cast<size_t>(pairs) * sizeof(unsigned));
   p.total = off;

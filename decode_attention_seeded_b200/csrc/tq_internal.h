@@ -41,10 +41,16 @@ struct Tables {
 // chunk * n_pairs + pair, one resident CTA per SM.
 constexpr int kMinChunkPages = 16;
 constexpr int kMaxChunkPages = 8192;
+constexpr int kMinShare = 48;          // balanced mode: least pages per CTA share
+constexpr int kMaxBalancedBatch = 4096;  // balanced mode keeps a [batch + 1] prefix in shared memory
 struct DecodePlan {
   int batch, n_q, n_kv, group, n_hg;  // n_hg = ceil(group / 4) groups of 4 query heads
   int n_pairs;                         // batch * n_kv
   int max_pages, pages_per_chunk, chunks;
+  // Balanced mode (chosen when uniform chunks per pair would leave SMs idle): `grid`
+  // CTAs take equal shares of all pages, each pair counted with seg_w extra pages for
+  // its fixed cost; pages_per_chunk then bounds one CTA's share (its block-table window).
+  int balanced, grid, seg_w, min_share, shares;
   size_t off_partial, off_counter, total;
 };
 

@@ -1059,6 +1059,12 @@ struct DecodeArgs {
   float* out;                    // [batch][n_q][128]
   int n_kv, n_q, group, n_hg, chunks, ppc, n_pairs;
   int merge_cap;                 // chunk records that fit in shared memory for the final merge
+  int batch;
+  int balanced;                  // 0: `chunks` uniform chunks of `ppc` pages per pair; 1: equal shares of all pages
+  int seg_w;                     // balanced: fixed cost of one pair, in pages
+  int min_share;                 // balanced: least share, in pages (fewer shares for small work)
+  int shares;                    // balanced: most shares (the SM count); the grid adds one CTA per pair
+  int vs_off;                    // balanced: byte offset of the [batch + 1] prefix array in shared memory
   int sparse;                    // Sparse V on: values of positions below the threshold are skipped
   float sparse_log2;             // log2 of the Sparse V threshold (relative attention weight)
   float* logits;                 // logits-only mode: [batch][n_q][logits_stride] (natural log units)
@@ -1133,8 +1139,17 @@ __device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float
 // APPEND: the CTA whose chunk holds a sequence's last page first quantizes
 // (k_new, v_new) of that sequence into position seq_len - 1; a warp that is
 // given that page before then holds its copy back until the token is written.
+// One piece of work of a CTA: logical pages [p0, p0 + len) of one (sequence, KV
+// head) pair (clipped to the sequence), whose merged record goes to slot `slot`;
+// the pair's records are slots first_slot .. first_slot + n_segs - 1.
+struct Segment {
+  int pair, p0, len;
+  int slot, first_slot, n_segs;
+  bool last;                     // the CTA's last segment
+};
+
 template <int BK, int BV, int NH, int MODE>
-__global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
+__device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs& A, const Segment& sg) {
   constexpr bool APPEND = MODE == 1;        // append the new token first (decode step)
   constexpr bool LOGITS = MODE == 2;        // write the logits; no softmax, no value sum
   constexpr bool KQ8 = BK == 8;              // q8_0 keys (raw query, block scales, no QJL)
@@ -1146,15 +1161,17 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   constexpr int kNormBytes = KQ8 ? 32 : 96;
   constexpr int kHeads = NH * kGroupHeads;
   constexpr bool kRegQ = NH <= 2;              // query fragments in registers (else shared memory)
-  // Launched as a programmatic dependent of the previous kernel in the stream: its
-  // memory operations are complete and visible once this wait returns, so nothing
-  // of the previous kernel's output is touched before it.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int pair = static_cast<int>(blockIdx.x % static_cast<unsigned>(A.n_pairs));
-  const int chunk = static_cast<int>(blockIdx.x / static_cast<unsigned>(A.n_pairs));
+  const int pair = sg.pair;
   const int b = pair / A.n_kv, hk = pair % A.n_kv;
+  // Table pointers made opaque for this segment: when one CTA serves several
+  // segments, the loads through them must not be hoisted out of the segment loop
+  // (that would keep their registers live across every main loop).
+  const uint16_t* tab_m = T.sketch_m;
+  const float* tab_sk = T.signs_k;
+  const float* tab_sv = T.signs_v;
+  asm volatile("" : "+l"(tab_m), "+l"(tab_sk), "+l"(tab_sv));
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + W * S * kBlock);
   static_assert((W * S * kBlock + W * S * 8) % 16 == 0, "prologue alignment");
@@ -1175,7 +1192,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   const int skw = warp - kSkW;
   uint4 amh[8], aml[8];
   if (!KQ8 && skw >= 0) {
-    const uint4* F = reinterpret_cast<const uint4*>(T.sketch_m) + skw * 8 * 32 + lane;
+    const uint4* F = reinterpret_cast<const uint4*>(tab_m) + skw * 8 * 32 + lane;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       amh[ks] = __ldg(F + ks * 32);
@@ -1195,19 +1212,19 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   const int ajob = warp == kHeads % W ? kHeads : (warp == (kHeads + 1) % W ? kHeads + 1 : -1);
   float xa[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (APPEND && ajob >= 0) load_row4(ajob == kHeads ? A.k_new : A.v_new, kv_row, A.kv_dtype, lane, xa);
-  const float4 sgk = __ldg(reinterpret_cast<const float4*>(T.signs_k) + lane);
-  const float4 sgv = __ldg(reinterpret_cast<const float4*>(T.signs_v) + lane);
+  const float4 sgk = __ldg(reinterpret_cast<const float4*>(tab_sk) + lane);
+  const float4 sgv = __ldg(reinterpret_cast<const float4*>(tab_sv) + lane);
   // this warp's static pages (lane k holds page p0 + warp + W k), fetched before
   // the length is known (bounded by the table width; pages past the sequence are
   // discarded below)
   const int32_t* btab = A.block_tables + static_cast<int64_t>(b) * A.max_pages_per_seq;
-  const int p0 = chunk * A.ppc;
+  const int p0 = sg.p0;
   const int first_j = p0 + warp + lane * W;
   const int spec_phys = (lane < kStatic && first_j < A.max_pages_per_seq) ? __ldg(btab + first_j) : -1;
   // the first kSpecWin entries of the chunk's claimable window, also fetched now
   // (entries past the table width are skipped; past the sequence, never claimed)
   constexpr int kSpecPer = 2, kSpecWin = kSpecPer * W * 32;
-  const int win_lim = min(A.ppc, A.max_pages_per_seq - p0) - W * kStatic;
+  const int win_lim = min(sg.len, A.max_pages_per_seq - p0) - W * kStatic;
   int spec_win[kSpecPer];
 #pragma unroll
   for (int r = 0; r < kSpecPer; ++r) {
@@ -1216,6 +1233,9 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   }
 
   if (lane == 0) {
+    // a previous segment of this CTA may have written these bytes through the
+    // generic proxy; they are next written by bulk copies
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     for (int s = 0; s < S; ++s) mbar_init(mybar + s, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1227,11 +1247,11 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     L = L < 0 ? 0 : A.max_seq_len;
   }
   const int seq_pages = (L + kPage - 1) / kPage;
-  const int p1 = min(p0 + A.ppc, seq_pages);
+  const int p1 = min(p0 + sg.len, seq_pages);
   const int n_static = p1 > p0 + warp ? min(kStatic, (p1 - p0 - warp + W - 1) / W) : 0;
   const int n_dyn = max(0, p1 - p0 - W * kStatic);      // pages handed out by the claim counter
   // the CTA holding the last page appends the new token before that page is fetched
-  const bool appender = APPEND && L > 0 && chunk == (seq_pages - 1) / A.ppc;
+  const bool appender = APPEND && L > 0 && p0 <= seq_pages - 1 && seq_pages - 1 < p0 + sg.len;
   const int held = appender ? seq_pages - 1 : -1;
 
   // lane 0 only: start the transfer of logical page lp (physical `phys`) into stage s
@@ -1806,7 +1826,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
       asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(mybar + s2)) : "memory");
   // the page stream is done: the next kernel in the stream may be scheduled on SMs
   // this grid frees (it waits for this grid's completion before touching memory)
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (sg.last) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if constexpr (LOGITS) return;                   // logits are written; nothing to merge
 
   // ---- merge the warps of this CTA (the pipeline buffers are free now)
@@ -1836,7 +1856,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     }
   }
   __syncthreads();
-  float* part = A.partial + (static_cast<size_t>(pair) * A.chunks + chunk) * NH * kGroupHeads * 132;
+  float* part = A.partial + static_cast<size_t>(sg.slot) * NH * kGroupHeads * 132;
   for (int i = threadIdx.x; i < NH * kGroupHeads * 128; i += blockDim.x) {
     const int hh = i >> 7, coord = i & 127;          // hh = group * 4 + head
     const int h = hh >> 2, h4 = hh & 3;
@@ -1865,7 +1885,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   if (threadIdx.x == 0) {
     unsigned ticket;
     asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(A.counters + pair) : "memory");
-    s_last = (ticket == static_cast<unsigned>(A.chunks - 1)) ? 1 : 0;
+    s_last = (ticket == static_cast<unsigned>(sg.n_segs - 1)) ? 1 : 0;
   }
   __syncthreads();
   if (!s_last) return;
@@ -1879,12 +1899,12 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   constexpr int kRec = 132;                                  // floats per (chunk, head slot) record
   constexpr int kSlots = NH * kGroupHeads;
   const unsigned chunk_bytes = kSlots * kRec * 4;
-  const float* pbase = A.partial + static_cast<size_t>(pair) * A.chunks * kSlots * kRec;
+  const float* pbase = A.partial + static_cast<size_t>(sg.first_slot) * kSlots * kRec;
   float* s_part = reinterpret_cast<float*>(smem);            // [merge_cap][kSlots][kRec]
   constexpr int kGroups = W / kGroupHeads;                   // warps per head slot
   float* s_mrg = s_part + static_cast<size_t>(A.merge_cap) * kSlots * kRec;   // [kGroups][kSlots][kRec]
   uint64_t* fbar = reinterpret_cast<uint64_t*>(s_mrg + kGroups * kSlots * kRec);
-  const float4 sv = __ldg(reinterpret_cast<const float4*>(T.signs_v) + lane);
+  const float4 sv = __ldg(reinterpret_cast<const float4*>(tab_sv) + lane);
   if (threadIdx.x == 0) {
     mbar_init(fbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1899,15 +1919,16 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   }
   bool landed = true;
   unsigned ph = 0;
-  for (int c0 = 0; c0 < A.chunks; c0 += A.merge_cap, ph ^= 1u) {
-    const int nc = min(A.merge_cap, A.chunks - c0);
+  for (int c0 = 0; c0 < sg.n_segs; c0 += A.merge_cap, ph ^= 1u) {
+    const int nc = min(A.merge_cap, sg.n_segs - c0);
     if (threadIdx.x == 0) {
       // generic-proxy writes of the other CTAs, read next by the bulk-copy unit
       asm volatile("fence.proxy.async.global;" ::: "memory");
       mbar_expect_tx(fbar, nc * chunk_bytes);
       tma_load_1d(s_part, pbase + static_cast<size_t>(c0) * kSlots * kRec, nc * chunk_bytes, fbar);
     }
-    if (!mbar_wait(fbar, ph)) {
+    // the whole CTA leaves together if any thread's wait ran out
+    if (__syncthreads_or(!mbar_wait(fbar, ph))) {
       if (threadIdx.x == 0) set_error(T.err, TQ_DEV_TIMEOUT);
       landed = false;
       break;
@@ -1933,6 +1954,8 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   }
   if (!landed) {
     mbar_wait(fbar, ph);                                      // bounded: let the copy land before exit
+    __syncthreads();
+    if (threadIdx.x == 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(fbar)) : "memory");
     return;
   }
 #pragma unroll
@@ -1968,6 +1991,173 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     const int qh = hk * A.group + slot;
     reinterpret_cast<float4*>(A.out + (static_cast<size_t>(b) * A.n_q + qh) * 128)[lane] = o;
   }
+  // the barrier's memory is reused by the next segment's stages
+  if (threadIdx.x == 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(fbar)) : "memory");
+}
+
+// The decode launch.
+// Uniform mode: CTA i serves chunk i / n_pairs of pair i % n_pairs (chunks of ppc pages).
+// Balanced mode (8-warp instantiations): the pairs' pages are laid end to end, each
+// non-empty pair preceded by seg_w "virtual" pages standing for its fixed cost
+// (prologue, merge), and the line is cut into G equal shares, one per CTA (share of
+// position y: ceil((y + 1) G / N) - 1). A CTA serves one segment per pair its share
+// overlaps, one after the other. (In the 16-warp instantiations, at the 128-register
+// cap, the loop around the segment body spills; they use the uniform mode only.)
+template <int BK, int BV, int NH, int MODE, bool BAL>
+__global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
+  // Launched as a programmatic dependent of the previous kernel in the stream: its
+  // memory operations are complete and visible once this wait returns, so nothing
+  // of the previous kernel's output is touched before it.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if constexpr (!BAL) {
+    Segment sg;
+    sg.pair = static_cast<int>(blockIdx.x % static_cast<unsigned>(A.n_pairs));
+    const int chunk = static_cast<int>(blockIdx.x / static_cast<unsigned>(A.n_pairs));
+    sg.p0 = chunk * A.ppc;
+    sg.len = A.ppc;
+    sg.slot = sg.pair * A.chunks + chunk;
+    sg.first_slot = sg.pair * A.chunks;
+    sg.n_segs = A.chunks;
+    sg.last = true;
+    decode_segment<BK, BV, NH, MODE>(T, A, sg);
+  } else {
+    extern __shared__ __align__(128) uint8_t smem[];
+    int* s_vs = reinterpret_cast<int*>(smem + A.vs_off);     // [batch + 1]: virtual pages before sequence b
+    int* s_ne = s_vs + A.batch + 1;                         // [batch + 1]: non-empty sequences before b
+    __shared__ Segment s_sg;
+    __shared__ long long s_n, s_g, s_x, s_hi;
+    __shared__ int s_wsum[32], s_carry, s_more;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    // block-wide exclusive prefix of v over [0, n) into dst[0..n], blockDim values at a time
+    auto block_scan = [&](int n, auto value, int* dst) {
+      if (threadIdx.x == 0) s_carry = 0;
+      __syncthreads();
+      for (int base = 0; base < n; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int v = i < n ? value(i) : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane == 31) s_wsum[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+          int w = lane < nw ? s_wsum[lane] : 0;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, w, o);
+            if (lane >= o) w += y;
+          }
+          if (lane < nw) s_wsum[lane] = w;              // inclusive over warps
+        }
+        __syncthreads();
+        const int incl = x + (warp > 0 ? s_wsum[warp - 1] : 0);
+        if (i < n) dst[i] = s_carry + incl - v;
+        __syncthreads();
+        if (threadIdx.x == 0) s_carry += s_wsum[nw - 1];
+        __syncthreads();
+      }
+      if (threadIdx.x == 0) dst[n] = s_carry;
+      __syncthreads();
+    };
+    // virtual length of sequence b: its pages plus seg_w, or 0 when empty
+    block_scan(A.batch, [&](int bb) {
+      const int L = min(max(A.seq_lens[bb], 0), A.max_seq_len);
+      const int pg = (L + kPage - 1) / kPage;
+      return pg > 0 ? pg + A.seg_w : 0;
+    }, s_vs);
+    block_scan(A.batch, [&](int bb) { return s_vs[bb + 1] > s_vs[bb] ? 1 : 0; }, s_ne);
+    if (threadIdx.x == 0) {
+      const long long n = static_cast<long long>(A.n_kv) * s_vs[A.batch];
+      s_n = n;
+      s_g = min(static_cast<long long>(A.shares), max(1LL, (n + A.min_share - 1) / A.min_share));
+    }
+    __syncthreads();
+    // pairs of empty sequences: zero outputs (nothing attends; logits are left alone)
+    if (MODE != 2) {
+      for (int p = blockIdx.x; p < A.n_pairs; p += gridDim.x) {
+        const int bb = p / A.n_kv, hk = p % A.n_kv;
+        if (s_vs[bb + 1] != s_vs[bb]) continue;
+        for (int i = threadIdx.x; i < A.group * 128; i += blockDim.x)
+          A.out[(static_cast<size_t>(bb) * A.n_q + hk * A.group) * 128 + i] = 0.0f;
+      }
+    }
+    const long long n = s_n, gg = s_g;
+    if (n == 0) return;
+    // the pair holding virtual position y: its ordinal among the pairs of non-empty
+    // sequences (consecutive along the line), first virtual page, virtual length
+    struct At { int p, vl; long long vp; };
+    auto pair_at = [&](long long y) {
+      int bl = 0, bh = A.batch;                       // n_kv s_vs[bl] <= y < n_kv s_vs[bh]
+      while (bh - bl > 1) {
+        const int mid = (bl + bh) >> 1;
+        if (static_cast<long long>(A.n_kv) * s_vs[mid] <= y) bl = mid; else bh = mid;
+      }
+      At r;
+      r.vl = s_vs[bl + 1] - s_vs[bl];                 // > 0: the largest such bl is a non-empty sequence
+      const long long vb = static_cast<long long>(A.n_kv) * s_vs[bl];
+      const int hk = static_cast<int>((y - vb) / r.vl);
+      r.p = s_ne[bl] * A.n_kv + hk;
+      r.vp = vb + static_cast<long long>(hk) * r.vl;
+      return r;
+    };
+    auto share_lo = [&](long long i) { return i * n / gg; };
+    if (static_cast<long long>(blockIdx.x) >= gg) return;
+    // This CTA serves share blockIdx.x: every pair it overlaps, one segment each,
+    // in order. The segment of share i in the pair of ordinal o writes record
+    // i + o, unique because consecutive pairs share at most one share; a pair's
+    // records run from (its first share) + o over its shares.
+    if (threadIdx.x == 0) {
+      s_x = share_lo(blockIdx.x);
+      s_hi = share_lo(blockIdx.x + 1);
+    }
+    auto next_segment = [&]() {                     // thread 0
+      auto cta_of = [&](long long y) { return static_cast<int>(((y + 1) * gg + n - 1) / n) - 1; };
+      s_more = 0;
+      long long x = s_x;
+      const long long hi = s_hi;
+      while (x < hi) {
+        const At a = pair_at(x);
+        const long long r0 = a.vp + A.seg_w, s0 = max(x, r0), s1 = min(hi, a.vp + a.vl);
+        x = a.vp + a.vl;
+        if (s1 > s0) {
+          const int t = a.p / A.n_kv, hk = a.p % A.n_kv;
+          int bl = 0, bh = A.batch;                   // the t-th non-empty sequence: largest bl, s_ne[bl] <= t
+          while (bh - bl > 1) {
+            const int mid = (bl + bh) >> 1;
+            if (s_ne[mid] <= t) bl = mid; else bh = mid;
+          }
+          Segment sg;
+          sg.pair = bl * A.n_kv + hk;
+          sg.p0 = static_cast<int>(s0 - r0);
+          sg.len = static_cast<int>(s1 - s0);
+          const int f = cta_of(r0), l = cta_of(r0 + (a.vl - A.seg_w) - 1);
+          sg.slot = static_cast<int>(blockIdx.x) + a.p;
+          sg.first_slot = f + a.p;
+          sg.n_segs = l - f + 1;
+          sg.last = x >= hi;
+          if (sg.len > A.ppc) {                       // the block-table window is sized by the host
+            set_error(T.err, TQ_DEV_BAD_LENGTH);
+            sg.len = A.ppc;
+          }
+          s_sg = sg;
+          s_more = 1;
+          break;
+        }
+      }
+      s_x = x;
+    };
+    if (threadIdx.x == 0) next_segment();
+    __syncthreads();
+    while (s_more) {
+      decode_segment<BK, BV, NH, MODE>(T, A, s_sg);
+      __syncthreads();
+      if (threadIdx.x == 0) next_segment();
+      __syncthreads();
+    }
+  }
 }
 
 template <int BK, int BV, int NH, int MODE>
@@ -1980,19 +2170,23 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
                       ((static_cast<size_t>(a.ppc) * 4 + 15) & ~static_cast<size_t>(15));
   // CTA merge: every warp's accumulators and softmax state
   const size_t merge = static_cast<size_t>(W) * NH * 8 * kAccPitch * 4 + W * NH * kGroupHeads * 3 * 4;
-  const size_t smem = pipe > merge ? pipe : merge;
+  const size_t base = ((pipe > merge ? pipe : merge) + 15) & ~static_cast<size_t>(15);
+  // balanced mode: two [batch + 1] prefixes of the split, after everything else
+  const size_t smem = base + (a.balanced ? (2 * static_cast<size_t>(a.batch) + 2) * 4 : 0);
   // final merge: merge_cap chunk records, then [W / 4][slots][132] floats and one barrier
   const size_t chunk_bytes = static_cast<size_t>(NH) * kGroupHeads * 132 * 4;
   const size_t groups = W / kGroupHeads;
-  if (smem > 227 * 1024 || smem < (groups + 1) * chunk_bytes + 16) return cudaErrorInvalidConfiguration;
+  if (smem > 227 * 1024 || base < (groups + 1) * chunk_bytes + 16) return cudaErrorInvalidConfiguration;
   DecodeArgs args = a;
-  args.merge_cap = static_cast<int>((smem - groups * chunk_bytes - 16) / chunk_bytes);
-  auto fn = decode_kernel<BK, BV, NH, MODE>;
-  static size_t configured = 0;     // raise the shared-memory limit once per instantiation
-  if (configured < smem) {
+  args.merge_cap = static_cast<int>((base - groups * chunk_bytes - 16) / chunk_bytes);
+  args.vs_off = static_cast<int>(base);
+  if (a.balanced && NH < 2) return cudaErrorInvalidConfiguration;   // no balanced 16-warp instantiation
+  auto fn = a.balanced ? decode_kernel<BK, BV, NH, MODE, (NH >= 2)> : decode_kernel<BK, BV, NH, MODE, false>;
+  static size_t configured[2] = {0, 0};   // raise the shared-memory limit once per instantiation
+  if (configured[a.balanced ? 1 : 0] < smem) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    configured = smem;
+    configured[a.balanced ? 1 : 0] = smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -2068,6 +2262,11 @@ DecodeArgs decode_args(const DecodePlan& plan, const void* q, int q_dtype, float
   a.chunks = plan.chunks;
   a.ppc = plan.pages_per_chunk;
   a.n_pairs = plan.n_pairs;
+  a.batch = plan.batch;
+  a.balanced = plan.balanced;
+  a.seg_w = plan.seg_w;
+  a.min_share = plan.min_share;
+  a.shares = plan.shares;
   a.sparse = sparse_tau > 0.0f ? 1 : 0;
   a.sparse_log2 = sparse_tau > 0.0f ? log2f(sparse_tau) : 0.0f;
   return a;
@@ -2147,7 +2346,7 @@ cudaError_t launch_decode(const Tables& t, const DecodePlan& plan, const void* q
                           float* out, void* workspace, float sparse_tau, cudaStream_t s) {
   const DecodeArgs a = decode_args(plan, q, q_dtype, scale, cache, n_pages, block_tables, max_pages_per_seq,
                                    seq_lens, max_seq_len, out, workspace, sparse_tau);
-  return dispatch_bk<0>(t, a, dim3(plan.chunks * plan.n_pairs), s);
+  return dispatch_bk<0>(t, a, dim3(plan.grid), s);
 }
 
 cudaError_t launch_logits(const Tables& t, const DecodePlan& plan, const void* q, int q_dtype, const void* cache,
@@ -2158,7 +2357,7 @@ cudaError_t launch_logits(const Tables& t, const DecodePlan& plan, const void* q
                              max_seq_len, nullptr, nullptr, 0.0f);
   a.logits = logits;
   a.logits_stride = logits_stride;
-  return dispatch_bk<2>(t, a, dim3(plan.chunks * plan.n_pairs), s);
+  return dispatch_bk<2>(t, a, dim3(plan.grid), s);
 }
 
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
@@ -2171,7 +2370,7 @@ cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const vo
   a.k_new = k_new;
   a.v_new = v_new;
   a.kv_dtype = kv_dtype;
-  return dispatch_bk<1>(t, a, dim3(plan.chunks * plan.n_pairs), s);
+  return dispatch_bk<1>(t, a, dim3(plan.grid), s);
 }
 
 }  // namespace tq

@@ -1,8 +1,9 @@
 """Decode with many (sequence, KV head) pairs, ragged and empty sequences, against the oracle.
 
-More pairs than SMs (the grid runs in several waves of one chunk per pair), and
-32 pairs (4 chunks each, 20 of 148 SMs idle), through tq_decode_attention,
-tq_decode_step and tq_decode_logits.
+More pairs than SMs, and 32 pairs (one uniform chunk count would leave 20 of 148 SMs
+idle), through tq_decode_attention, tq_decode_step and tq_decode_logits. With four
+query heads per KV head these run the uniform split (several waves of chunks); with
+8 or 12 they run the balanced split (equal shares of all pages, one CTA per share).
 """
 import numpy as np
 import pytest
@@ -47,7 +48,8 @@ def _lens(rng, n, hi, zeros):
     return [int(x) for x in lens]
 
 
-@pytest.mark.parametrize("n_seq,n_kv,g,hi,zeros", [(20, 8, 4, 300, 3), (8, 4, 4, 2500, 1), (40, 4, 12, 120, 5)])
+@pytest.mark.parametrize("n_seq,n_kv,g,hi,zeros", [(20, 8, 4, 300, 3), (8, 4, 4, 2500, 1), (40, 4, 12, 120, 5),
+                                                   (8, 4, 8, 2500, 1), (20, 8, 8, 300, 3)])
 def test_balanced_decode_matches_oracle(n_seq, n_kv, g, hi, zeros):
     seq_lens = _lens(np.random.default_rng(n_seq + hi), n_seq, hi, zeros)
     tab, _, _, cache_np, bt, n_pages, q, ctx = _case(seq_lens, n_kv, g, seed=n_seq)
@@ -68,9 +70,10 @@ def test_balanced_decode_matches_oracle(n_seq, n_kv, g, hi, zeros):
         print("worst rel err", assert_outputs_close(got[live], want[live]))
 
 
-def test_balanced_decode_step_and_logits():
-    rng = np.random.default_rng(7)
-    n_seq, n_kv, g = 20, 8, 4
+@pytest.mark.parametrize("g", [4, 8])
+def test_balanced_decode_step_and_logits(g):
+    rng = np.random.default_rng(7 + g)
+    n_seq, n_kv = 20, 8
     seq_lens = _lens(rng, n_seq, 260, 2)
     steps = 2
     tab, ks, vs, cache_np, bt, n_pages, q, ctx = _case(seq_lens, n_kv, g, seed=11, extra_steps=steps)
