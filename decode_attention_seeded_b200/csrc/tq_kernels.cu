@@ -1148,7 +1148,8 @@ struct Segment {
   bool last;                     // the CTA's last segment
 };
 
-template <int BK, int BV, int NH, int MODE>
+// LOOP: the CTA serves several segments one after the other (balanced split).
+template <int BK, int BV, int NH, int MODE, bool LOOP>
 __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs& A, const Segment& sg) {
   constexpr bool APPEND = MODE == 1;        // append the new token first (decode step)
   constexpr bool LOGITS = MODE == 2;        // write the logits; no softmax, no value sum
@@ -1165,13 +1166,13 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   const int g = lane >> 2, t = lane & 3;
   const int pair = sg.pair;
   const int b = pair / A.n_kv, hk = pair % A.n_kv;
-  // Table pointers made opaque for this segment: when one CTA serves several
-  // segments, the loads through them must not be hoisted out of the segment loop
-  // (that would keep their registers live across every main loop).
+  // When one CTA serves several segments, the table pointers are made opaque per
+  // segment, so that the loads through them are not hoisted out of the segment
+  // loop (that would keep their registers live across every main loop).
   const uint16_t* tab_m = T.sketch_m;
   const float* tab_sk = T.signs_k;
   const float* tab_sv = T.signs_v;
-  asm volatile("" : "+l"(tab_m), "+l"(tab_sk), "+l"(tab_sv));
+  if constexpr (LOOP) asm volatile("" : "+l"(tab_m), "+l"(tab_sk), "+l"(tab_sv));
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + W * S * kBlock);
   static_assert((W * S * kBlock + W * S * 8) % 16 == 0, "prologue alignment");
@@ -1927,8 +1928,12 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       mbar_expect_tx(fbar, nc * chunk_bytes);
       tma_load_1d(s_part, pbase + static_cast<size_t>(c0) * kSlots * kRec, nc * chunk_bytes, fbar);
     }
-    // the whole CTA leaves together if any thread's wait ran out
-    if (__syncthreads_or(!mbar_wait(fbar, ph))) {
+    // a thread whose wait ran out leaves; when the CTA serves more segments, the
+    // whole CTA leaves together, so that all of it meets the same barriers
+    bool ran_out;
+    if constexpr (LOOP) ran_out = __syncthreads_or(!mbar_wait(fbar, ph));
+    else ran_out = !mbar_wait(fbar, ph);
+    if (ran_out) {
       if (threadIdx.x == 0) set_error(T.err, TQ_DEV_TIMEOUT);
       landed = false;
       break;
@@ -1954,8 +1959,10 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   }
   if (!landed) {
     mbar_wait(fbar, ph);                                      // bounded: let the copy land before exit
-    __syncthreads();
-    if (threadIdx.x == 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(fbar)) : "memory");
+    if constexpr (LOOP) {                                     // CTA-uniform here: the barrier is reused
+      __syncthreads();
+      if (threadIdx.x == 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(fbar)) : "memory");
+    }
     return;
   }
 #pragma unroll
@@ -2019,7 +2026,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     sg.first_slot = sg.pair * A.chunks;
     sg.n_segs = A.chunks;
     sg.last = true;
-    decode_segment<BK, BV, NH, MODE>(T, A, sg);
+    decode_segment<BK, BV, NH, MODE, false>(T, A, sg);
   } else {
     extern __shared__ __align__(128) uint8_t smem[];
     int* s_vs = reinterpret_cast<int*>(smem + A.vs_off);     // [batch + 1]: virtual pages before sequence b
@@ -2152,7 +2159,7 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
     if (threadIdx.x == 0) next_segment();
     __syncthreads();
     while (s_more) {
-      decode_segment<BK, BV, NH, MODE>(T, A, s_sg);
+      decode_segment<BK, BV, NH, MODE, true>(T, A, s_sg);
       __syncthreads();
       if (threadIdx.x == 0) next_segment();
       __syncthreads();
