@@ -309,8 +309,7 @@ DecodePlan make_plan(int batch, int n_q, int n_kv, int max_seq_len, int sm_count
   const bool sm_limited = p.chunks == sm_chunks && pairs <= sm_count;
   const bool idle = sm_limited && (sm_count - p.chunks * pairs) * 20 > sm_count;
   p.balanced = 0;
-  // (8-warp instantiations only: groups of more than 4 query heads per KV head)
-  if ((idle || pairs > sm_count) && p.n_hg >= 2 && batch <= kMaxBalancedBatch) {
+  if ((idle || pairs > sm_count) && batch <= kMaxBalancedBatch) {
     const int seg_w = std::max(8, 36 / p.n_hg);
     const int64_t all = static_cast<int64_t>(pairs) * (p.max_pages + seg_w);
     const int64_t share = std::max<int64_t>(kMinShare, (all + sm_count - 1) / sm_count) + 2;

@@ -912,10 +912,12 @@ __device__ __forceinline__ int warp_isum(int v) {
 }
 
 // ================================================================== decode
-// Warps per decode CTA: 16 when a CTA serves one group of 4 query heads (the
-// kernel then fits 128 registers), else 8; either way one CTA per SM.
-template <int NH>
-struct DecodeWarps { static constexpr int value = NH == 1 ? 16 : 8; };
+// Warps per decode CTA: 16 when a CTA serves one group of 4 query heads in the
+// uniform split (the kernel then fits 128 registers), else 8; either way one CTA
+// per SM. The balanced split always takes 8 warps: its loop over segments needs
+// the registers that 16 warps do not leave.
+template <int NH, bool BAL = false>
+struct DecodeWarps { static constexpr int value = (NH == 1 && !BAL) ? 16 : 8; };
 // TMA stages per warp: six when they fit in 160 KB of shared memory, else four.
 constexpr int kAccPitch = 132;      // floats per accumulator column in the CTA merge
 
@@ -1155,7 +1157,7 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   constexpr bool LOGITS = MODE == 2;        // write the logits; no softmax, no value sum
   constexpr bool KQ8 = BK == 8;              // q8_0 keys (raw query, block scales, no QJL)
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int W = DecodeWarps<NH>::value;
+  constexpr int W = DecodeWarps<NH, LOOP>::value;
   constexpr int kBlock = block_bytes_of(BK, BV);
   constexpr int S = decode_stages(W, kBlock);
   constexpr int kSignOff = sec_scale(BK), kVOff = sec_v(BK), kNormOff = sec_norm(BK, BV);
@@ -2004,14 +2006,13 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
 
 // The decode launch.
 // Uniform mode: CTA i serves chunk i / n_pairs of pair i % n_pairs (chunks of ppc pages).
-// Balanced mode (8-warp instantiations): the pairs' pages are laid end to end, each
+// Balanced mode (always 8 warps): the pairs' pages are laid end to end, each
 // non-empty pair preceded by seg_w "virtual" pages standing for its fixed cost
 // (prologue, merge), and the line is cut into G equal shares, one per CTA (share of
 // position y: ceil((y + 1) G / N) - 1). A CTA serves one segment per pair its share
-// overlaps, one after the other. (In the 16-warp instantiations, at the 128-register
-// cap, the loop around the segment body spills; they use the uniform mode only.)
+// overlaps, one after the other.
 template <int BK, int BV, int NH, int MODE, bool BAL>
-__global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
+__global__ void __launch_bounds__(DecodeWarps<NH, BAL>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
   // Launched as a programmatic dependent of the previous kernel in the stream: its
   // memory operations are complete and visible once this wait returns, so nothing
   // of the previous kernel's output is touched before it.
@@ -2167,9 +2168,9 @@ __global__ void __launch_bounds__(DecodeWarps<NH>::value * 32, 1) decode_kernel(
   }
 }
 
-template <int BK, int BV, int NH, int MODE>
-cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
-  constexpr int W = DecodeWarps<NH>::value;
+template <int BK, int BV, int NH, int MODE, bool BAL>
+cudaError_t launch_decode_tb(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
+  constexpr int W = DecodeWarps<NH, BAL>::value;
   constexpr int kBlock = block_bytes_of(BK, BV);
   constexpr int S = decode_stages(W, kBlock);
   // main loop: stages, barriers, prologue scratch, the chunk's block-table window
@@ -2179,7 +2180,7 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
   const size_t merge = static_cast<size_t>(W) * NH * 8 * kAccPitch * 4 + W * NH * kGroupHeads * 3 * 4;
   const size_t base = ((pipe > merge ? pipe : merge) + 15) & ~static_cast<size_t>(15);
   // balanced mode: two [batch + 1] prefixes of the split, after everything else
-  const size_t smem = base + (a.balanced ? (2 * static_cast<size_t>(a.batch) + 2) * 4 : 0);
+  const size_t smem = base + (BAL ? (2 * static_cast<size_t>(a.batch) + 2) * 4 : 0);
   // final merge: merge_cap chunk records, then [W / 4][slots][132] floats and one barrier
   const size_t chunk_bytes = static_cast<size_t>(NH) * kGroupHeads * 132 * 4;
   const size_t groups = W / kGroupHeads;
@@ -2187,13 +2188,12 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
   DecodeArgs args = a;
   args.merge_cap = static_cast<int>((base - groups * chunk_bytes - 16) / chunk_bytes);
   args.vs_off = static_cast<int>(base);
-  if (a.balanced && NH < 2) return cudaErrorInvalidConfiguration;   // no balanced 16-warp instantiation
-  auto fn = a.balanced ? decode_kernel<BK, BV, NH, MODE, (NH >= 2)> : decode_kernel<BK, BV, NH, MODE, false>;
-  static size_t configured[2] = {0, 0};   // raise the shared-memory limit once per instantiation
-  if (configured[a.balanced ? 1 : 0] < smem) {
+  auto fn = decode_kernel<BK, BV, NH, MODE, BAL>;
+  static size_t configured = 0;     // raise the shared-memory limit once per instantiation
+  if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    configured[a.balanced ? 1 : 0] = smem;
+    configured = smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -2207,6 +2207,12 @@ cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cud
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, fn, T, args);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int BK, int BV, int NH, int MODE>
+cudaError_t launch_decode_t(const Tables& T, const DecodeArgs& a, dim3 grid, cudaStream_t s) {
+  return a.balanced ? launch_decode_tb<BK, BV, NH, MODE, true>(T, a, grid, s)
+                    : launch_decode_tb<BK, BV, NH, MODE, false>(T, a, grid, s);
 }
 
 template <int BK, int BV, int MODE>
