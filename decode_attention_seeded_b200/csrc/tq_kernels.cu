@@ -1120,10 +1120,10 @@ __device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float
   o.gamma = n * sqrtf(warp_sum(uu));
 }
 
-// Split-K decode attention, one launch per call. 1-D grid: CTA i serves chunk
-// i / n_pairs of (sequence, KV head) pair i % n_pairs, so that CTAs launched
-// together cover every pair. W warps per CTA, one CTA per SM. A chunk is
-// ppc consecutive pages; each warp streams pages through a private ring of S
+// Split-K decode attention, one launch per call; this is the body for one
+// segment: a run of consecutive pages of one (sequence, KV head) pair (the
+// kernel below says which segments a CTA serves). W warps per CTA, one CTA per
+// SM. Each warp streams the segment's pages through a private ring of S
 // shared-memory stages filled by 1-D bulk TMA copies. The first kStatic pages
 // of every warp are fixed (page p0 + warp + W k) and their copies go out before
 // any barrier; all later pages are claimed one at a time from a shared counter,
@@ -1138,9 +1138,10 @@ __device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float
 //   values  fp16 m16n8k16: A = value centroids (coordinates x tokens),
 //           B = softmax weights split into fp16 high parts (columns 0-3) and
 //           low parts (columns 4-7), transposed into place with shuffles.
-// APPEND: the CTA whose chunk holds a sequence's last page first quantizes
+// APPEND: the CTA whose segment holds a sequence's last page first quantizes
 // (k_new, v_new) of that sequence into position seq_len - 1; a warp that is
 // given that page before then holds its copy back until the token is written.
+//
 // One piece of work of a CTA: logical pages [p0, p0 + len) of one (sequence, KV
 // head) pair (clipped to the sequence), whose merged record goes to slot `slot`;
 // the pair's records are slots first_slot .. first_slot + n_segs - 1.
