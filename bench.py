@@ -289,7 +289,7 @@ class DecodeBench:
                 "tokens": self.T0, "kv_heads": n_kv, "bytes_in": bytes_in, "bytes_out": bytes_out,
                 "kernel": "quantize_prefill_kernel via tq_quantize_prefill (bf16 K/V, one layer)"}
 
-    def logits_timing(self, reps=3):
+    def logits_timing(self, reps=10):
         """Logits only (tq_decode_logits) against logits from full-precision fp32 keys.
 
         The pages compare attention-logit speed on compressed keys with 32-bit keys.
