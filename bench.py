@@ -25,6 +25,7 @@ slowest rank's time.
 """
 
 import argparse
+import re
 import hashlib
 import json
 import os
@@ -50,9 +51,14 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the library's code with comments and whitespace removed, so that a
+    recorded ncu measurement stays tied to the code it was taken on, not its comments."""
     h = hashlib.sha256()
     for f in ("tq_kernels.cu", "tq_host.cpp", "tq_internal.h"):
-        h.update(open(os.path.join(ROOT, "decode_attention_seeded_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "decode_attention_seeded_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update("".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -9,12 +9,14 @@
 // Decode estimates q.k = |k| <R q, c> + gamma sqrt(pi/2)/m <S R q, sign(S u)>.
 //
 // Block layout of one (page, KV head), 16 tokens (the same definition is
-// written out in the header comment of the Python layout description):
+// written out independently by the oracle's layout module):
 //   [K codes 32 lanes x 8*bk B][sign bits 32 x 8 B][V codes 32 x 8*bv B][norms 96 B]
+// or, with q8_0 keys (bk = 8):
+//   [int8 K values 32 lanes x 64 B][fp16 block scales 128 B][V codes 32 x 8*bv B][V norms 32 B]
 // Lane chunks are laid out so that lane (g, t) = (lane>>2, lane&3) of a warp
 // finds in its own chunk exactly the bits of its mma.sync fragments:
-//   keys:   B operand of m16n8k32 (k = coordinate, n = token), token halves th
-//   signs:  B operand of m16n8k32 (k = sketch row,  n = token)
+//   keys:   A operand of m16n8k32 (m = token: g and g + 8, k = coordinate)
+//   signs:  A operand of m16n8k32 (m = token, k = sketch row)
 //   values: A operand of m16n8k16 (m = coordinate, k = token)
 
 #include "tq.h"
