@@ -19,6 +19,15 @@
  *     legacy default stream). Nothing throws across the ABI.
  *   - Arguments the host can check are checked before any launch; a bad one
  *     returns TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED and enqueues nothing.
+ *   - Decode calls (tq_decode_attention, tq_decode_step, tq_decode_logits,
+ *     tq_decode_attention_noalloc) launch as programmatic dependents of the
+ *     previous work in the stream: their kernel waits for it to complete before
+ *     touching memory, so stream order holds as usual. They also allow the next
+ *     kernel to launch early, once their page stream is done. A caller kernel
+ *     launched with programmatic stream serialization must therefore wait for its
+ *     grid dependency (cudaGridDependencySynchronize) before it reads their
+ *     outputs, as programmatic dependent launch requires anyway. Kernels launched
+ *     without that attribute see ordinary stream order.
  *   - Faults detected on the device (a page id or slot out of range, a wait
  *     that ran out) are not traps: the kernel skips the access, records a code
  *     in the context's device error word and finishes. tq_get_device_error
