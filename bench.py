@@ -14,9 +14,15 @@ caches (about 0.86 GB) exceed the 126 MB L2, so every step streams from HBM.
 ``e2e``     the same steps through the C ABI with host buffers: per step the
             new K/V and queries are copied from pinned host memory and the
             attention outputs copied back, inside the timed region.
-``roofline`` decode attention (tq_decode_attention: one kernel doing the query
-            transform, split-K decode and the split merge) against the measured HBM copy bandwidth: algorithmic bytes =
-            compressed bytes of every cached token-head read (102 B each).
+``roofline`` the kernel the timed step launches (decode_kernel via
+            tq_decode_step: append, query transform, split-K decode and merge,
+            once per layer) against the measured HBM copy bandwidth: algorithmic
+            bytes = compressed bytes of every cached token-head read (102 B each)
+            over its mean launch time in the timed replays. ``roofline_attention``
+            is the same for tq_decode_attention (no append) at the final context.
+``parity``  a sampled oracle check of the bench's own cache after the timed
+            steps (appended tokens' codes, signs and norms; decode outputs of a few
+            (sequence, KV head) pairs over the full context).
 ``cpu_baseline`` the float64 oracle on the host, on a bounded sample.
 
 Multi-GPU: one process per GPU (torchrun); each rank serves its own sequence
@@ -54,8 +60,11 @@ def kernel_source_hash():
     """Hash of the library's code with comments and whitespace removed, so that a
     recorded ncu measurement stays tied to the code it was taken on, not its comments."""
     h = hashlib.sha256()
-    for f in ("tq_kernels.cu", "tq_host.cpp", "tq_internal.h"):
-        src = open(os.path.join(ROOT, "decode_attention_seeded_b200", "csrc", f)).read()
+    csrc = os.path.join(ROOT, "decode_attention_seeded_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if not f.endswith((".cu", ".cuh", ".cpp", ".h")):
+            continue
+        src = open(os.path.join(csrc, f)).read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
         src = re.sub(r"//[^\n]*", " ", src)
         h.update("".join(src.split()).encode())
@@ -158,7 +167,8 @@ class DecodeBench:
         bpt = self.ctx.block_bytes // 16
         per_layer = int(np.sum(self.lens0)) * n_kv * bpt
         # rotate through enough layer caches that they exceed the L2 several times over
-        self.n_layers = max(wl.n_layers, min(64, int(np.ceil(4 * self.L2_BYTES / per_layer))))
+        self.n_layers = bench_layers(wl, self.ctx.block_bytes, self.L2_BYTES)
+        assert per_layer > 0
         self.page_bytes = self.ctx.page_bytes(n_kv)
         self.caches, self.btabs = [], []
         g = torch.Generator(device=device)
@@ -460,6 +470,41 @@ def timed(torch, dev, fn):
     return a.elapsed_time(b) / 1e3
 
 
+def bench_layers(wl, block_bytes, l2_bytes=126e6):
+    """Layer caches the bench rotates through: the workload's layers, or more, so that
+    they exceed the L2 four times over (at most 64)."""
+    per_layer = int(np.sum(seq_lens_of(wl))) * wl.n_kv_heads * (block_bytes // 16)
+    return max(wl.n_layers, min(64, int(np.ceil(4 * l2_bytes / per_layer))))
+
+
+def seq_lens_of(wl):
+    from decode_attention_seeded_b200 import synth
+    return synth.Generator(wl, layer=0).seq_lens().astype(np.int64)
+
+
+def block_bytes_of(wl):
+    """Bytes of one (page, KV head) block (include/tq.h): 16 tokens x per-token bytes."""
+    if wl.key_bits == 8:
+        return 16 * (128 + 8 + 16 * wl.value_bits + 2)
+    return 16 * (16 * wl.key_bits + 16 + 4 + 16 * wl.value_bits + 2)
+
+
+def workload_config(wl, world, steps, warmup, sparse_v=0.0, peaked=False):
+    """The `config` object of the JSON line; both arms print the same one."""
+    bb = block_bytes_of(wl)
+    lens0 = seq_lens_of(wl)
+    layers = bench_layers(wl, bb)
+    pages = (lens0 + steps + warmup + 15) // 16
+    step_bytes = layers * int(np.sum(pages) + 3) * wl.n_kv_heads * bb
+    return {"workload": wl.name, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
+            "head_dim": 128, "context": wl.context, "context_lens": [int(x) for x in lens0[:16]],
+            "layers": layers, "key_bits": wl.key_bits, "value_bits": wl.value_bits,
+            "qjl_rows": 0 if wl.key_bits == 8 else 128, "page_tokens": 16,
+            "l2": f"inputs larger than L2: {layers} layer caches, about {step_bytes / 1e9:.2f} GB per step",
+            "parallelism": f"replica x{world} (each GPU serves its own batch)",
+            "sparse_v": sparse_v, "queries": "peaked (5 x 3 cached key directions)" if peaked else "N(0,1)"}
+
+
 # -------------------------------------------------------------- CPU baseline
 def oracle_sample(wl, budget_s=12.0, gpu_cache=None):
     """Time the float64 oracle on a bounded sample of one decode step.
@@ -531,6 +576,181 @@ def oracle_sample(wl, budget_s=12.0, gpu_cache=None):
                       f"{wl.n_kv_heads * wl.n_layers} to a full step", "seconds": round(el, 2)}
 
 
+# ------------------------------------------------------------------- parity
+def bench_parity(bench, layer, pairs=4, near=1e-5, rtol=1e-3):
+    """Sampled oracle check of the bench's own cache (one layer, after the timed steps).
+
+    Quantize: every token the timed decode steps appended to this layer (all KV
+    heads), unpacked from the GPU cache and compared with the oracle's
+    quantization of the same bf16 rows: codes and sign bits bit-exact except
+    within `near` of a decision boundary (counted as excused), fp16 norms within
+    one unit in the last place. Decode: `pairs` (sequence, KV head) pairs decoded
+    by the oracle over the full context from the bytes the GPU wrote, against
+    the outputs of the last decode call on this layer."""
+    from oracle import codebook as ocb, decode as odec, layout as lay, quantize as oq, rng as orng
+    torch, wl = bench.torch, bench.wl
+    if wl.key_bits == 8:
+        return {"skipped": "q8_0 keys: checked by the q8 tests"}
+    bk, bv, n_kv = wl.key_bits, wl.value_bits, wl.n_kv_heads
+    kb, vb = ocb.codebook(bk), ocb.codebook(bv)
+    seeds = bench.seeds
+    tab = dict(signs_k=orng.sign_vector(seeds[0], 128), signs_v=orng.sign_vector(seeds[1], 128),
+               sketch=orng.gaussian_sketch(seeds[2], 128, 128), centroids_k=kb.centroids,
+               centroids_v=vb.centroids, bk=bk, bv=bv)
+    cache, n_pages = bench.caches[layer]
+    host = cache.view(n_pages, n_kv, -1).cpu().numpy()
+    bt = bench.btabs[layer].cpu().numpy()
+    res = {"layer": layer}
+    # quantize: the appended tokens
+    xk = bench.newk[layer].float().cpu().numpy().astype(np.float64)     # [steps, B, n_kv, 128]
+    xv = bench.newv[layer].float().cpu().numpy().astype(np.float64)
+    fk, fv, fs, nk, gm, nv, rk, rv = [], [], [], [], [], [], [], []
+    for s in range(bench.total_steps):
+        for b in range(wl.batch):
+            pos = int(bench.lens0[b]) + s
+            for h in range(n_kv):
+                f = lay.read_page(host[bt[b, pos // 16], h], bk, bv)
+                tau = pos % 16
+                fk.append(f[0][tau]); fs.append(f[1][tau]); fv.append(f[2][tau])
+                nk.append(f[3][tau]); gm.append(f[4][tau]); nv.append(f[5][tau])
+                rk.append(xk[s, b, h]); rv.append(xv[s, b, h])
+    qk = oq.quantize(np.array(rk), tab["signs_k"], kb.centroids, kb.thresholds, tab["sketch"])
+    qv = oq.quantize(np.array(rv), tab["signs_v"], vb.centroids, vb.thresholds)
+    near_k = np.min(np.abs(qk.y[..., None] - kb.thresholds), axis=-1) < near
+    near_v = np.min(np.abs(qv.y[..., None] - vb.thresholds), axis=-1) < near
+    dk, dv = np.array(fk) != qk.codes, np.array(fv) != qv.codes
+    same = ~np.any(dk, axis=1)
+    near_s = np.abs(qk.projection) < near * np.linalg.norm(qk.residual, axis=1)[:, None]
+    ds = (np.array(fs) != qk.sign_bits) & same[:, None]
+
+    def ulps(a, b):
+        ia = np.asarray(a, dtype=np.float16).view(np.int16).astype(np.int64)
+        ib = np.asarray(b, dtype=np.float16).view(np.int16).astype(np.int64)
+        ia = np.where(ia < 0, -(ia & 0x7FFF), ia)
+        ib = np.where(ib < 0, -(ib & 0x7FFF), ib)
+        return np.abs(ia - ib)
+
+    res.update({"quantize_rows": len(rk), "bad_k_codes": int(np.sum(dk & ~near_k)),
+                "excused_k_codes": int(np.sum(dk & near_k)), "bad_v_codes": int(np.sum(dv & ~near_v)),
+                "excused_v_codes": int(np.sum(dv & near_v)), "bad_signs": int(np.sum(ds & ~near_s)),
+                "excused_signs": int(np.sum(ds & near_s)),
+                "bad_norms": int(np.sum(ulps(nk, qk.norm16) > 1) + np.sum(ulps(nv, qv.norm16) > 1)
+                                 + np.sum(ulps(np.array(gm)[same], qk.gamma16[same]) > 1))})
+    # decode: sampled (sequence, KV head) pairs of the last call on this layer
+    last = bench.total_steps - 1
+    L = bench.lens[last].cpu().numpy()
+    q = bench.q[last, layer].float().cpu().numpy().astype(np.float64)
+    out = bench.out[layer].cpu().numpy().astype(np.float64)
+    g = wl.n_q_heads // n_kv
+    rng = np.random.default_rng(0)
+    allp = [(b, h) for b in range(wl.batch) for h in range(n_kv)]
+    pick = [allp[int(i)] for i in rng.permutation(len(allp))[:pairs]]
+    worst, worst_e = 0.0, 0.0
+    for b, h in pick:
+        want = odec.decode_paged(host[:, h:h + 1], bt[b:b + 1], [int(L[b])], q[b:b + 1, h * g:(h + 1) * g], tab)[0]
+        got = out[b, h * g:(h + 1) * g]
+        ref = np.linalg.norm(want, axis=-1)
+        worst = max(worst, float(np.max(np.linalg.norm(got - want, axis=-1) / ref)))
+        floor = ref[:, None] / np.sqrt(128)
+        worst_e = max(worst_e, float(np.max(np.abs(got - want) / np.maximum(np.abs(want), floor))))
+    res.update({"decode_pairs": [list(x) for x in pick], "decode_tokens": [int(L[b]) for b, _ in pick],
+                "worst_rel_err": worst, "worst_elem_err": worst_e, "tolerance": rtol,
+                "ok": bool(worst <= rtol and worst_e <= rtol and all(
+                    res[k] == 0 for k in res if isinstance(k, str) and k.startswith("bad")))})
+    return res
+
+
+def reference_arm(wl, args, world):
+    """The float64 oracle on the host's cores, timed over K sample steps after W warm-up ones.
+
+    One sample step: quantize one new token (K and V) of one KV head, and decode
+    that KV head's query heads over a slice of the context of `sample_pages`
+    pages, from packed bytes. Its time scales to a full step (every page of every
+    sequence, KV head and layer, and every appended token): the line's value is
+    that extrapolation, and ms_per_step is the time of one sample step."""
+    import threadpoolctl
+    from oracle import codebook as ocb, decode as odec, layout as lay, quantize as oq, rng as orng, q8 as oq8
+    from decode_attention_seeded_b200 import synth
+    gen = synth.Generator(wl, layer=0)
+    seeds = gen.method_seeds()
+    q8k = wl.key_bits == 8
+    kb, vb = ocb.codebook(2 if q8k else wl.key_bits), ocb.codebook(wl.value_bits)
+    tab = dict(signs_k=orng.sign_vector(seeds[0], 128), signs_v=orng.sign_vector(seeds[1], 128),
+               sketch=orng.gaussian_sketch(seeds[2], 128, 128))
+    rng = np.random.default_rng(0)
+    lens0 = seq_lens_of(wl)
+    total_pages = int(np.sum((lens0 + 15) // 16))
+    budget = min(args.oracle_budget * 5, 120.0)                  # seconds for the whole run
+    # packed bytes of a synthetic slice (random bits: the oracle's cost does not depend on them)
+    npg = min(total_pages, 2048)
+    blocks = rng.integers(0, 256, size=(npg, lay.block_bytes(wl.key_bits, wl.value_bits)), dtype=np.uint8)
+    off = lay.section_offsets(wl.key_bits, wl.value_bits)
+    no = off["norm"]
+    blocks[:, no:] = np.frombuffer(np.abs(rng.standard_normal((npg, (blocks.shape[1] - no) // 2)))
+                                   .astype(np.float16).tobytes(), dtype=np.uint8).reshape(npg, -1)
+    if q8k:
+        so = off["sign"]
+        blocks[:, so:so + 128] = np.frombuffer(np.abs(rng.standard_normal((npg, 64))).astype(np.float16)
+                                               .tobytes(), dtype=np.uint8).reshape(npg, 128)
+    bt = np.arange(npg)
+
+    def sample_step(pages):
+        x = rng.standard_normal((1, 128))
+        if q8k:
+            oq8.quantize_q8(x)
+        else:
+            oq.quantize(x, tab["signs_k"], kb.centroids, kb.thresholds, tab["sketch"])
+        oq.quantize(x, tab["signs_v"], vb.centroids, vb.thresholds)
+        T = pages * 16
+        if q8k:
+            k8, sc, vc, nv = odec.gather_sequence_q8(blocks[:, None, :], bt, T, 0, wl.value_bits)
+        else:
+            kc, sb, vc, nk, gm, nv = odec.gather_sequence(blocks[:, None, :], bt, T, 0, wl.key_bits, wl.value_bits)
+        for _ in range(wl.group):
+            if q8k:
+                lg = oq8.logits_q8(rng.standard_normal(128), k8, sc, 1 / np.sqrt(128))
+            else:
+                qt, p = odec.transform_query(rng.standard_normal(128), tab["signs_k"], tab["sketch"])
+                lg = odec.logits(qt, p, kc, nk, gm, sb, kb.centroids, 1 / np.sqrt(128), 128)
+            odec.attend(lg, vc, nv, vb.centroids, tab["signs_v"])
+
+    with threadpoolctl.threadpool_limits(1):
+        t0 = time.perf_counter()
+        sample_step(1)
+        t_one = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        sample_step(min(npg, 64))
+        per_page = max((time.perf_counter() - t0 - t_one) / max(min(npg, 64) - 1, 1), 1e-7)
+        fixed = max(t_one - per_page, 0.0)
+        per_step = budget / (args.steps + args.warmup)
+        pages = int(min(npg, max(1, (per_step - fixed) / per_page)))
+        for _ in range(args.warmup):
+            sample_step(pages)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            sample_step(pages)
+        el = time.perf_counter() - t0
+    t_sample = el / args.steps
+    # a full step: every page of every (sequence, KV head) of every layer, plus the
+    # fixed per-(sequence, KV head) cost (quantize of the new token, query transform)
+    page_cost = max(t_sample - fixed, 0.0) / pages
+    layers = bench_layers(wl, block_bytes_of(wl))
+    full_step = layers * wl.n_kv_heads * (total_pages * page_cost + wl.batch * fixed)
+    value = wl.batch / full_step
+    cpu = {"kind": "oracle", "cores": 1, "value": value, "unit": "tokens/s",
+           "sample": f"{args.steps} sample steps after {args.warmup} warm-up ones, each: quantize one token-head "
+                     f"(K and V) and decode {wl.group} query heads of one KV head over {pages} pages "
+                     f"({pages * 16} tokens), float64 NumPy, 1 thread; scaled to a full step of "
+                     f"{layers} layers x {wl.n_kv_heads} KV heads x {total_pages} pages"}
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_sample * 1e3,
+            "ms_per_full_step_extrapolated": full_step * 1e3, "extrapolated": True,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, world, args.steps, args.warmup, args.sparse_v, args.peaked),
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 # --------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -541,6 +761,7 @@ def main():
     ap.add_argument("--workload", default="llama8b")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-parity", action="store_true", help="skip the sampled oracle check (profiling runs)")
     ap.add_argument("--oracle-budget", type=float, default=12.0)
     ap.add_argument("--sparse-v", type=float, default=0.0,
                     help="Sparse V threshold (relative attention weight; 0 = dense)")
@@ -563,17 +784,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        cpu = oracle_sample(wl, budget_s=min(args.oracle_budget, 20.0))
-        v = cpu["value"]
-        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.n_q_heads,
-                           "kv_heads": wl.n_kv_heads, "context": wl.context, "layers": wl.n_layers,
-                           "key_bits": wl.key_bits, "value_bits": wl.value_bits},
-                "cpu_baseline": {k: cpu[k] for k in ("kind", "cores", "sample")} | {"value": v, "unit": "tokens/s"},
-                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        print(json.dumps(reference_arm(wl, args, world)), flush=True)
         return
 
     import torch
@@ -613,7 +824,7 @@ def main():
     t_e2e = max_over_ranks(timed(torch, dev, g_e2e.replay), world, dev)
     barrier()
 
-    # roofline: decode attention alone, back-to-back over the 32 layer caches
+    # decode attention alone (no append), back-to-back over the layer caches
     reps = 4
     g_dec = bench.decode_only_graph(reps)
     g_dec.replay()
@@ -622,6 +833,7 @@ def main():
     n_dec = reps * bench.n_layers
     dec_s = t_dec / n_dec
     assert bench.ctx.device_error() == 0
+    parity = bench_parity(bench, bench.n_layers - 1) if rank == 0 and not args.no_parity else None
 
     base16 = bench.bf16_baseline()
     logits_cmp = bench.logits_timing()
@@ -630,7 +842,12 @@ def main():
     peak, peak_kind = load_peaks()
     bpt = bench.ctx.block_bytes // 16                     # bytes per token-head (102 for 3/2 bits)
     alg_bytes = bpt * bench.cache_tokens * wl.n_kv_heads
-    achieved = alg_bytes / dec_s / 1e9
+    # the timed step launches one decode kernel per layer and nothing else
+    step_launch_s = t_main / (K * bench.n_layers)
+    # cached tokens per call, averaged over the timed steps (the context grows by one each step)
+    step_tokens = int(np.sum(bench.lens0)) + wl.batch * (W + (K + 1) / 2)
+    step_bytes = bpt * step_tokens * wl.n_kv_heads
+    achieved = step_bytes / step_launch_s / 1e9
     traffic = recorded_traffic("bytes_per_launch")
 
     tokens = K * wl.batch * world
@@ -641,20 +858,19 @@ def main():
         "ms_per_step": t_main / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": f"int8/fp16 tensor-core, fp32 accumulate ({key_format(wl.key_bits)}, {wl.value_bits}-bit values)",
         "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
-                   "head_dim": 128, "context": wl.context, "context_lens": [int(x) for x in bench.lens0[:16]],
-                   "layers": bench.n_layers, "key_bits": wl.key_bits,
-                   "value_bits": wl.value_bits, "qjl_rows": 0 if wl.key_bits == 8 else 128, "page_tokens": 16,
-                   "l2": f"inputs larger than L2: {bench.n_layers} layer caches, "
-                         f"{bench.n_layers * bench.caches[0][1] * bench.page_bytes / 1e9:.2f} GB per step",
-                   "parallelism": f"replica x{world} (each GPU serves its own batch)",
-                   "sparse_v": args.sparse_v, "queries": "peaked (5 x 3 cached key directions)" if args.peaked
-                   else "N(0,1)"},
+        "config": workload_config(wl, world, K, W, args.sparse_v, args.peaked),
         "e2e": {"value": job_throughput(K * wl.batch, world, t_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                     "kernel": "decode_kernel via tq_decode_attention (query transform, split-K decode, merge)",
-                     "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
+                     "kernel": "decode_kernel via tq_decode_step (append, query transform, split-K decode, "
+                               "merge): the one kernel the timed step launches, once per layer",
+                     "us_per_launch": step_launch_s * 1e6, "alg_bytes_per_launch": step_bytes,
+                     "timing": "CUDA events around the timed graph replays / launches"},
+        "roofline_attention": {"bound": "hbm", "achieved": alg_bytes / dec_s / 1e9, "peak": peak, "unit": "GB/s",
+                               "frac": alg_bytes / dec_s / 1e9 / peak, "peak_kind": peak_kind,
+                               "kernel": "decode_kernel via tq_decode_attention (no append), final context",
+                               "us_per_launch": dec_s * 1e6, "alg_bytes_per_launch": alg_bytes},
+        "parity": parity,
         "quantize": quant,
         "logits": logits_cmp,
         "bf16_baseline": dict(base16, **({"compressed_us_per_layer": dec_s * 1e6,

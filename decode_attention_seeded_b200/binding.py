@@ -19,6 +19,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace", 4: "
           5: "device error", 6: "not initialised"}
 DTYPES = {"fp32": 0, "bf16": 1, "fp16": 2}
 DEV_BAD_SLOT, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_LENGTH = 0x1, 0x2, 0x4, 0x8
+TEST_WAIT_RUNS_OUT = 0x1
 
 _lib = None
 
@@ -49,6 +50,7 @@ _SIGS = {
                                                _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int,
                                                _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p]),
     "tq_set_sparse_v": (_c.c_int, [_c.c_void_p, _c.c_float]),
+    "tq_set_test_flags": (_c.c_int, [_c.c_void_p, _c.c_uint]),
     "tq_decode_logits": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_void_p, _c.c_int64, _c.c_void_p,
                                     _c.c_int, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_float,
                                     _c.c_void_p, _c.c_int64, _c.c_void_p]),
@@ -209,6 +211,10 @@ class Context:
     def set_sparse_v(self, tau: float):
         """Sparse V threshold of later decode calls (0: dense attention)."""
         _check("tq_set_sparse_v", lib().tq_set_sparse_v(self._h, tau))
+
+    def set_test_flags(self, flags: int):
+        """Test hook bits (TEST_WAIT_RUNS_OUT) of later decode calls; 0 turns them off."""
+        _check("tq_set_test_flags", lib().tq_set_test_flags(self._h, flags))
 
     def device_error(self, stream=None) -> int:
         code = ctypes.c_uint32(0)

@@ -659,9 +659,16 @@ tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dty
                                       int max_pages_per_seq, const int32_t* seq_lens, int batch,
                                       int n_q_heads, int n_kv_heads, int max_seq_len, float scale,
                                       float* out, tq_stream stream) {
-  if (!ctx) return TQ_ERR_INVALID_ARG;
-  if (tq_status st = check_device(ctx)) return st;
-  // The scratch address is looked up once per device and kept for the process.
+  // Arguments first (nothing touches the device before they pass), then the size
+  // limit, and only then the scratch address.
+  tq::DecodePlan plan;
+  if (tq_status st = check_decode_args(ctx, q, q_dtype, cache, n_cache_pages, block_tables, max_pages_per_seq,
+                                       seq_lens, batch, n_q_heads, n_kv_heads, max_seq_len, scale, out,
+                                       nullptr, 0, &plan, false))
+    return st;
+  if (plan.total > tq::kNoAllocScratchBytes) return TQ_ERR_WORKSPACE;   // use tq_decode_attention
+  // The scratch address is looked up once per device and kept for the process
+  // (it does not survive a cudaDeviceReset of that device).
   static std::mutex mu;
   static std::map<int, void*> scratch_of_device;
   void* scratch = nullptr;
@@ -675,11 +682,6 @@ tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dty
       scratch_of_device[ctx->device] = scratch;
     }
   }
-  tq::DecodePlan plan;
-  if (tq_status st = check_decode_args(ctx, q, q_dtype, cache, n_cache_pages, block_tables, max_pages_per_seq,
-                                       seq_lens, batch, n_q_heads, n_kv_heads, max_seq_len, scale, out,
-                                       scratch, tq::kNoAllocScratchBytes, &plan))
-    return st;   // TQ_ERR_WORKSPACE: the call needs more than the fixed scratch holds
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(tq::kHeadDim));
   return from_cuda(tq::launch_decode(ctx->tables, plan, q, q_dtype, cache, n_cache_pages,
                                      block_tables, max_pages_per_seq, seq_lens, max_seq_len,
@@ -701,6 +703,12 @@ tq_status tq_decode_logits(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const v
   return from_cuda(tq::launch_logits(ctx->tables, plan, q, q_dtype, cache, n_cache_pages, block_tables,
                                      max_pages_per_seq, seq_lens, max_seq_len, scale, logits, logits_stride,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+tq_status tq_set_test_flags(tq_ctx* ctx, unsigned flags) {
+  if (!ctx || (flags & ~TQ_TEST_WAIT_RUNS_OUT)) return TQ_ERR_INVALID_ARG;
+  ctx->tables.test_flags = flags;
+  return TQ_OK;
 }
 
 tq_status tq_set_sparse_v(tq_ctx* ctx, float tau) {

@@ -34,6 +34,7 @@ struct Tables {
   float m_rownorm = 0.0f;             // max over rows r of |M_r| (bounds |p_r| <= |M_r| |q|)
   const uint16_t* sketch_qb = nullptr;  // device fp16 bits of S as prefill B fragments [8 ks][16 nt][32 lane][2 reg][2]
   unsigned* err = nullptr;            // device error word
+  unsigned test_flags = 0;            // TQ_TEST_* bits (tq_set_test_flags)
 };
 
 // Workspace carve-up for one decode call; all offsets in bytes, 256-aligned.

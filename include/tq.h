@@ -251,13 +251,29 @@ tq_status tq_set_sparse_v(tq_ctx* ctx, float tau);
  * First call: the first call on a device looks up the scratch's device
  * address (cudaGetSymbolAddress), which may load the library's device code on
  * that device. Make that first call before any stream capture begins; later
- * calls only enqueue the kernel.
+ * calls only enqueue the kernel. Arguments and the size limit are checked
+ * before that lookup, so a rejected call touches no device. The address is
+ * kept for the life of the process: after a cudaDeviceReset of that device the
+ * call must not be used again.
  */
 tq_status tq_decode_attention_noalloc(tq_ctx* ctx, const void* q, tq_dtype q_dtype, const void* cache,
                                       int64_t n_cache_pages, const int32_t* block_tables,
                                       int max_pages_per_seq, const int32_t* seq_lens, int batch,
                                       int n_q_heads, int n_kv_heads, int max_seq_len, float scale,
                                       float* out, tq_stream stream);
+
+/*
+ * Test hook (no counterpart on the pages): makes a device-side failure path run
+ * without any fault. With TQ_TEST_WAIT_RUNS_OUT set, in every later decode call
+ * of this context warp 0 of thread block 0 first waits, with a short limit
+ * (2^16 clock cycles), on a shared-memory barrier that nothing completes. That
+ * wait runs out: the warp records TQ_DEV_TIMEOUT, lets its copies in flight
+ * land, stops reading pages and joins the merge, so the call finishes and its
+ * output stays finite but leaves out that warp's pages. flags = 0 (the
+ * default) turns it off. Unknown bits: TQ_ERR_INVALID_ARG. Host-side setting.
+ */
+#define TQ_TEST_WAIT_RUNS_OUT 0x1u
+tq_status tq_set_test_flags(tq_ctx* ctx, unsigned flags);
 
 /* Synchronise `stream`, then read and clear the device error word (TQ_DEV_* bits). */
 tq_status tq_get_device_error(tq_ctx* ctx, uint32_t* code, tq_stream stream);

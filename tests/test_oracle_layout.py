@@ -58,3 +58,26 @@ def test_byte_accounting():
     fp16_bytes = 80 * 8 * 128 * 2 * 2 * 131072
     assert fp16_bytes > 40e9
     assert abs(512 / 102 - 5.02) < 0.01
+
+
+def test_hand_derived_norm_and_scale_bytes():
+    # Each case writes one token with distinctive fp16 fields into a zero block and
+    # reads the two bytes at the hand-derived offset (not through norm_slot).
+    ref = json.load(open(os.path.join(GOLDEN, "layout_positions.json")))
+    vals = {"norm_k": 1.5, "gamma": 2.5, "norm_v": 3.5, "q8_norm_v": 3.5, "q8_scale": 0.75}
+    for c in ref["byte_cases"]:
+        bk, bv, tau = c["bk"], c["bv"], c["token"]
+        blk = np.zeros(lay.block_bytes(bk, bv), dtype=np.uint8)
+        if bk == 8:
+            scales = [0.25, 0.5, 0.75, 1.0]
+            lay.write_token_q8(blk, tau, bv, np.zeros(128, dtype=np.int64), scales, np.zeros(128, dtype=np.int64),
+                               3.5)
+        else:
+            lay.write_token(blk, tau, bk, bv, np.zeros(128, dtype=np.int64), np.zeros(128, dtype=np.int64),
+                            np.zeros(128, dtype=np.int64), 1.5, 2.5, 3.5)
+        got = float(blk[c["byte"]:c["byte"] + 2].view(np.float16)[0])
+        assert got == vals[c["field"]], c["derivation"]
+        # and nothing else in the norm/scale sections holds that value's bytes
+        want = np.array([vals[c["field"]]], dtype=np.float16).view(np.uint8)
+        hits = [i for i in range(0, blk.size - 1, 2) if blk[i] == want[0] and blk[i + 1] == want[1]]
+        assert hits == [c["byte"]], c["derivation"]

@@ -48,3 +48,17 @@ def test_sketch_rows_independent_across_seeds():
     b = rng.gaussian_sketch(2, 64, 64).ravel()
     r = np.corrcoef(a, b)[0, 1]
     assert abs(r) < 5 / np.sqrt(a.size)
+
+
+def test_sign_vector_first_entries_from_published_words():
+    # the top bits of the published seed-0 outputs fix the first three signs
+    ref = json.load(open(os.path.join(GOLDEN, "splitmix64_seed0.json")))
+    assert list(rng.sign_vector(0, 3)) == ref["sign_vector_first3"]
+
+
+def test_sketch_first_entry_from_published_words():
+    # entry (0, 0) of the seed-0 sketch, derived by hand from the published outputs 0 and 1
+    ref = json.load(open(os.path.join(GOLDEN, "splitmix64_seed0.json")))["sketch_entry0"]
+    s = rng.gaussian_sketch(0, 1, 1)
+    bits = np.array([s[0, 0]], dtype=np.float16).view(np.uint16)[0]
+    assert int(bits) == int(ref["value_fp16_bits"], 16)
