@@ -31,7 +31,6 @@ struct DecodeArgs {
   unsigned* counters;            // [pair]: finished CTAs; zero between calls
   float* out;                    // [batch][n_q][128]
   int n_kv, n_q, group, n_hg, chunks, ppc, n_pairs;
-  int merge_cap;                 // chunk records that fit in shared memory for the final merge
   int batch;
   int balanced;                  // 0: `chunks` uniform chunks of `ppc` pages per pair; 1: equal shares of all pages
   int seg_w;                     // balanced: fixed cost of one pair, in pages
@@ -903,7 +902,6 @@ constexpr int kAccPitch = 132;      // floats per accumulator column in the CTA 
 __host__ __device__ constexpr int decode_stages(int warps, int block) {
   return warps * 6 * block <= 160 * 1024 ? 6 : warps * 4 * block <= 160 * 1024 ? 4 : 3;
 }
-constexpr int kStatic = 2;       // pages per warp assigned before the block-table window is cached
 
 
 // ---- code words -> mma operands --------------------------------------------
@@ -1031,7 +1029,7 @@ constexpr int kQrawPitch = 136;     // floats per raw query row: the sketch's B 
 template <int NH>
 struct alignas(16) Prologue {
   alignas(16) float qraw[NH * kGroupHeads][kQrawPitch];   // queries as given (fp32)
-  alignas(16) uint32_t limb[NH * kGroupHeads][192];  // [which (q, p)][limb 0..2][32 words of 4 int8]
+  alignas(16) uint4 qb[NH][2][4][32];              // B fragments [group][q~ / p][k-tile][lane] (see put_frag)
   alignas(16) float cst[NH * kGroupHeads][4];      // a, b, sum P (int bits)
   alignas(16) float qn[NH * kGroupHeads];          // |q|
   alignas(16) float u[128];                        // appended key: R_K^T u (original domain)
@@ -1041,6 +1039,24 @@ struct alignas(16) Prologue {
   alignas(16) int sig[NH * kGroupHeads + 1];       // fp16 scaling exponents (last: appended key residual)
 };
 static_assert(offsetof(Prologue<1>, u) % 16 == 0 && offsetof(Prologue<3>, u) % 16 == 0, "alignment");
+
+// Store the three int8 limb words (Q2, Q1, Q0) of limb word `w` (coordinates or
+// sketch rows 4w .. 4w + 3) of head `hj` (0..3) of a group straight into the
+// B-fragment order the main loop reads: frag[k-tile][lane] holds, for lane (g, t),
+// the words (n-tile 0: k rows 4t.., 16 + 4t..; n-tile 1: the same rows) of column g,
+// where column 2 hj carries Q2 (n-tile 0) and Q0 (n-tile 1) and column 2 hj + 1
+// carries Q1 (n-tile 0) and zero (n-tile 1). Word w sits in k-tile w >> 3, at row
+// offset 16 ((w >> 2) & 1) + 4 (w & 3), i.e. lane t = w & 3, register (w >> 2) & 1.
+__device__ __forceinline__ void put_frag(uint4 (&frag)[4][32], int hj, int w, uint32_t q2, uint32_t q1,
+                                         uint32_t q0) {
+  const int kt = w >> 3, sub = (w >> 2) & 1, tt = w & 3;
+  uint32_t* even = reinterpret_cast<uint32_t*>(&frag[kt][4 * (2 * hj) + tt]);
+  uint32_t* odd = reinterpret_cast<uint32_t*>(&frag[kt][4 * (2 * hj + 1) + tt]);
+  even[sub] = q2;
+  odd[sub] = q1;
+  even[2 + sub] = q0;
+  odd[2 + sub] = 0u;
+}
 
 // Rotate and code one vector held 4 per lane; returns codes in o, n and (keys) gamma,
 // and the residual u = y - c[code] per lane.
@@ -1075,12 +1091,13 @@ __device__ __forceinline__ void rotate_and_code(const float (&x)[4], const float
 // segment: a run of consecutive pages of one (sequence, KV head) pair (the
 // kernel below says which segments a CTA serves). W warps per CTA, one CTA per
 // SM. Each warp streams the segment's pages through a private ring of S
-// shared-memory stages filled by 1-D bulk TMA copies. The first kStatic pages
-// of every warp are fixed (page p0 + warp + W k) and their copies go out before
-// any barrier; all later pages are claimed one at a time from a shared counter,
-// so warps that the scheduler favours take more pages and the warps of a CTA
-// finish together. The prologue (query transform, and with APPEND the
-// quantization of the new token) runs while the first copies are in flight.
+// shared-memory stages filled by 1-D bulk TMA copies. The first S pages of
+// every warp, one per stage, are fixed (page p0 + warp + W k) and their copies
+// go out as soon as the lengths and block table are read, before any barrier;
+// all later pages are claimed one at a time from a shared counter, so warps
+// that the scheduler favours take more pages and the warps of a CTA finish
+// together. The prologue (query transform, and with APPEND the quantization of
+// the new token) runs while the first copies are in flight.
 //
 // Per 16-token page a warp computes, with tokens on the rows of the products:
 //   logits  int8 m16n8k32: A = key-code limbs (hi, lo) or 0/1 sign bytes of
@@ -1112,10 +1129,10 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   constexpr int W = DecodeWarps<NH, LOOP>::value;
   constexpr int kBlock = block_bytes_of(BK, BV);
   constexpr int S = decode_stages(W, kBlock);
+  constexpr int kStatic = S;                   // pages per warp assigned before the claim counter
   constexpr int kSignOff = sec_scale(BK), kVOff = sec_v(BK), kNormOff = sec_norm(BK, BV);
   constexpr int kNormBytes = KQ8 ? 32 : 96;
   constexpr int kHeads = NH * kGroupHeads;
-  constexpr bool kRegQ = NH <= 2;              // query fragments in registers (else shared memory)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int pair = sg.pair;
@@ -1155,6 +1172,37 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       aml[ks] = __ldg(F + kQjlRows / 16 * 8 * 32 + ks * 32);
     }
   }
+  const float4 sgk = __ldg(reinterpret_cast<const float4*>(tab_sk) + lane);
+  const float4 sgv = __ldg(reinterpret_cast<const float4*>(tab_sv) + lane);
+  if (threadIdx.x < 16) {
+    P.tab[threadIdx.x] = T.thr_k[threadIdx.x];
+    P.tab[16 + threadIdx.x] = T.cen_k[threadIdx.x];
+    P.tab[32 + threadIdx.x] = T.thr_v[threadIdx.x];
+    P.tab[48 + threadIdx.x] = T.cen_v[threadIdx.x];
+  }
+  // Everything above reads only the context's own tables, which no kernel writes.
+  // Launched as a programmatic dependent of the previous kernel in the stream:
+  // its memory operations are complete and visible once this wait returns, so
+  // nothing it may have written (queries, lengths, block tables, the cache) is
+  // read before it. (With LOOP, the kernel has already waited.) Before the wait,
+  // only L2 prefetch hints go out for the lines read first after it: they move
+  // no data into the SM, so they cannot observe anything stale.
+  if constexpr (!LOOP) {
+    const int n_bt = (min(sg.len, A.max_pages_per_seq - sg.p0) * 4 + 127) >> 7;   // block-table lines
+    const int n_q = (A.group * 128 * (A.q_dtype == TQ_F32 ? 4 : 2) + 127) >> 7;   // query lines
+    const int i = threadIdx.x;
+    const char* addr = nullptr;
+    if (i == 0) addr = reinterpret_cast<const char*>(A.seq_lens + b);
+    else if (i <= n_bt)
+      addr = reinterpret_cast<const char*>(A.block_tables + static_cast<int64_t>(b) * A.max_pages_per_seq + sg.p0) +
+             128 * (i - 1);
+    else if (i <= n_bt + n_q)
+      addr = static_cast<const char*>(A.q) +
+             (static_cast<size_t>(b) * A.n_q + hk * A.group) * 128 * (A.q_dtype == TQ_F32 ? 4 : 2) +
+             128 * (i - 1 - n_bt);
+    if (addr) asm volatile("prefetch.global.L2 [%0];" ::"l"(addr));
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  }
   const size_t kv_row = static_cast<size_t>(b) * A.n_kv + hk;
   constexpr int kQJobs = (kHeads + W - 1) / W;     // query heads per warp (at most)
   float xq[kQJobs][4];
@@ -1168,8 +1216,6 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   const int ajob = warp == kHeads % W ? kHeads : (warp == (kHeads + 1) % W ? kHeads + 1 : -1);
   float xa[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (APPEND && ajob >= 0) load_row4(ajob == kHeads ? A.k_new : A.v_new, kv_row, A.kv_dtype, lane, xa);
-  const float4 sgk = __ldg(reinterpret_cast<const float4*>(tab_sk) + lane);
-  const float4 sgv = __ldg(reinterpret_cast<const float4*>(tab_sv) + lane);
   // this warp's static pages (lane k holds page p0 + warp + W k), fetched before
   // the length is known (bounded by the table width; pages past the sequence are
   // discarded below)
@@ -1266,12 +1312,6 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       }
     }
   }
-  if (threadIdx.x < 16) {
-    P.tab[threadIdx.x] = T.thr_k[threadIdx.x];
-    P.tab[16 + threadIdx.x] = T.cen_k[threadIdx.x];
-    P.tab[32 + threadIdx.x] = T.thr_v[threadIdx.x];
-    P.tab[48 + threadIdx.x] = T.cen_v[threadIdx.x];
-  }
   if (threadIdx.x == 0) s_claim = W * kStatic;
 #pragma unroll
   for (int r = 0; r < kSpecPer; ++r) {
@@ -1329,8 +1369,7 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     }
     const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
     const Limbs lq = split3(x, eq);
-    uint32_t* lm = P.limb[j];                      // [which (q, p)][limb 0..2][32 words of 4 int8]
-    lm[0 * 32 + lane] = lq.w0;  lm[1 * 32 + lane] = lq.w1;  lm[2 * 32 + lane] = lq.w2;
+    put_frag(P.qb[j >> 2][0], j & 3, lane, lq.w2, lq.w1, lq.w0);   // lane l: coordinates 4l .. 4l + 3
     if (lane == 0) {
       const bool real = j < A.group;
       P.cst[j][0] = real ? A.scale * kLog2e * pow2i(-eq - (KQ8 ? 0 : T.k_exp)) : 0.0f;
@@ -1438,14 +1477,10 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       ps += __shfl_xor_sync(kFull, ps, 4);
       ps += __shfl_xor_sync(kFull, ps, 8);
       ps += __shfl_xor_sync(kFull, ps, 16);
-      uint32_t* lm = P.limb[j] + 96;
       if ((g & 3) == 0) {
         const int wd = 4 * skw + (g >> 2);
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          lm[k * 32 + wd] = w[k];
-          lm[k * 32 + wd + 2] = w[3 + k];
-        }
+        put_frag(P.qb[h][1], t, wd, w[2], w[1], w[0]);
+        put_frag(P.qb[h][1], t, wd + 2, w[5], w[4], w[3]);
       }
       if (g == 0) {
         atomicAdd(reinterpret_cast<int*>(&P.cst[j][2]), j < A.group ? ps : 0);
@@ -1485,27 +1520,8 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   __syncwarp();
   __syncwarp();                           // lane 0's stage records are visible to the warp
 
-  // B fragment of lane (g, t): column g -> head 4h + g/2; rows 4t.. (+16 for reg 1) of k-tile kt
-  //   n-tile 0: limb 2 (g even) or 1 (g odd); n-tile 1: limb 0 (g even) or zero (g odd)
-  auto qword = [&](int h, int which, int kt, int nt, int sub) -> uint32_t {
-    const int limb = nt == 0 ? ((g & 1) ? 1 : 2) : 0;
-    const uint32_t v = P.limb[4 * h + (g >> 1)][which * 96 + limb * 32 + 8 * kt + 4 * sub + t];
-    return (nt == 1 && (g & 1)) ? 0u : v;
-  };
-  uint32_t bq[kRegQ ? NH : 1][4][2][2], bp[kRegQ ? NH : 1][4][2][2];
-  if constexpr (kRegQ) {
-#pragma unroll
-    for (int h = 0; h < NH; ++h)
-#pragma unroll
-      for (int kt = 0; kt < 4; ++kt)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int sub = 0; sub < 2; ++sub) {
-            bq[h][kt][nt][sub] = qword(h, 0, kt, nt, sub);
-            bp[h][kt][nt][sub] = qword(h, 1, kt, nt, sub);
-          }
-  }
+  // B fragments (query limbs): P.qb[group][q~ / p][k-tile][lane], one uint4 per lane
+  // and k-tile, read with one vector load per use (see put_frag).
   float ca[NH], cb[NH];
   int csum[NH];
 #pragma unroll
@@ -1619,13 +1635,9 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
           int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-          if constexpr (kRegQ) {
-            mma_s8(d0, ak, bq[h][kt][0][0], bq[h][kt][0][1]);
-            mma_s8(d1, ak, bq[h][kt][1][0], bq[h][kt][1][1]);
-          } else {
-            mma_s8(d0, ak, qword(h, 0, kt, 0, 0), qword(h, 0, kt, 0, 1));
-            mma_s8(d1, ak, qword(h, 0, kt, 1, 0), qword(h, 0, kt, 1, 1));
-          }
+          const uint4 fq = P.qb[h][0][kt][lane];
+          mma_s8(d0, ak, fq.x, fq.y);
+          mma_s8(d1, ak, fq.z, fq.w);
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             // columns: (Q2, Q1) of head t in d0, Q0 in d1; |Q2 . k| 2^16 can pass 2^31, so in fp32
@@ -1651,20 +1663,18 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
         as[2] = __umulhi(sw.x, 1u << (31 - 2 * kt)) & 0x01010101u;
         as[3] = __umulhi(sw.y, 1u << (31 - 2 * kt)) & 0x01010101u;
 #pragma unroll
-        for (int h = 0; h < NH; ++h)
+        for (int h = 0; h < NH; ++h) {
+          const uint4 fq = P.qb[h][0][kt][lane];
+          const uint4 fp = P.qb[h][1][kt][lane];
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
-            uint32_t q0, q1, r0, r1;
-            if constexpr (kRegQ) {
-              q0 = bq[h][kt][nt][0]; q1 = bq[h][kt][nt][1]; r0 = bp[h][kt][nt][0]; r1 = bp[h][kt][nt][1];
-            } else {
-              q0 = qword(h, 0, kt, nt, 0); q1 = qword(h, 0, kt, nt, 1);
-              r0 = qword(h, 1, kt, nt, 0); r1 = qword(h, 1, kt, nt, 1);
-            }
+            const uint32_t q0 = nt ? fq.z : fq.x, q1 = nt ? fq.w : fq.y;
+            const uint32_t r0 = nt ? fp.z : fp.x, r1 = nt ? fp.w : fp.y;
             mma_s8(dh[h][nt], ah, q0, q1);
-            mma_s8(dl[h][nt], al, q0, q1);
+            if (nt == 0) mma_s8(dl[h][nt], al, q0, q1);   // Q0 x C_lo (below 2^-22 of the sum) is left out
             mma_s8(ds[h][nt], as, r0, r1);
           }
+        }
       }
     }
 
@@ -1691,7 +1701,7 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
           l2 = ca[h] * lq8[h][r];
         } else {
           const int hiw = 256 * dh[h][0][2 * r] + dl[h][0][2 * r] + dh[h][0][2 * r + 1];
-          const int low = 256 * (dl[h][0][2 * r + 1] + dh[h][1][2 * r]) + dl[h][1][2 * r];
+          const int low = 256 * (dl[h][0][2 * r + 1] + dh[h][1][2 * r]);
           const float main = fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
           const int sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + ds[h][1][2 * r];
           const float nk = r ? nK.y : nK.x, gg = r ? gm.y : gm.x;
@@ -1806,53 +1816,67 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   if (sg.last) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if constexpr (LOGITS) return;                   // logits are written; nothing to merge
 
-  // ---- merge the warps of this CTA (the pipeline buffers are free now)
+  // ---- merge the warps of this CTA
 #pragma unroll
-  for (int h = 0; h < NH; ++h) {                 // sum each head's denominator over its 8 lanes
+  for (int h = 0; h < NH; ++h) {                        // each head's denominator over its 8 lanes
     lsum[h] += __shfl_xor_sync(kFull, lsum[h], 4);
     lsum[h] += __shfl_xor_sync(kFull, lsum[h], 8);
     lsum[h] += __shfl_xor_sync(kFull, lsum[h], 16);
   }
-  __syncthreads();
-  // [warp][NH][8 columns][kAccPitch]: the pitch of 132 floats puts the four
-  // column pairs a quad stores at once in different banks
+  __syncthreads();                                      // every warp is out of its page loop: stages free
+  // s_acc [W][kSlots][kAccPitch]: each warp's head sums (lanes t < 2 store the even
+  // m-tiles, t >= 2 the odd ones: with a pitch of 132 floats one store touches 32
+  // banks); s_m, s_l, s_f [W][kSlots]: running maximum, denominator and the factor
+  // 2^(m_w - M) towards the CTA's maximum M (s_M [kSlots]).
+  constexpr int kSlots = NH * kGroupHeads;
   float* s_acc = reinterpret_cast<float*>(smem);
-  float* s_st = s_acc + W * NH * 8 * kAccPitch;                          // [warp][NH][4 heads][3]
+  float* s_m = s_acc + W * kSlots * kAccPitch;
+  float* s_l = s_m + W * kSlots;
+  float* s_f = s_l + W * kSlots;
+  float* s_M = s_f + W * kSlots;
+  // Value-accumulator columns 2t, 2t + 1 of lane (g, t) hold heads 2 (t & 1) and
+  // 2 (t & 1) + 1 of each group: the high weight parts for t < 2, the low parts
+  // for t >= 2. Lanes t and t ^ 2 add them, so that both hold the head sums.
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
+    for (int mt = 0; mt < 8; ++mt) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int coord = 16 * mt + g + 8 * (c >> 1), col = 2 * t + (c & 1);
-        s_acc[((warp * NH + h) * 8 + col) * kAccPitch + coord] = acc[h][mt][c];
+        const float sum = acc[h][mt][c] + __shfl_xor_sync(kFull, acc[h][mt][c], 2);
+        const int slot = 4 * h + 2 * (t & 1) + (c & 1), coord = 16 * mt + g + 8 * (c >> 1);
+        if ((mt & 1) == (t >> 1)) s_acc[(warp * kSlots + slot) * kAccPitch + coord] = sum;
       }
+    }
     if (g == 0) {
-      float* st = s_st + ((warp * NH + h) * kGroupHeads + t) * 3;
-      st[0] = mp2[h]; st[1] = lsum[h];
+      s_m[warp * kSlots + 4 * h + t] = mp2[h];
+      s_l[warp * kSlots + 4 * h + t] = lsum[h];
     }
   }
   __syncthreads();
-  float* part = A.partial + static_cast<size_t>(sg.slot) * NH * kGroupHeads * 132;
-  for (int i = threadIdx.x; i < NH * kGroupHeads * 128; i += blockDim.x) {
-    const int hh = i >> 7, coord = i & 127;          // hh = group * 4 + head
-    const int h = hh >> 2, h4 = hh & 3;
+  if (threadIdx.x < W * kSlots) {                       // one thread per (warp, head slot)
+    const int w = threadIdx.x / kSlots, slot = threadIdx.x % kSlots;
     float M = kNegBig;
 #pragma unroll
-    for (int w = 0; w < W; ++w) M = fmaxf(M, s_st[((w * NH + h) * kGroupHeads + h4) * 3 + 0]);
-    float a = 0.0f, l = 0.0f;
+    for (int v = 0; v < W; ++v) M = fmaxf(M, s_m[v * kSlots + slot]);
+    s_f[w * kSlots + slot] = ex2(s_m[w * kSlots + slot] - M);
+    if (w == 0) s_M[slot] = M;
+  }
+  __syncthreads();
+  constexpr int kRec = 132;                             // floats per (segment, head slot) record
+  float* part = A.partial + static_cast<size_t>(sg.slot) * kSlots * kRec;
+  for (int i = threadIdx.x; i < kSlots * 128; i += blockDim.x) {
+    const int slot = i >> 7, coord = i & 127;
+    float a = 0.0f;
 #pragma unroll
-    for (int w = 0; w < W; ++w) {
-      const float* st = s_st + ((w * NH + h) * kGroupHeads + h4) * 3;
-      const float* ac = s_acc + ((w * NH + h) * 8) * kAccPitch;
-      const float f = ex2(st[0] - M);
-      a = fmaf(ac[h4 * kAccPitch + coord] + ac[(h4 + 4) * kAccPitch + coord], f, a);
-      l = fmaf(st[1], f, l);
-    }
-    part[hh * 132 + coord] = a;
+    for (int w = 0; w < W; ++w) a = fmaf(s_acc[(w * kSlots + slot) * kAccPitch + coord], s_f[w * kSlots + slot], a);
+    part[slot * kRec + coord] = a;
     if (coord == 0) {
-      part[hh * 132 + 128] = M;
-      part[hh * 132 + 129] = l;
+      float l = 0.0f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) l = fmaf(s_l[w * kSlots + slot], s_f[w * kSlots + slot], l);
+      part[slot * kRec + 128] = s_M[slot];
+      part[slot * kRec + 129] = l;
     }
   }
   // Publish the record: the barrier orders every thread's stores before thread 0's
@@ -1868,96 +1892,58 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   if (!s_last) return;
   if (threadIdx.x == 0) A.counters[pair] = 0u;    // every CTA has counted: ready for the next call
 
-  // ---- last CTA of this (sequence, KV head): merge the chunks, de-rotate, store.
-  // The chunk records (written by the other CTAs, published by the counter) come
-  // into shared memory by bulk copies, merge_cap chunks at a time. Warp w merges
-  // head slots w % 4 (+4, +8, ...) over the chunks c with c % (W / 4) == w / 4,
-  // with an online maximum; the W / 4 partial merges meet in shared memory.
-  constexpr int kRec = 132;                                  // floats per (chunk, head slot) record
-  constexpr int kSlots = NH * kGroupHeads;
-  const unsigned chunk_bytes = kSlots * kRec * 4;
+  // ---- last CTA of this (sequence, KV head): merge the records of all the pair's
+  // segments, de-rotate, store. kParts warps share a head slot, each taking every
+  // kParts-th record; lane l holds coordinates 4l .. 4l + 3 (the layout of the
+  // inverse rotation). Records come straight from L2 (ld.global.cg), all of a
+  // warp's loads in flight at once; the parts meet in shared memory.
+  constexpr int kParts = W >= kSlots ? W / kSlots : 1;
   const float* pbase = A.partial + static_cast<size_t>(sg.first_slot) * kSlots * kRec;
-  float* s_part = reinterpret_cast<float*>(smem);            // [merge_cap][kSlots][kRec]
-  constexpr int kGroups = W / kGroupHeads;                   // warps per head slot
-  float* s_mrg = s_part + static_cast<size_t>(A.merge_cap) * kSlots * kRec;   // [kGroups][kSlots][kRec]
-  uint64_t* fbar = reinterpret_cast<uint64_t*>(s_mrg + kGroups * kSlots * kRec);
-  const float4 sv = __ldg(reinterpret_cast<const float4*>(tab_sv) + lane);
-  if (threadIdx.x == 0) {
-    mbar_init(fbar, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  const int grp = warp / kGroupHeads, sl0 = warp % kGroupHeads;
-  float M[NH], l[NH], a[NH][4];
+  const int n_rec = sg.n_segs;
+  float* s_v = reinterpret_cast<float*>(smem);           // [kParts][kSlots][kRec]
+  for (int sl0 = 0; sl0 < kSlots; sl0 += (kParts > 1 ? kSlots : W)) {
+    const int slot = sl0 + (kParts > 1 ? warp % kSlots : warp);
+    const int prt = kParts > 1 ? warp / kSlots : 0;
+    if (slot < kSlots && prt < kParts) {                  // warp-uniform
+      // the slot's largest maximum over all records (lane c reads record c)
+      float M = kNegBig;
+      for (int c = lane; c < n_rec; c += 32)
+        M = fmaxf(M, __ldcg(pbase + (static_cast<size_t>(c) * kSlots + slot) * kRec + 128));
+      M = warp_max(M);
+      float v[4] = {0.f, 0.f, 0.f, 0.f}, lt = 0.0f;
+      for (int c0 = prt; c0 < n_rec; c0 += 8 * kParts) {
+        float4 x[8];
+        float2 ml[8];
 #pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    M[h] = kNegBig; l[h] = 0.0f;
-    a[h][0] = a[h][1] = a[h][2] = a[h][3] = 0.0f;
-  }
-  bool landed = true;
-  unsigned ph = 0;
-  for (int c0 = 0; c0 < sg.n_segs; c0 += A.merge_cap, ph ^= 1u) {
-    const int nc = min(A.merge_cap, sg.n_segs - c0);
-    if (threadIdx.x == 0) {
-      // generic-proxy writes of the other CTAs, read next by the bulk-copy unit
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      mbar_expect_tx(fbar, nc * chunk_bytes);
-      tma_load_1d(s_part, pbase + static_cast<size_t>(c0) * kSlots * kRec, nc * chunk_bytes, fbar);
-    }
-    // the whole CTA leaves together when any thread's wait ran out, so that all
-    // of it meets the same barriers
-    if (__syncthreads_or(!mbar_wait(fbar, ph))) {
-      if (threadIdx.x == 0) set_error(T.err, TQ_DEV_TIMEOUT);
-      landed = false;
-      break;
-    }
+        for (int k = 0; k < 8; ++k) {                     // issue every load of the batch first
+          const int c = c0 + k * kParts;
+          const float* rec = pbase + (static_cast<size_t>(c < n_rec ? c : prt) * kSlots + slot) * kRec;
+          x[k] = __ldcg(reinterpret_cast<const float4*>(rec) + lane);
+          ml[k] = __ldcg(reinterpret_cast<const float2*>(rec + 128));
+        }
 #pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      const int slot = sl0 + kGroupHeads * h;
-      if (slot >= A.group) continue;
-#pragma unroll 4
-      for (int c = grp; c < nc; c += kGroups) {
-        const float* rec = s_part + (c * kSlots + slot) * kRec;
-        const float Mc = rec[128];
-        const float Mn = fmaxf(M[h], Mc);
-        const float fo = ex2(M[h] - Mn), fc = ex2(Mc - Mn);
-        const float4 v = reinterpret_cast<const float4*>(rec)[lane];
-        l[h] = fmaf(l[h], fo, rec[129] * fc);
-        a[h][0] = fmaf(a[h][0], fo, v.x * fc); a[h][1] = fmaf(a[h][1], fo, v.y * fc);
-        a[h][2] = fmaf(a[h][2], fo, v.z * fc); a[h][3] = fmaf(a[h][3], fo, v.w * fc);
-        M[h] = Mn;
+        for (int k = 0; k < 8; ++k) {
+          const float f = c0 + k * kParts < n_rec ? ex2(ml[k].x - M) : 0.0f;
+          lt = fmaf(ml[k].y, f, lt);
+          v[0] = fmaf(x[k].x, f, v[0]); v[1] = fmaf(x[k].y, f, v[1]);
+          v[2] = fmaf(x[k].z, f, v[2]); v[3] = fmaf(x[k].w, f, v[3]);
+        }
       }
+      float* mine = s_v + (prt * kSlots + slot) * kRec;
+      reinterpret_cast<float4*>(mine)[lane] = make_float4(v[0], v[1], v[2], v[3]);
+      if (lane == 0) mine[128] = lt;
     }
-    __syncthreads();                                          // s_part is free for the next piece
-  }
-  if (!landed) {                                              // CTA-uniform
-    mbar_wait(fbar, ph);                                      // bounded: let the copy land before exit
-    if constexpr (LOOP) {                                     // the barrier's memory is reused
-      __syncthreads();
-      if (threadIdx.x == 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(fbar)) : "memory");
-    }
-    return;
-  }
-#pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    const int slot = sl0 + kGroupHeads * h;
-    float* mine = s_mrg + (grp * kSlots + slot) * kRec;
-    reinterpret_cast<float4*>(mine)[lane] = make_float4(a[h][0], a[h][1], a[h][2], a[h][3]);
-    if (lane == 0) { mine[128] = M[h]; mine[129] = l[h]; }
   }
   __syncthreads();
+  const float4 sv = __ldg(reinterpret_cast<const float4*>(tab_sv) + lane);
   for (int slot = warp; slot < A.group; slot += W) {
-    float Mx = kNegBig;
+    float v[4] = {0.f, 0.f, 0.f, 0.f}, lt = 0.0f;
 #pragma unroll
-    for (int q = 0; q < kGroups; ++q) Mx = fmaxf(Mx, s_mrg[(q * kSlots + slot) * kRec + 128]);
-    float lt = 0.0f, v[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int q = 0; q < kGroups; ++q) {
-      const float* r = s_mrg + (q * kSlots + slot) * kRec;
-      const float f = ex2(r[128] - Mx);
+    for (int q = 0; q < kParts; ++q) {
+      const float* r = s_v + (q * kSlots + slot) * kRec;
       const float4 x = reinterpret_cast<const float4*>(r)[lane];
-      lt = fmaf(r[129], f, lt);
-      v[0] = fmaf(x.x, f, v[0]); v[1] = fmaf(x.y, f, v[1]); v[2] = fmaf(x.z, f, v[2]); v[3] = fmaf(x.w, f, v[3]);
+      lt += r[128];
+      v[0] += x.x; v[1] += x.y; v[2] += x.z; v[3] += x.w;
     }
     const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
 #pragma unroll
@@ -1971,8 +1957,6 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     const int qh = hk * A.group + slot;
     reinterpret_cast<float4*>(A.out + (static_cast<size_t>(b) * A.n_q + qh) * 128)[lane] = o;
   }
-  // the barrier's memory is reused by the next segment's stages
-  if (threadIdx.x == 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(fbar)) : "memory");
 }
 
 // The decode launch.
@@ -1985,9 +1969,10 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
 template <int BK, int BV, int NH, int MODE, bool BAL>
 __global__ void __launch_bounds__(DecodeWarps<NH, BAL>::value * 32, 1) decode_kernel(Tables T, DecodeArgs A) {
   // Launched as a programmatic dependent of the previous kernel in the stream: its
-  // memory operations are complete and visible once this wait returns, so nothing
-  // of the previous kernel's output is touched before it.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // memory operations are complete and visible once the grid-dependency wait
+  // returns. The uniform split waits inside the segment body, after loading the
+  // context's constant tables; the balanced split reads the lengths first.
+  if constexpr (BAL) asm volatile("griddepcontrol.wait;" ::: "memory");
   if constexpr (!BAL) {
     Segment sg;
     sg.pair = static_cast<int>(blockIdx.x % static_cast<unsigned>(A.n_pairs));
@@ -2147,17 +2132,17 @@ cudaError_t launch_decode_tb(const Tables& T, const DecodeArgs& a, dim3 grid, cu
   // main loop: stages, barriers, prologue scratch, the chunk's block-table window
   const size_t pipe = static_cast<size_t>(W) * S * kBlock + W * S * sizeof(uint64_t) + sizeof(Prologue<NH>) +
                       ((static_cast<size_t>(a.ppc) * 4 + 15) & ~static_cast<size_t>(15));
-  // CTA merge: every warp's accumulators and softmax state
-  const size_t merge = static_cast<size_t>(W) * NH * 8 * kAccPitch * 4 + W * NH * kGroupHeads * 3 * 4;
+  // CTA merge: every warp's head sums [W][slots][kAccPitch] and softmax state
+  // [3][W][slots] + [slots]; the final merge reuses the same space for at most
+  // max(W, slots) records of 132 floats
+  constexpr size_t kSlotsL = static_cast<size_t>(NH) * kGroupHeads;
+  const size_t merge = (W * kSlotsL * kAccPitch + 3 * W * kSlotsL + kSlotsL) * 4;
+  static_assert((W > static_cast<int>(kSlotsL) ? W : kSlotsL) * 132 <= W * kSlotsL * kAccPitch, "final merge space");
   const size_t base = ((pipe > merge ? pipe : merge) + 15) & ~static_cast<size_t>(15);
   // balanced mode: two [batch + 1] prefixes of the split, after everything else
   const size_t smem = base + (BAL ? (2 * static_cast<size_t>(a.batch) + 2) * 4 : 0);
-  // final merge: merge_cap chunk records, then [W / 4][slots][132] floats and one barrier
-  const size_t chunk_bytes = static_cast<size_t>(NH) * kGroupHeads * 132 * 4;
-  const size_t groups = W / kGroupHeads;
-  if (smem > 227 * 1024 || base < (groups + 1) * chunk_bytes + 16) return cudaErrorInvalidConfiguration;
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   DecodeArgs args = a;
-  args.merge_cap = static_cast<int>((base - groups * chunk_bytes - 16) / chunk_bytes);
   args.vs_off = static_cast<int>(base);
   auto fn = decode_kernel<BK, BV, NH, MODE, BAL>;
   static size_t configured = 0;     // raise the shared-memory limit once per instantiation
