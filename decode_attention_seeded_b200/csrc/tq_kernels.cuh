@@ -1157,7 +1157,17 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   uint64_t* mybar = bars + warp * S;
   int* mylp = s_lp + warp * S;
 
-  // The prologue's own loads go out first, ahead of the page stream, so that they
+  // The ring barriers first: they touch only this CTA's shared memory, and their
+  // initialisation fences wait for this thread's earlier memory operations, so
+  // they go ahead of every global load (a previous segment of this CTA may have
+  // written the stage bytes through the generic proxy; bulk copies write them next).
+  if (lane == 0) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    for (int s = 0; s < S; ++s) mbar_init(mybar + s, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  // The prologue's own loads go out next, ahead of the page stream, so that they
   // do not queue behind it: the last eight warps' rows of M = S R_K (fp16 high
   // and low parts as m16n8k16 A fragments) and the inputs of this warp's jobs
   // (query heads warp, warp + W, ...; with APPEND the new key or value).
@@ -1233,15 +1243,6 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     const int i = threadIdx.x + r * W * 32;
     spec_win[r] = i < win_lim ? __ldg(btab + p0 + W * kStatic + i) : -1;
   }
-
-  if (lane == 0) {
-    // a previous segment of this CTA may have written these bytes through the
-    // generic proxy; they are next written by bulk copies
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    for (int s = 0; s < S; ++s) mbar_init(mybar + s, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncwarp();
 
   int L = A.seq_lens[b];
   if (L < 0 || L > A.max_seq_len) {
@@ -1566,23 +1567,19 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     }
     __syncwarp();
   }
-  while (inflight > 0) {
-    // warp-uniform outcome: the page body runs warp-wide shuffles and mma.sync
-    bool landed;
-    if (runout) {
-      landed = __all_sync(kFull, mbar_wait(&s_never, 0u, 1ll << 16));
-      runout = false;
-    } else {
-      landed = __all_sync(kFull, mbar_wait(mybar + s, parity));
-    }
-    if (!landed) {
-      if (lane == 0) set_error(T.err, TQ_DEV_TIMEOUT);
-      alive = false;
-      break;
-    }
-    const int lp = mylp[s];
+  // ---- one page's logits (row a4, first half): returns, for tokens g and g + 8 of
+  // the page in stage st and each head group, l2 + log2|v| (l2 = the logit in log2
+  // units; -inf outside the sequence), the token's 1 / |v| and log2|v|, and the
+  // page's value-code words.
+  struct PageLogits {
+    float lp2[NH][2];
+    float rnv[2], lgv[2];
+    uint32_t vw[2 * BV];
+  };
+  auto page_logits = [&](int st, PageLogits& o) {
+    const int lp = mylp[st];
     const bool page_ok = lp >= 0;
-    const uint8_t* blk = stage0 + s * kBlock;
+    const uint8_t* blk = stage0 + st * kBlock;
 
     // ---- this lane's operands from the staged block (tokens g and g + 8)
     // (q8_0 keys: 16 words of int8 key values, the same count as 2 * 8 code words)
@@ -1592,8 +1589,7 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     uint4 sc4 = make_uint4(0u, 0u, 0u, 0u);   // q8_0: fp16 block scales 4 th + kt of tokens g, g + 8
     if constexpr (KQ8) sc4 = *reinterpret_cast<const uint4*>(blk + kSignOff + 16 * g);
     else sw = reinterpret_cast<const uint2*>(blk + kSignOff)[lane];
-    uint32_t vw[2 * BV];
-    if constexpr (!LOGITS) lds_words<2 * BV>(reinterpret_cast<const uint32_t*>(blk + kVOff) + lane * 2 * BV, vw);
+    if constexpr (!LOGITS) lds_words<2 * BV>(reinterpret_cast<const uint32_t*>(blk + kVOff) + lane * 2 * BV, o.vw);
     const uint32_t* nrm = reinterpret_cast<const uint32_t*>(blk + kNormOff);
     float2 nK = make_float2(0.0f, 0.0f), gm = make_float2(0.0f, 0.0f), nV;
     if constexpr (KQ8) {
@@ -1678,24 +1674,19 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       }
     }
 
-    // ---- softmax: one running maximum of l2 + log2|v| per head. The fp16 weight
-    // of token t is w_t = 2^(l2_t + log2|v_t| - m) <= 2^8 (the maximum is only
-    // moved when it grows by more than 8), and the softmax denominator gathers
-    // w_t / |v_t| = 2^(l2_t - m). Norms are floored at 2^-24 so that a zero value
-    // vector still counts in the denominator.
+    // One running maximum of l2 + log2|v| per head (see the softmax below). Norms
+    // are floored at 2^-24 so that a zero value vector still counts in the denominator.
     const int n_valid = page_ok ? L - lp * kPage : 0;     // tokens of this page inside the sequence
-    const float lgv0 = lg2(fmaxf(nV.x, 5.9604645e-8f)), lgv1 = lg2(fmaxf(nV.y, 5.9604645e-8f));
-    const float rnv0 = ex2(-lgv0), rnv1 = ex2(-lgv1);
-    uint32_t pb[NH][2];
-    bool kept = false;                      // Sparse V: this lane keeps a (token, head) value
+    o.lgv[0] = lg2(fmaxf(nV.x, 5.9604645e-8f));
+    o.lgv[1] = lg2(fmaxf(nV.y, 5.9604645e-8f));
+    o.rnv[0] = ex2(-o.lgv[0]);
+    o.rnv[1] = ex2(-o.lgv[1]);
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
-      float lp2[2];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         // accumulator columns: n-tile 0 -> (Q2, Q1) of head t, n-tile 1 -> (Q0, 0)
-        //   <Q,C> = 2^16 (256 Q2.Chi + Q2.Clo + Q1.Chi) + 256 (Q1.Clo + Q0.Chi) + Q0.Clo
-        const float lv = r ? lgv1 : lgv0;
+        //   <Q,C> = 2^16 (256 Q2.Chi + Q2.Clo + Q1.Chi) + 256 (Q1.Clo + Q0.Chi) [+ Q0.Clo, left out]
         float l2;
         if constexpr (KQ8) {
           l2 = ca[h] * lq8[h][r];
@@ -1713,10 +1704,23 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
             A.logits[(static_cast<int64_t>(b) * A.n_q + hk * A.group + qi) * A.logits_stride + lp * kPage + g +
                      8 * r] = l2 * 0.6931471805599453f;
         }
-        lp2[r] = (g + 8 * r) < n_valid ? l2 + lv : -INFINITY;
+        o.lp2[h][r] = (g + 8 * r) < n_valid ? l2 + o.lgv[r] : -INFINITY;
       }
-      if constexpr (LOGITS) continue;
-      float pm = fmaxf(lp2[0], lp2[1]);
+    }
+  };
+
+  // ---- softmax over one or two pages (row a4, second half): one running maximum
+  // of l2 + log2|v| per head. The fp16 weight of token t is
+  // w_t = 2^(l2_t + log2|v_t| - m) <= 2^8 (the maximum is only moved when it grows
+  // by more than 8), and the softmax denominator gathers w_t / |v_t| = 2^(l2_t - m).
+  // Returns each page's value-product B operand (weights as fp16 high and low
+  // parts, transposed into place) and whether its values may be skipped (Sparse V).
+  auto softmax = [&](int npg, PageLogits* pg, uint32_t (*pb)[NH][2], bool* skip) {
+    bool kept[2] = {false, false};        // Sparse V: this lane keeps a (token, head) value
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      float pm = fmaxf(pg[0].lp2[h][0], pg[0].lp2[h][1]);
+      if (npg == 2) pm = fmaxf(pm, fmaxf(pg[1].lp2[h][0], pg[1].lp2[h][1]));
       pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 4));
       pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 8));
       pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 16));
@@ -1733,69 +1737,112 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
           acc[h][mt][0] *= f0; acc[h][mt][1] *= f1; acc[h][mt][2] *= f0; acc[h][mt][3] *= f1;
         }
       }
-      float w0 = ex2(lp2[0] - mp2[h]), w1 = ex2(lp2[1] - mp2[h]);
-      lsum[h] = fmaf(w0, rnv0, fmaf(w1, rnv1, lsum[h]));
-      if (A.sparse) {
-        // Sparse V: a value is skipped when its attention weight is below the
-        // threshold times the largest weight seen so far by this warp (never more
-        // than the largest overall); the denominator above still counts it.
-        const float l20 = lp2[0] - lgv0, l21 = lp2[1] - lgv1;
-        float ps = fmaxf(l20, l21);
-        ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 4));
-        ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 8));
-        ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 16));
-        smx[h] = fmaxf(smx[h], ps);
-        const float cut = smx[h] + A.sparse_log2;
-        const bool k0 = l20 >= cut, k1 = l21 >= cut;
-        w0 = k0 ? w0 : 0.0f;
-        w1 = k1 ? w1 : 0.0f;
-        kept = kept || k0 || k1;
-      }
-      // weights of (token g, head t) and (token g+8, head t): high fp16 parts and residuals
-      const __half2 whi = __floats2half2_rn(w0, w1);
-      const float2 wr = __half22float2(whi);
-      const __half2 wlo = __floats2half2_rn(w0 - wr.x, w1 - wr.y);
-      const uint32_t uhi = *reinterpret_cast<const uint32_t*>(&whi);
-      const uint32_t ulo = *reinterpret_cast<const uint32_t*>(&wlo);
-      // value-product B operand: lane (g', t') needs column g' (head g'&3, high part
-      // if g' < 4) at tokens 2t', 2t'+1 (-> b0) and 2t'+8, 2t'+9 (-> b1); tokens 2t'
-      // and 2t'+8 of a head live in lane 4*(2t') + head, tokens 2t'+1, 2t'+9 in the next quad.
-      const uint32_t x0h = __shfl_sync(kFull, uhi, src0), x0l = __shfl_sync(kFull, ulo, src0);
-      const uint32_t x1h = __shfl_sync(kFull, uhi, src1), x1l = __shfl_sync(kFull, ulo, src1);
-      const uint32_t x0 = hi_col ? x0h : x0l, x1 = hi_col ? x1h : x1l;
-      pb[h][0] = prmt(x0, x1, 0x5410u);
-      pb[h][1] = prmt(x0, x1, 0x7632u);
-    }
-
-    // ---- weighted value sum in the rotated domain: fp16 tensor-core products
-    // (Sparse V: skipped for a page whose values are all below the threshold)
-    if (!LOGITS && (!A.sparse || __any_sync(kFull, kept))) {
-      uint32_t vs[16];
-      value_selectors<BV>(vw, vs);
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        value_regs<BV>(vs[2 * mt], vlo_, vhi_, a0, a1);
-        value_regs<BV>(vs[2 * mt + 1], vlo_, vhi_, a2, a3);
-#pragma unroll
-        for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pb[h][0], pb[h][1]);
+      for (int q = 0; q < 2; ++q) {
+        if (q == 1 && npg == 1) break;
+        const PageLogits& o = pg[q];
+        float w0 = ex2(o.lp2[h][0] - mp2[h]), w1 = ex2(o.lp2[h][1] - mp2[h]);
+        lsum[h] = fmaf(w0, o.rnv[0], fmaf(w1, o.rnv[1], lsum[h]));
+        if (A.sparse) {
+          // Sparse V: a value is skipped when its attention weight is below the
+          // threshold times the largest weight seen so far by this warp (never more
+          // than the largest overall); the denominator above still counts it.
+          const float l20 = o.lp2[h][0] - o.lgv[0], l21 = o.lp2[h][1] - o.lgv[1];
+          float ps = fmaxf(l20, l21);
+          ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 4));
+          ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 8));
+          ps = fmaxf(ps, __shfl_xor_sync(kFull, ps, 16));
+          smx[h] = fmaxf(smx[h], ps);
+          const float cut = smx[h] + A.sparse_log2;
+          const bool k0 = l20 >= cut, k1 = l21 >= cut;
+          w0 = k0 ? w0 : 0.0f;
+          w1 = k1 ? w1 : 0.0f;
+          kept[q] = kept[q] || k0 || k1;
+        }
+        // weights of (token g, head t) and (token g+8, head t): high fp16 parts and residuals
+        const __half2 whi = __floats2half2_rn(w0, w1);
+        const float2 wr = __half22float2(whi);
+        const __half2 wlo = __floats2half2_rn(w0 - wr.x, w1 - wr.y);
+        const uint32_t uhi = *reinterpret_cast<const uint32_t*>(&whi);
+        const uint32_t ulo = *reinterpret_cast<const uint32_t*>(&wlo);
+        // value-product B operand: lane (g', t') needs column g' (head g'&3, high part
+        // if g' < 4) at tokens 2t', 2t'+1 (-> b0) and 2t'+8, 2t'+9 (-> b1); tokens 2t'
+        // and 2t'+8 of a head live in lane 4*(2t') + head, tokens 2t'+1, 2t'+9 in the next quad.
+        const uint32_t x0h = __shfl_sync(kFull, uhi, src0), x0l = __shfl_sync(kFull, ulo, src0);
+        const uint32_t x1h = __shfl_sync(kFull, uhi, src1), x1l = __shfl_sync(kFull, ulo, src1);
+        const uint32_t x0 = hi_col ? x0h : x0l, x1 = hi_col ? x1h : x1l;
+        pb[q][h][0] = prmt(x0, x1, 0x5410u);
+        pb[q][h][1] = prmt(x0, x1, 0x7632u);
       }
     }
+    skip[0] = A.sparse && !__any_sync(kFull, kept[0]);
+    skip[1] = A.sparse && !__any_sync(kFull, kept[1]);
+  };
 
-    // ---- refill this stage with the pending claim (all its reads are consumed),
-    // and claim the next page; that claim is only used at the next refill
+  // ---- weighted value sum in the rotated domain: fp16 tensor-core products
+  auto value_product = [&](const uint32_t (&vw)[2 * BV], const uint32_t (&pbq)[NH][2]) {
+    uint32_t vs[16];
+    value_selectors<BV>(vw, vs);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      value_regs<BV>(vs[2 * mt], vlo_, vhi_, a0, a1);
+      value_regs<BV>(vs[2 * mt + 1], vlo_, vhi_, a2, a3);
+#pragma unroll
+      for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pbq[h][0], pbq[h][1]);
+    }
+  };
+
+  // ---- refill stage st with the pending claim (all its reads are consumed), and
+  // claim the next page; that claim is only used at the next refill
+  auto refill_stage = [&](int st) {
     const bool refill = __shfl_sync(kFull, pend, 0) >= 0;
     __syncwarp();
     if (lane == 0 && refill) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(s_btab[pend - p0 - W * kStatic], pend, s);
+      issue(s_btab[pend - p0 - W * kStatic], pend, st);
       const int next = p0 + atomicAdd(&s_claim, 1);
       pend = next < p1 ? next : -1;
     }
     __syncwarp();
     if (!refill) --inflight;
-    if (++s == S) {
-      s = 0;
+  };
+
+  while (inflight > 0) {
+    // Two pages per iteration while two are in flight: their key work is
+    // independent and interleaves; the softmax reduction is shared.
+    const int npg = inflight >= 2 ? 2 : 1;
+    const int s2 = s + 1 == S ? 0 : s + 1;
+    const unsigned parity2 = s + 1 == S ? parity ^ 1u : parity;
+    // warp-uniform outcome: the page body runs warp-wide shuffles and mma.sync
+    bool landed;
+    if (runout) {
+      landed = __all_sync(kFull, mbar_wait(&s_never, 0u, 1ll << 16));
+      runout = false;
+    } else {
+      landed = __all_sync(kFull, mbar_wait(mybar + s, parity));
+    }
+    if (landed && npg == 2) landed = __all_sync(kFull, mbar_wait(mybar + s2, parity2));
+    if (!landed) {
+      if (lane == 0) set_error(T.err, TQ_DEV_TIMEOUT);
+      alive = false;
+      break;
+    }
+    PageLogits pg[2];
+    page_logits(s, pg[0]);
+    if (npg == 2) page_logits(s2, pg[1]);
+    if constexpr (!LOGITS) {
+      uint32_t pb[2][NH][2];
+      bool skip[2];
+      softmax(npg, pg, pb, skip);
+      if (!skip[0]) value_product(pg[0].vw, pb[0]);
+      if (npg == 2 && !skip[1]) value_product(pg[1].vw, pb[1]);
+    }
+    refill_stage(s);
+    if (npg == 2) refill_stage(s2);
+    s += npg;
+    if (s >= S) {
+      s -= S;
       parity ^= 1u;
     }
   }
