@@ -801,6 +801,9 @@ def main():
     g_warm = bench.capture(bench.step, range(W))
     g_main = bench.capture(bench.step, range(W, W + K))
     g_warm.replay()
+    # one untimed replay of the timed graph: its first launch uploads the graph to
+    # the device; the K steps rewrite the same slots with the same data when timed
+    g_main.replay()
     torch.cuda.synchronize(dev)
     assert bench.ctx.device_error() == 0
 
@@ -820,6 +823,7 @@ def main():
     g_e2e = bench.capture(bench.step_e2e, range(W, W + K))
     g_e2e_w = bench.capture(bench.step_e2e, range(W))
     g_e2e_w.replay()
+    g_e2e.replay()                                        # graph upload, untimed (as above)
     barrier()
     t_e2e = max_over_ranks(timed(torch, dev, g_e2e.replay), world, dev)
     barrier()

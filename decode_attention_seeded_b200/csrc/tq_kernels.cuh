@@ -75,6 +75,15 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -560,13 +569,98 @@ __device__ __forceinline__ void pf_fwht(float (&v)[2][32], int lane) {
   }
 }
 
+// Rotation of 16-bit inputs on the tensor cores. The Walsh-Hadamard matrix
+// factors over the coordinate bits, H_128 = H_8 (bits 4-6) x H_16 (bits 0-3), so
+// each 16-coordinate block ks of the 16-token tile is one m16n8k16 product pair
+// X_ks (D_ks H_16) with the rotation signs D_ks folded into the B operand: the
+// products are +-x exactly and only the fp32 accumulation rounds. The three
+// stages across blocks stay in registers.
+//
+// The k index kappa of the product is ordered so that the A fragment registers
+// are the staged input words as they are (lane (g, t): coordinates 4t .. 4t + 3
+// of its two tokens, two per word), and the columns so that the accumulators
+// land in the lane layout of pf_coord: kappa -> block coordinate pf_kin(kappa),
+// column n of n-tile nt -> block coordinate pf_kout(nt, n).
+__host__ __device__ constexpr int pf_kin(int kappa) {
+  return 4 * ((kappa & 7) >> 1) + 2 * (kappa >> 3) + (kappa & 1);
+}
+__host__ __device__ constexpr int pf_kout(int nt, int n) { return 4 * (n >> 1) + 2 * nt + (n & 1); }
+
+// B fragments of all blocks of one sign vector, [ks][lane] uint4 = (b0, b1) of
+// n-tile 0, then of n-tile 1; entries +-1 as bf16 (bf16 inputs) or fp16.
+__device__ __forceinline__ uint4 pf_rot_frag(const float* signs, int ks, int lane, bool bf16) {
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t one = bf16 ? 0x3F80u : 0x3C00u;
+  uint32_t w[4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      uint32_t word = 0u;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int c = pf_kin(2 * t + 8 * r + j), o = pf_kout(nt, g);
+        const bool neg = (signs[16 * ks + c] < 0.0f) != ((__popc(c & o) & 1) != 0);
+        word |= (one | (neg ? 0x8000u : 0u)) << (16 * j);
+      }
+      w[2 * nt + r] = word;
+    }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The lane's 32 rotated (unnormalised: H D x) coordinates of tokens g, g + 8 from
+// staged 16-bit rows, and both tokens' squared norms |x|^2 = |H D x|^2 / 128.
+// Rows of tokens outside the run hold stale data; their results are never stored
+// (every product row depends only on its own input row).
+__device__ __forceinline__ void pf_rotate16(const uint8_t* rows, int pitch, bool bf16, int g, int t,
+                                            const uint4* frag, int lane, float (&v)[2][32], float (&ss)[2]) {
+  const uint8_t* r0 = rows + g * pitch + 8 * t;
+  const uint8_t* r1 = r0 + 8 * pitch;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const uint2 x0 = *reinterpret_cast<const uint2*>(r0 + 32 * ks);
+    const uint2 x1 = *reinterpret_cast<const uint2*>(r1 + 32 * ks);
+    const uint4 b = frag[ks * 32 + lane];
+    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+    if (bf16) {
+      mma_bf16(z0, x0.x, x1.x, x0.y, x1.y, b.x, b.y);
+      mma_bf16(z1, x0.x, x1.x, x0.y, x1.y, b.z, b.w);
+    } else {
+      mma_f16(z0, x0.x, x1.x, x0.y, x1.y, b.x, b.y);
+      mma_f16(z1, x0.x, x1.x, x0.y, x1.y, b.z, b.w);
+    }
+    v[0][4 * ks + 0] = z0[0]; v[0][4 * ks + 1] = z0[1]; v[1][4 * ks + 0] = z0[2]; v[1][4 * ks + 1] = z0[3];
+    v[0][4 * ks + 2] = z1[0]; v[0][4 * ks + 3] = z1[1]; v[1][4 * ks + 2] = z1[2]; v[1][4 * ks + 3] = z1[3];
+  }
+#pragma unroll
+  for (int th = 0; th < 2; ++th) {
+#pragma unroll
+    for (int bit = 2; bit < 5; ++bit)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (!(i & (1 << bit))) {
+          const float a = v[th][i], b = v[th][i | (1 << bit)];
+          v[th][i] = a + b;
+          v[th][i | (1 << bit)] = a - b;
+        }
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc = fmaf(v[th][i], v[th][i], acc);
+    acc += __shfl_xor_sync(kFull, acc, 1);
+    acc += __shfl_xor_sync(kFull, acc, 2);
+    ss[th] = acc * (1.0f / 128.0f);
+  }
+}
+
 // Shared memory of the prefill kernel, per CTA of W warps: W value-transpose
 // tiles (2 KB), W x 2 half-stages (16 staged K rows, 16 staged V rows, pf_pitch
-// bytes apart), W x 2 barriers. A half-stage is refilled with the next tile's
-// rows as soon as its rows have been read, so copies overlap the arithmetic.
+// bytes apart), the rotation B fragments of D_K and D_V (8 KB), W x 2 barriers.
+// A half-stage is refilled with the next tile's rows as soon as its rows have
+// been read, so copies overlap the arithmetic.
 __host__ __device__ constexpr int pf_pitch(int elem) { return 128 * elem + 32; }
+constexpr int kPfRotBytes = 2 * 8 * 32 * 16;
 __host__ __device__ constexpr size_t pf_smem(int warps, int elem) {
-  return size_t(warps) * 2048 + size_t(warps) * 32 * pf_pitch(elem) + size_t(warps) * 2 * 8;
+  return size_t(warps) * 2048 + size_t(warps) * 32 * pf_pitch(elem) + kPfRotBytes + size_t(warps) * 2 * 8;
 }
 
 template <int BK, int BV>
@@ -583,12 +677,17 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
   const int g = lane >> 2, t = lane & 3;
   uint8_t* vt = smem + warp * 2048;                                          // value transpose tile
   uint8_t* stage0 = smem + W * 2048 + warp * 32 * pitch;                     // K rows, then V rows
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + W * 2048 + W * 32 * pitch) + warp * 2;
+  uint4* rot = reinterpret_cast<uint4*>(smem + W * 2048 + W * 32 * pitch);  // [kv][ks][lane]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + W * 2048 + W * 32 * pitch + kPfRotBytes) + warp * 2;
   if (lane == 0) {
     mbar_init(bar, 1);
     mbar_init(bar + 1, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (elem == 2)
+    for (int e = threadIdx.x; e < 2 * 8 * 32; e += blockDim.x)
+      rot[e] = pf_rot_frag(e < 256 ? T.signs_k : T.signs_v, (e >> 5) & 7, e & 31, dtype == TQ_BF16);
+  __syncthreads();
   uint32_t dmk = 0u, dmv = 0u;                  // rotation sign bits of the lane's coordinates
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
@@ -658,7 +757,13 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
       break;
     }
     float vv[2][32], ss[2];
-    pf_load(stage0 + kv * 16 * pitch, pitch, dtype, g, t, ok0, ok1, kv ? dmv : (BK == 8 ? 0u : dmk), vv, ss);
+    // 16-bit inputs are rotated on the tensor cores as they are read; fp32 inputs
+    // and q8_0 keys (not rotated) are read into registers
+    const bool mma_rot = elem == 2 && !(BK == 8 && kv == 0);
+    if (mma_rot)
+      pf_rotate16(stage0 + kv * 16 * pitch, pitch, dtype == TQ_BF16, g, t, rot + kv * 256, lane, vv, ss);
+    else
+      pf_load(stage0 + kv * 16 * pitch, pitch, dtype, g, t, ok0, ok1, kv ? dmv : (BK == 8 ? 0u : dmk), vv, ss);
     __syncwarp();                                  // the rows are read: refill with the next tile's
     if (next < n_tiles) stage_rows(next, kv);
     if (!good) continue;
@@ -705,7 +810,7 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
       }
       continue;
     }
-    pf_fwht(vv, lane);
+    if (!mma_rot) pf_fwht(vv, lane);
     if (kv == 0) {
     if constexpr (BK != 8) {
     // ---------------- keys: norm, codes, residual, z = S u, signs
@@ -890,12 +995,15 @@ __device__ __forceinline__ int warp_isum(int v) {
 }
 
 // ================================================================== decode
-// Warps per decode CTA: 16 when a CTA serves one group of 4 query heads in the
-// uniform split (the kernel then fits 128 registers), else 8; either way one CTA
-// per SM. The balanced split always takes 8 warps: its loop over segments needs
-// the registers that 16 warps do not leave.
+// Warps per decode CTA, one CTA per SM. Uniform split: 16 for one group of 4
+// query heads (the kernel then fits 128 registers), 12 for two groups (168
+// registers: a few spill, and the extra warps hide more latency than the spills
+// cost), 8 for three. The balanced split always takes 8 warps: its loop over
+// segments needs the registers that more warps do not leave.
 template <int NH, bool BAL = false>
-struct DecodeWarps { static constexpr int value = (NH == 1 && !BAL) ? 16 : 8; };
+struct DecodeWarps {
+  static constexpr int value = BAL ? 8 : NH == 1 ? 16 : NH == 2 ? 12 : 8;
+};
 // TMA stages per warp: six when they fit in 160 KB of shared memory, else four.
 constexpr int kAccPitch = 132;      // floats per accumulator column in the CTA merge
 
@@ -1943,21 +2051,17 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   // segments, de-rotate, store. kParts warps share a head slot, each taking every
   // kParts-th record; lane l holds coordinates 4l .. 4l + 3 (the layout of the
   // inverse rotation). Records come straight from L2 (ld.global.cg), all of a
-  // warp's loads in flight at once; the parts meet in shared memory.
+  // warp's loads in flight at once, in one pass: each part keeps its own running
+  // maximum, and the parts meet in shared memory with their maxima.
   constexpr int kParts = W >= kSlots ? W / kSlots : 1;
   const float* pbase = A.partial + static_cast<size_t>(sg.first_slot) * kSlots * kRec;
   const int n_rec = sg.n_segs;
-  float* s_v = reinterpret_cast<float*>(smem);           // [kParts][kSlots][kRec]
+  float* s_v = reinterpret_cast<float*>(smem);           // [kParts][kSlots][kRec]: sums, l, max
   for (int sl0 = 0; sl0 < kSlots; sl0 += (kParts > 1 ? kSlots : W)) {
     const int slot = sl0 + (kParts > 1 ? warp % kSlots : warp);
     const int prt = kParts > 1 ? warp / kSlots : 0;
     if (slot < kSlots && prt < kParts) {                  // warp-uniform
-      // the slot's largest maximum over all records (lane c reads record c)
-      float M = kNegBig;
-      for (int c = lane; c < n_rec; c += 32)
-        M = fmaxf(M, __ldcg(pbase + (static_cast<size_t>(c) * kSlots + slot) * kRec + 128));
-      M = warp_max(M);
-      float v[4] = {0.f, 0.f, 0.f, 0.f}, lt = 0.0f;
+      float M = kNegBig, v[4] = {0.f, 0.f, 0.f, 0.f}, lt = 0.0f;
       for (int c0 = prt; c0 < n_rec; c0 += 8 * kParts) {
         float4 x[8];
         float2 ml[8];
@@ -1967,6 +2071,16 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
           const float* rec = pbase + (static_cast<size_t>(c < n_rec ? c : prt) * kSlots + slot) * kRec;
           x[k] = __ldcg(reinterpret_cast<const float4*>(rec) + lane);
           ml[k] = __ldcg(reinterpret_cast<const float2*>(rec + 128));
+        }
+        float bm = M;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (c0 + k * kParts < n_rec) bm = fmaxf(bm, ml[k].x);
+        if (bm > M) {                                     // rescale what this part has so far
+          const float r = ex2(M - bm);
+          lt *= r;
+          v[0] *= r; v[1] *= r; v[2] *= r; v[3] *= r;
+          M = bm;
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -1978,19 +2092,25 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       }
       float* mine = s_v + (prt * kSlots + slot) * kRec;
       reinterpret_cast<float4*>(mine)[lane] = make_float4(v[0], v[1], v[2], v[3]);
-      if (lane == 0) mine[128] = lt;
+      if (lane == 0) {
+        mine[128] = lt;
+        mine[129] = M;
+      }
     }
   }
   __syncthreads();
   const float4 sv = __ldg(reinterpret_cast<const float4*>(tab_sv) + lane);
   for (int slot = warp; slot < A.group; slot += W) {
-    float v[4] = {0.f, 0.f, 0.f, 0.f}, lt = 0.0f;
+    float v[4] = {0.f, 0.f, 0.f, 0.f}, lt = 0.0f, M = kNegBig;
+#pragma unroll
+    for (int q = 0; q < kParts; ++q) M = fmaxf(M, s_v[(q * kSlots + slot) * kRec + 129]);
 #pragma unroll
     for (int q = 0; q < kParts; ++q) {
       const float* r = s_v + (q * kSlots + slot) * kRec;
       const float4 x = reinterpret_cast<const float4*>(r)[lane];
-      lt += r[128];
-      v[0] += x.x; v[1] += x.y; v[2] += x.z; v[3] += x.w;
+      const float f = ex2(r[129] - M);
+      lt = fmaf(r[128], f, lt);
+      v[0] = fmaf(x.x, f, v[0]); v[1] = fmaf(x.y, f, v[1]); v[2] = fmaf(x.z, f, v[2]); v[3] = fmaf(x.w, f, v[3]);
     }
     const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
 #pragma unroll
