@@ -396,7 +396,7 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   cudaError_t e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, device);
   if (e == cudaSuccess && c->sm_count <= 0) e = cudaErrorInvalidDevice;
   if (e == cudaSuccess) e = cudaMalloc(&c->d_signs, 2 * tq::kHeadDim * sizeof(float));
-  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 4 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
+  if (e == cudaSuccess) e = cudaMalloc(&c->d_sketch_t, 5 * tq::kQjlRows * tq::kHeadDim * sizeof(uint16_t));
   if (e == cudaSuccess) e = cudaMalloc(&c->d_err, sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(unsigned));
   if (e != cudaSuccess) {
@@ -408,6 +408,7 @@ tq_status tq_create(tq_ctx** out, int head_dim, int qjl_rows, int page_size, int
   c->tables.sketch_t = c->d_sketch_t;
   c->tables.sketch_m = c->d_sketch_t + tq::kQjlRows * tq::kHeadDim;
   c->tables.sketch_qb = c->d_sketch_t + 3 * tq::kQjlRows * tq::kHeadDim;
+  c->tables.sketch_umma = c->d_sketch_t + 4 * tq::kQjlRows * tq::kHeadDim;
   c->tables.err = c->d_err;
   *out = c;
   return TQ_OK;
@@ -430,7 +431,7 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
   if (tq_status st = check_device(ctx)) return st;
   const int d = tq::kHeadDim, m = tq::kQjlRows;
   std::vector<int8_t> sk(d), sv(d);
-  std::vector<uint16_t> s(m * d), st(4 * m * d);
+  std::vector<uint16_t> s(m * d), st(5 * m * d);
   tq_host_sign_vector(seed_k, d, sk.data());
   tq_host_sign_vector(seed_v, d, sv.data());
   tq_host_gaussian_sketch(seed_s, m, d, s.data());
@@ -467,6 +468,17 @@ tq_status tq_init_rotation(tq_ctx* ctx, uint64_t seed_k, uint64_t seed_v, uint64
             const int row = 32 * (nt >> 2) + 16 * ((nt >> 1) & 1) + 4 * (c >> 1) + 2 * (nt & 1) + (c & 1);
             qb[(((ks * (m / 8) + nt) * 32 + lane) * 2 + r) * 2 + h] = s[row * d + coord];
           }
+  // S as the B operand of the tensor-core prefill product (K-major, no swizzle):
+  // operand row n = 8 nt + c holds the sketch row of n-tile nt, column c above;
+  // coordinate k of row n at element 1024 (n >> 3) + 64 (k >> 3) + 8 (n & 7) + (k & 7),
+  // i.e. 8-row x 8-coordinate core matrices of 128 bytes, K-adjacent ones 128 bytes
+  // apart and 8-row groups 2048 bytes apart.
+  uint16_t* bu = st.data() + 4 * m * d;
+  for (int nt = 0; nt < m / 8; ++nt)
+    for (int c = 0; c < 8; ++c) {
+      const int row = 32 * (nt >> 2) + 16 * ((nt >> 1) & 1) + 4 * (c >> 1) + 2 * (nt & 1) + (c & 1);
+      for (int kk = 0; kk < d; ++kk) bu[1024 * nt + 64 * (kk >> 3) + 8 * c + (kk & 7)] = s[row * d + kk];
+    }
   std::vector<uint16_t> mhi(m * d), mlo(m * d);
   double rownorm = 0.0;
   for (int r = 0; r < m; ++r) {

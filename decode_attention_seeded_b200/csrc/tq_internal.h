@@ -33,6 +33,7 @@ struct Tables {
                                        //   fragments [2][8 w][8 ks][32 lane][4 reg][2]
   float m_rownorm = 0.0f;             // max over rows r of |M_r| (bounds |p_r| <= |M_r| |q|)
   const uint16_t* sketch_qb = nullptr;  // device fp16 bits of S as prefill B fragments [8 ks][16 nt][32 lane][2 reg][2]
+  const uint16_t* sketch_umma = nullptr;  // device fp16 bits of S as the prefill's tensor-core B operand (32 KB)
   unsigned* err = nullptr;            // device error word
   unsigned test_flags = 0;            // TQ_TEST_* bits (tq_set_test_flags)
 };

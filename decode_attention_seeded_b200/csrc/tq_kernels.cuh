@@ -401,6 +401,76 @@ __device__ __forceinline__ void tma_load_1d(void* dst, const void* src, unsigned
       : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ------------------------------------------------ 5th-generation tensor cores
+// Tensor memory (TMEM) is allocated per CTA in columns of 128 lanes x 32 bits; a
+// TMEM address holds the lane in bits 31-16 and the column in bits 15-0. Warp w
+// may only touch lanes 32 (w % 4) .. 32 (w % 4) + 31.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t cols) {   // one full warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(cols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {  // the allocating warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// 16 lanes x 8 columns, 8 times along the columns: register 4j + i of lane (g, t)
+// is (lane g + 8 (i >> 1), column 8j + 2t + (i & 1)) -- the m16n8 accumulator
+// order of mma.sync. The store waits for its completion.
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n"
+      "tcgen05.wait::st.sync.aligned;\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// The matching load; the registers are defined only after its completion wait.
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+// D (TMEM, fp32) (+)= A (TMEM, fp16, M x 16) B (shared memory, fp16, 16 x N); one thread.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every tensor-core operation this thread issued is complete.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// Shared-memory descriptor of a K-major operand without swizzle: 8-row x 16-byte
+// core matrices, K-adjacent ones `lbo` bytes apart, 8-row groups `sbo` apart.
+__device__ __forceinline__ uint64_t umma_desc_noswizzle(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
 // ===================================================================== prefill
 // Quantize a contiguous run of one sequence, one warp per (page, KV head) tile.
 //
@@ -652,6 +722,130 @@ __device__ __forceinline__ void pf_rotate16(const uint8_t* rows, int pitch, bool
   }
 }
 
+constexpr float kPfInvRootD = 0.08838834764831845f;   // 1 / sqrt(128)
+
+// Keys of one tile from the rotated coordinates vv (H D x, both tokens): norms
+// |k|, codes (packed into the lane's key words kw), the residual u = y - c^ in
+// the rotated unit domain with |u|^2, and u 2^10 as fp16 high and low parts in
+// the m16n8k16 A-fragment order of z = S u (tokens on the rows): ah[ks][r],
+// r = token half (r & 1), coordinate pair 4ks + 2 (r >> 1).
+template <int BK, typename TA>
+__device__ __forceinline__ void pf_key_residual(float (&vv)[2][32], const float (&ss)[2], const TA& thk,
+                                                const TA& cnk, uint32_t (&kw)[2][4], float (&nk)[2],
+                                                float (&uu)[2], uint32_t (&ah)[8][4], uint32_t (&al)[8][4]) {
+#pragma unroll
+  for (int th = 0; th < 2; ++th) {
+    kw[th][0] = kw[th][1] = kw[th][2] = kw[th][3] = 0u;
+    uu[th] = 0.0f;
+    nk[th] = sqrtf(ss[th]);
+    const float inv = nk[th] > 0.0f ? kPfInvRootD / nk[th] : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float y = vv[th][i] * inv;
+      float chat;
+      const int c = cell_of<BK>(y, thk, cnk, chat);
+      put_key_code<BK>(kw[th], i, static_cast<uint32_t>(c));
+      const float u = y - chat;
+      uu[th] = fmaf(u, u, uu[th]);
+      vv[th][i] = u * 1024.0f;                  // u 2^10: well inside the fp16 range
+    }
+    uu[th] += __shfl_xor_sync(kFull, uu[th], 1);
+    uu[th] += __shfl_xor_sync(kFull, uu[th], 2);
+  }
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int th = r & 1, i = 4 * ks + 2 * (r >> 1);
+      const float x0 = vv[th][i], x1 = vv[th][i + 1];
+      const __half2 hi = __floats2half2_rn(x0, x1);
+      const float2 hf = __half22float2(hi);
+      ah[ks][r] = *reinterpret_cast<const uint32_t*>(&hi);
+      al[ks][r] = pack_half2(x0 - hf.x, x1 - hf.y);
+    }
+}
+
+// Sign bits of one 8-row block nt of z = S u, in the m16n8 accumulator order
+// (z[r]: token half r >> 1, column 2t + (r & 1)), added to the lane's sign words.
+__device__ __forceinline__ void pf_sign_bits(uint32_t (&sw)[2], int nt, const float (&z)[4]) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int th = r >> 1, j = 2 * nt + (r & 1);          // lane-local sketch row
+    sw[th] |= (z[r] >= 0.0f ? 1u : 0u) << (8 * (j & 3) + (j >> 2));
+  }
+}
+
+// Store one tile's key words, sign words and the norms |k| and gamma = |k| |u|
+// (tokens g, g + 8 of the lane, where inside the run).
+template <int BK, int BV>
+__device__ __forceinline__ void pf_key_store(uint8_t* blk, int lane, int g, bool ok0, bool ok1,
+                                             const uint32_t (&kw)[2][4], const uint32_t (&sw)[2],
+                                             const float (&nk)[2], const float (&uu)[2]) {
+  uint32_t* kwd = reinterpret_cast<uint32_t*>(blk) + lane * 2 * BK;
+  uint32_t* swd = reinterpret_cast<uint32_t*>(blk + sec_scale(BK)) + lane * 2;
+#pragma unroll
+  for (int th = 0; th < 2; ++th) {
+    if (!(th ? ok1 : ok0)) continue;
+#pragma unroll
+    for (int w = 0; w < BK; ++w) kwd[th * BK + w] = kw[th][w];
+    swd[th] = sw[th];
+  }
+  if ((lane & 3) == 0) {
+    __half* nrm = reinterpret_cast<__half*>(blk + sec_norm(BK, BV));
+    const float gk0 = nk[0] * sqrtf(uu[0]), gk1 = nk[1] * sqrtf(uu[1]);
+    if (ok0) { nrm[2 * g] = __float2half_rn(nk[0]); nrm[16 + 2 * g] = __float2half_rn(gk0); }
+    if (ok1) { nrm[2 * g + 1] = __float2half_rn(nk[1]); nrm[16 + 2 * g + 1] = __float2half_rn(gk1); }
+  }
+}
+
+// Values of one tile from the rotated coordinates: norms, codes, transposed to
+// the value chunks (coordinates x 4 tokens) through the warp's 2 KB tile vt, and
+// stored (merged under the token mask at the ends of a run).
+template <int BK, int BV, typename TA>
+__device__ __forceinline__ void pf_values(const float (&vv)[2][32], const float (&ss)[2], const TA& thv,
+                                          const TA& cnv, uint8_t* vt, uint8_t* blk, int lane, int g, int t,
+                                          int tau0, int tau1, bool full, bool ok0, bool ok1) {
+  float nv[2];
+#pragma unroll
+  for (int th = 0; th < 2; ++th) nv[th] = sqrtf(ss[th]);
+  {
+    const float inv0 = nv[0] > 0.0f ? kPfInvRootD / nv[0] : 0.0f;
+    const float inv1 = nv[1] > 0.0f ? kPfInvRootD / nv[1] : 0.0f;
+    __syncwarp();                                            // the tile's previous readers are done
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float chat;
+      const int c0 = cell_of<BV>(vv[0][i] * inv0, thv, cnv, chat);
+      const int c1 = cell_of<BV>(vv[1][i] * inv1, thv, cnv, chat);
+      // tokens g, g + 8 sit at bytes 2g, 2g + 1 of the coordinate's 16-byte row
+      *reinterpret_cast<uint16_t*>(vt + pf_coord(i, t) * 16 + 2 * g) = static_cast<uint16_t>(c0 | (c1 << 8));
+    }
+    __syncwarp();
+  }
+  // value chunk of this lane: coordinates g + 8 hf + 16 mt, tokens 2t + e + 8 tg
+  uint32_t vw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, vm[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  const bool tv[4] = {2 * t >= tau0 && 2 * t < tau1, 2 * t + 8 >= tau0 && 2 * t + 8 < tau1,
+                      2 * t + 1 >= tau0 && 2 * t + 1 < tau1, 2 * t + 9 >= tau0 && 2 * t + 9 < tau1};
+  const uint32_t maskx = (tv[0] ? 0xFFu : 0u) | (tv[1] ? 0xFF00u : 0u) | (tv[2] ? 0xFF0000u : 0u) |
+                         (tv[3] ? 0xFF000000u : 0u);
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint32_t x = *reinterpret_cast<const uint32_t*>(vt + (g + 8 * hf + 16 * mt) * 16 + 4 * t);
+      put_value_codes<BV>(vw, mt, hf, x & maskx);
+      if (!full) put_value_codes<BV>(vm, mt, hf, maskx);
+    }
+  uint32_t* vwd = reinterpret_cast<uint32_t*>(blk + sec_v(BK)) + lane * 2 * BV;
+#pragma unroll
+  for (int w = 0; w < 2 * BV; ++w) vwd[w] = full ? vw[w] : ((vwd[w] & ~vm[w]) | vw[w]);
+  if (t == 0) {
+    __half* nrm = reinterpret_cast<__half*>(blk + sec_norm(BK, BV)) + vnorm_entry0(BK);
+    if (ok0) nrm[2 * g] = __float2half_rn(nv[0]);
+    if (ok1) nrm[2 * g + 1] = __float2half_rn(nv[1]);
+  }
+}
+
 // Shared memory of the prefill kernel, per CTA of W warps: W value-transpose
 // tiles (2 KB), W x 2 half-stages (16 staged K rows, 16 staged V rows, pf_pitch
 // bytes apart), the rotation B fragments of D_K and D_V (8 KB), W x 2 barriers.
@@ -703,7 +897,6 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
   const int first_page = start_pos / kPage;
   const int n_tiles = ((start_pos + n_tokens - 1) / kPage - first_page + 1) * n_kv;
   const int bb = T.block_bytes;
-  const float kInvRootD = 0.08838834764831845f;   // 1 / sqrt(128)
   const int stride = gridDim.x * W;
 
   // Stage the 16 rows of K (kv = 0) or V (kv = 1) of `tile`: lane tau copies token
@@ -812,126 +1005,292 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
     }
     if (!mma_rot) pf_fwht(vv, lane);
     if (kv == 0) {
-    if constexpr (BK != 8) {
-    // ---------------- keys: norm, codes, residual, z = S u, signs
-    float nk[2], uu[2] = {0.f, 0.f};
-    uint32_t kw[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-#pragma unroll
-    for (int th = 0; th < 2; ++th) {
-      nk[th] = sqrtf(ss[th]);
-      const float inv = nk[th] > 0.0f ? kInvRootD / nk[th] : 0.0f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float y = vv[th][i] * inv;
-        float chat;
-        const int c = cell_of<BK>(y, thk, cnk, chat);
-        put_key_code<BK>(kw[th], i, static_cast<uint32_t>(c));
-        const float u = y - chat;
-        uu[th] = fmaf(u, u, uu[th]);
-        vv[th][i] = u * 1024.0f;                  // u 2^10: well inside the fp16 range
-      }
-      uu[th] += __shfl_xor_sync(kFull, uu[th], 1);
-      uu[th] += __shfl_xor_sync(kFull, uu[th], 2);
-    }
-    // A fragments (fp16 high and low parts) of the residual tile
-    uint32_t ah[8][4], al[8][4];
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int th = r & 1, i = 4 * ks + 2 * (r >> 1);
-        const float x0 = vv[th][i], x1 = vv[th][i + 1];
-        const __half2 hi = __floats2half2_rn(x0, x1);
-        const float2 hf = __half22float2(hi);
-        ah[ks][r] = *reinterpret_cast<const uint32_t*>(&hi);
-        al[ks][r] = pack_half2(x0 - hf.x, x1 - hf.y);
-      }
-    uint32_t sw[2] = {0u, 0u};
+      if constexpr (BK != 8) {
+        // ---------------- keys: norm, codes, residual, z = S u, signs
+        float nk[2], uu[2];
+        uint32_t kw[2][4], sw[2] = {0u, 0u};
+        uint32_t ah[8][4], al[8][4];
+        pf_key_residual<BK>(vv, ss, thk, cnk, kw, nk, uu, ah, al);
 #pragma unroll 1
-    for (int nt = 0; nt < 16; nt += 2) {             // two independent accumulator chains
-      float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int nt = 0; nt < 16; nt += 2) {             // two independent accumulator chains
+          float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint2 b0 = __ldg(qb + (ks * 16 + nt) * 32 + lane), b1 = __ldg(qb + (ks * 16 + nt + 1) * 32 + lane);
-        mma_f16(z0, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], b0.x, b0.y);
-        mma_f16(z1, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], b1.x, b1.y);
-        mma_f16(z0, al[ks][0], al[ks][1], al[ks][2], al[ks][3], b0.x, b0.y);
-        mma_f16(z1, al[ks][0], al[ks][1], al[ks][2], al[ks][3], b1.x, b1.y);
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int th = r >> 1, j0 = 2 * nt + (r & 1), j1 = j0 + 2;   // lane-local sketch rows
-        sw[th] |= (z0[r] >= 0.0f ? 1u : 0u) << (8 * (j0 & 3) + (j0 >> 2));
-        sw[th] |= (z1[r] >= 0.0f ? 1u : 0u) << (8 * (j1 & 3) + (j1 >> 2));
-      }
-    }
-    {
-      uint32_t* kwd = reinterpret_cast<uint32_t*>(blk) + lane * 2 * BK;
-      uint32_t* swd = reinterpret_cast<uint32_t*>(blk + sec_scale(BK)) + lane * 2;
-#pragma unroll
-      for (int th = 0; th < 2; ++th) {
-        if (!(th ? ok1 : ok0)) continue;
-#pragma unroll
-        for (int w = 0; w < BK; ++w) kwd[th * BK + w] = kw[th][w];
-        swd[th] = sw[th];
-      }
-      if (t == 0) {
-        __half* nrm = reinterpret_cast<__half*>(blk + sec_norm(BK, BV));
-        const float gk0 = nk[0] * sqrtf(uu[0]), gk1 = nk[1] * sqrtf(uu[1]);
-        if (ok0) { nrm[2 * g] = __float2half_rn(nk[0]); nrm[16 + 2 * g] = __float2half_rn(gk0); }
-        if (ok1) { nrm[2 * g + 1] = __float2half_rn(nk[1]); nrm[16 + 2 * g + 1] = __float2half_rn(gk1); }
-      }
-    }
-
-    }
-    } else {
-    // ---------------- values: norm, codes, transpose to value chunks
-    float nv[2];
-#pragma unroll
-    for (int th = 0; th < 2; ++th) nv[th] = sqrtf(ss[th]);
-    {
-      const float inv0 = nv[0] > 0.0f ? kInvRootD / nv[0] : 0.0f;
-      const float inv1 = nv[1] > 0.0f ? kInvRootD / nv[1] : 0.0f;
-      __syncwarp();                                            // the tile's previous readers are done
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float chat;
-        const int c0 = cell_of<BV>(vv[0][i] * inv0, thv, cnv, chat);
-        const int c1 = cell_of<BV>(vv[1][i] * inv1, thv, cnv, chat);
-        // tokens g, g + 8 sit at bytes 2g, 2g + 1 of the coordinate's 16-byte row
-        *reinterpret_cast<uint16_t*>(vt + pf_coord(i, t) * 16 + 2 * g) =
-            static_cast<uint16_t>(c0 | (c1 << 8));
-      }
-      __syncwarp();
-    }
-    {
-      // value chunk of this lane: coordinates g + 8 hf + 16 mt, tokens 2t + e + 8 tg
-      uint32_t vw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, vm[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-      const bool tv[4] = {2 * t >= tau0 && 2 * t < tau1, 2 * t + 8 >= tau0 && 2 * t + 8 < tau1,
-                          2 * t + 1 >= tau0 && 2 * t + 1 < tau1, 2 * t + 9 >= tau0 && 2 * t + 9 < tau1};
-      const uint32_t maskx = (tv[0] ? 0xFFu : 0u) | (tv[1] ? 0xFF00u : 0u) | (tv[2] ? 0xFF0000u : 0u) |
-                             (tv[3] ? 0xFF000000u : 0u);
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t x = *reinterpret_cast<const uint32_t*>(vt + (g + 8 * hf + 16 * mt) * 16 + 4 * t);
-          put_value_codes<BV>(vw, mt, hf, x & maskx);
-          if (!full) put_value_codes<BV>(vm, mt, hf, maskx);
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint2 b0 = __ldg(qb + (ks * 16 + nt) * 32 + lane), b1 = __ldg(qb + (ks * 16 + nt + 1) * 32 + lane);
+            mma_f16(z0, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], b0.x, b0.y);
+            mma_f16(z1, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], b1.x, b1.y);
+            mma_f16(z0, al[ks][0], al[ks][1], al[ks][2], al[ks][3], b0.x, b0.y);
+            mma_f16(z1, al[ks][0], al[ks][1], al[ks][2], al[ks][3], b1.x, b1.y);
+          }
+          pf_sign_bits(sw, nt, z0);
+          pf_sign_bits(sw, nt + 1, z1);
         }
-      uint32_t* vwd = reinterpret_cast<uint32_t*>(blk + sec_v(BK)) + lane * 2 * BV;
-#pragma unroll
-      for (int w = 0; w < 2 * BV; ++w) vwd[w] = full ? vw[w] : ((vwd[w] & ~vm[w]) | vw[w]);
-      if (t == 0) {
-        __half* nrm = reinterpret_cast<__half*>(blk + sec_norm(BK, BV)) + vnorm_entry0(BK);
-        if (ok0) nrm[2 * g] = __float2half_rn(nv[0]);
-        if (ok1) nrm[2 * g + 1] = __float2half_rn(nv[1]);
+        pf_key_store<BK, BV>(blk, lane, g, ok0, ok1, kw, sw, nk, uu);
       }
-    }
+    } else {
+      pf_values<BK, BV>(vv, ss, thv, cnv, vt, blk, lane, g, t, tau0, tau1, full, ok0, ok1);
     }
     }
   }
   __syncwarp();
+  if (lane == 0) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar + 1)) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------------
+// Prefill with z = S u on the 5th-generation tensor cores (16-bit K/V inputs,
+// TurboQuant keys). One CTA of 16 warps per SM; each half of the CTA (8 warps)
+// quantizes 8 tiles at a time, one per warp, and forms the sketch product of
+// their 128 tokens in one 128 x 128 x 128 tensor-core pass:
+//   - each warp writes its 16 residual rows (u 2^10 as fp16 high and low parts)
+//     to its lanes of the group's A tiles in tensor memory and arrives on the
+//     group's barrier;
+//   - one thread issues 2 x 8 MMAs (K = 16 each; high parts, then low parts into
+//     the same fp32 accumulators) with S in shared memory as the B operand, and
+//     commits them to the group's product barrier;
+//   - meanwhile the warps quantize their tiles' values; then each reads its 16
+//     rows of z back and packs the sign bits.
+// Tensor-memory rows: warp w owns lanes 32 (w % 4) + 16 ((w / 4) % 2) + 0..15.
+// Columns of group c: A high parts 256c + 0..63, low parts + 64..127 (two fp16
+// coordinates per column, natural order), accumulators + 128..255 (column n =
+// the B operand's row n, arranged so that column block nt holds the sketch rows
+// of the mma.sync n-tile nt, whose sign-packing order is kept).
+// S (fp16, 32 KB) is one bulk copy of Tables::sketch_umma: row n = 8 nt + c,
+// coordinate k at byte 2048 (n >> 3) + 128 (k >> 3) + 16 (n & 7) + 2 (k & 7).
+constexpr int kTcWarps = 16;
+constexpr int kTcStageBytes = 32 * pf_pitch(2);
+constexpr size_t kTcOffRot = 32768;
+constexpr size_t kTcOffVt = kTcOffRot + kPfRotBytes;
+constexpr size_t kTcOffStage = kTcOffVt + kTcWarps * 2048;
+constexpr size_t kTcOffBar = kTcOffStage + size_t(kTcWarps) * kTcStageBytes;
+constexpr int kTcBars = 2 * kTcWarps + 1 + 2 + 2;          // staging, S copy, A ready x 2, z ready x 2
+constexpr size_t kTcSmem = kTcOffBar + kTcBars * 8 + 16;
+constexpr uint32_t kTcCols = 512;
+
+template <int BK, int BV>
+__global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
+    Tables T, const void* k, const void* v, int dtype, int n_tokens, int n_kv, const int32_t* block_table,
+    int start_pos, uint8_t* cache, int64_t n_pages) {
+  static_assert(BK >= 2 && BK <= 4, "TurboQuant keys only");
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int W = kTcWarps;
+  const int pitch = pf_pitch(2), rb = 256;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int grp = warp >> 3, wg = warp & 7;
+  uint8_t* sk = smem;                                            // S, tensor-core B layout
+  uint4* rot = reinterpret_cast<uint4*>(smem + kTcOffRot);       // rotation B fragments [kv][ks][lane]
+  uint8_t* vt = smem + kTcOffVt + warp * 2048;
+  uint8_t* stage0 = smem + kTcOffStage + warp * kTcStageBytes;   // K rows, then V rows
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTcOffBar);
+  uint64_t* bar = bars + 2 * warp;                               // this warp's K and V rows landed
+  uint64_t* bar_sk = bars + 2 * W;                               // S landed
+  uint64_t* bar_a = bars + 2 * W + 1 + grp;                      // the group's A rows are written
+  uint64_t* bar_z = bars + 2 * W + 3 + grp;                      // the group's products are complete
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kTcBars);
+  __shared__ int s_abort;
+
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar_sk, 1);
+    for (int c = 0; c < 2; ++c) {
+      mbar_init(bars + 2 * W + 1 + c, 8);
+      mbar_init(bars + 2 * W + 3 + c, 1);
+    }
+    s_abort = 0;
+  }
+  if (lane == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  for (int e = threadIdx.x; e < 2 * 8 * 32; e += blockDim.x)
+    rot[e] = pf_rot_frag(e < 256 ? T.signs_k : T.signs_v, (e >> 5) & 7, e & 31, dtype == TQ_BF16);
+  if (warp == 0) tmem_alloc(s_tmem, kTcCols);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *s_tmem;
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(bar_sk, 32768u);
+    tma_load_1d(sk, T.sketch_umma, 32768u, bar_sk);
+  }
+  float thk[16], cnk[16], thv[16], cnv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    thk[i] = T.thr_k[i]; cnk[i] = T.cen_k[i]; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
+  }
+  const bool bf16 = dtype == TQ_BF16;
+  const int first_page = start_pos / kPage;
+  const int n_tiles = ((start_pos + n_tokens - 1) / kPage - first_page + 1) * n_kv;
+  const int bb = T.block_bytes;
+  const int gstride = gridDim.x * 2 * 8;                       // tiles per round over the grid
+
+  auto stage_rows = [&](int tile, int kv) {
+    const int lp = first_page + tile / n_kv, h = tile % n_kv;
+    const int phys = block_table[lp];
+    const bool good = phys >= 0 && phys < n_pages;
+    const int tau0 = max(start_pos - lp * kPage, 0), tau1 = min(start_pos + n_tokens - lp * kPage, kPage);
+    if (lane == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");    // earlier reads of these rows
+      mbar_expect_tx(bar + kv, good ? static_cast<unsigned>((tau1 - tau0) * rb) : 0u);
+    }
+    __syncwarp();
+    if (good && lane >= tau0 && lane < tau1) {
+      const int64_t row = static_cast<int64_t>(lp * kPage + lane - start_pos) * n_kv + h;
+      const uint8_t* src = static_cast<const uint8_t*>(kv ? v : k) + row * rb;
+      tma_load_1d(stage0 + (kv * 16 + lane) * pitch, src, rb, bar + kv);
+    }
+  };
+
+  const uint32_t lanes = static_cast<uint32_t>(32 * (warp & 3) + 16 * ((warp >> 2) & 1)) << 16;
+  const uint32_t col0 = 256u * grp;
+  // f32 accumulators, f16 A and B, both K-major, N = 128 (bits 17-22: N / 8), M = 128 (bits 24-28: M / 16)
+  constexpr uint32_t kIdesc = (1u << 4) | (16u << 17) | (8u << 24);
+  const uint32_t sk_addr = smem_u32(sk);
+
+  int tile = (blockIdx.x * 2 + grp) * 8 + wg;
+  if (tile < n_tiles) {
+    stage_rows(tile, 0);
+    stage_rows(tile, 1);
+  }
+  // staging barriers: phase of the next wait, and whether a copy is in flight
+  unsigned kph = 0, vph = 0;
+  bool kpend = tile < n_tiles, vpend = tile < n_tiles;
+  bool dead = false;               // a staging wait ran out: no more copies, no more work
+  auto aborted = [&]() { return __any_sync(kFull, *reinterpret_cast<volatile int*>(&s_abort) != 0); };
+  for (int r = 0;; ++r, tile += gstride) {
+    if (tile - wg >= n_tiles) break;                              // the group is done (group-uniform)
+    if (aborted()) break;
+    const int next = tile + gstride;
+    bool work = tile < n_tiles && !dead;
+    int lp = 0, h = 0, tau0 = 0, tau1 = 0;
+    bool good = false;
+    if (work) {
+      lp = first_page + tile / n_kv;
+      h = tile % n_kv;
+      const int phys = block_table[lp];
+      good = phys >= 0 && phys < n_pages;
+      if (!good && lane == 0) set_error(T.err, TQ_DEV_BAD_SLOT);
+      tau0 = max(start_pos - lp * kPage, 0);
+      tau1 = min(start_pos + n_tokens - lp * kPage, kPage);
+    }
+    uint8_t* blk = cache + (static_cast<int64_t>(good ? block_table[lp] : 0) * n_kv + h) * bb;
+    const bool full = tau0 == 0 && tau1 == kPage;
+    const bool ok0 = g >= tau0 && g < tau1, ok1 = g + 8 >= tau0 && g + 8 < tau1;
+
+    // ---- keys: rotation, codes, residual rows into tensor memory
+    float nk[2] = {0.f, 0.f}, uu[2] = {0.f, 0.f};
+    uint32_t kw[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+    if (work && !__all_sync(kFull, mbar_wait(bar, kph))) {
+      if (lane == 0) set_error(T.err, TQ_DEV_TIMEOUT);
+      dead = true;
+      work = false;
+    }
+    if (work) {
+      kpend = false;
+      kph ^= 1u;
+      float vv[2][32], ss[2];
+      pf_rotate16(stage0, pitch, bf16, g, t, rot, lane, vv, ss);
+      __syncwarp();                                               // the K rows are read
+      if (next < n_tiles) {
+        stage_rows(next, 0);
+        kpend = true;
+      }
+      uint32_t ah[8][4], al[8][4];
+      pf_key_residual<BK>(vv, ss, thk, cnk, kw, nk, uu, ah, al);
+      uint32_t ra[32];
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        ra[4 * ks + 0] = ah[ks][0]; ra[4 * ks + 1] = ah[ks][2]; ra[4 * ks + 2] = ah[ks][1]; ra[4 * ks + 3] = ah[ks][3];
+      }
+      tmem_st_16x256b_x8(tmem + lanes + col0, ra);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        ra[4 * ks + 0] = al[ks][0]; ra[4 * ks + 1] = al[ks][2]; ra[4 * ks + 2] = al[ks][1]; ra[4 * ks + 3] = al[ks][3];
+      }
+      tmem_st_16x256b_x8(tmem + lanes + col0 + 64, ra);
+    }
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_a);
+
+    // ---- one thread of the group: z = S u for the group's 128 rows
+    if (wg == 0 && lane == 0) {
+      const bool ready = (r > 0 || mbar_wait(bar_sk, 0)) && mbar_wait(bar_a, r & 1);
+      if (ready) {
+        tc_fence_after_sync();
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            umma_f16_ts(tmem + col0 + 128, tmem + col0 + 64 * hl + 8 * ks,
+                        umma_desc_noswizzle(sk_addr + 256 * ks, 128, 2048), kIdesc, (hl | ks) ? 1u : 0u);
+        umma_commit(bar_z);
+      } else {
+        set_error(T.err, TQ_DEV_TIMEOUT);
+        s_abort = 1;
+        mbar_arrive(bar_z);                                       // release the group; nothing is read
+      }
+    }
+
+    // ---- values, while the product runs
+    if (work && !__all_sync(kFull, mbar_wait(bar + 1, vph))) {
+      if (lane == 0) set_error(T.err, TQ_DEV_TIMEOUT);
+      dead = true;
+      work = false;
+    }
+    if (work) {
+      vpend = false;
+      vph ^= 1u;
+      float vv[2][32], ss[2];
+      pf_rotate16(stage0 + 16 * pitch, pitch, bf16, g, t, rot + 256, lane, vv, ss);
+      __syncwarp();                                               // the V rows are read
+      if (next < n_tiles) {
+        stage_rows(next, 1);
+        vpend = true;
+      }
+      if (good) pf_values<BK, BV>(vv, ss, thv, cnv, vt, blk, lane, g, t, tau0, tau1, full, ok0, ok1);
+    }
+
+    // ---- this warp's rows of z: sign bits, then the key words
+    if (!__all_sync(kFull, mbar_wait(bar_z, r & 1))) {
+      if (lane == 0) {
+        set_error(T.err, TQ_DEV_TIMEOUT);
+        s_abort = 1;
+      }
+      break;
+    }
+    tc_fence_after_sync();
+    if (aborted()) break;
+    if (work && good) {
+      uint32_t sw[2] = {0u, 0u};
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t zr[32];
+        tmem_ld_16x256b_x8(tmem + lanes + col0 + 128 + 64 * hf, zr);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float z[4] = {__uint_as_float(zr[4 * j]), __uint_as_float(zr[4 * j + 1]),
+                              __uint_as_float(zr[4 * j + 2]), __uint_as_float(zr[4 * j + 3])};
+          pf_sign_bits(sw, 8 * hf + j, z);
+        }
+      }
+      pf_key_store<BK, BV>(blk, lane, g, ok0, ok1, kw, sw, nk, uu);
+    }
+    tc_fence_before_sync();
+  }
+  // bounded: let this warp's copies still in flight (after a wait ran out or an
+  // abort) land before the CTA exits
+  if (kpend) mbar_wait(bar, kph);
+  if (vpend) mbar_wait(bar + 1, vph);
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTcCols);
+  }
   if (lane == 0) {
     asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
     asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar + 1)) : "memory");
@@ -2339,6 +2698,25 @@ cudaError_t launch_prefill_t(const Tables& t, const void* k, const void* v, int 
   const int first = start_pos / kPage, last = (start_pos + n_tokens - 1) / kPage;
   const int tiles = (last - first + 1) * n_kv;
   const int elem = dtype == TQ_F32 ? 4 : 2;
+  if constexpr (BK != 8) {
+    if (elem == 2) {                      // TurboQuant keys from 16-bit inputs: z = S u on tcgen05
+      auto fn = quantize_prefill_tc_kernel<BK, BV>;
+      static int max_blocks = 0;
+      if (max_blocks == 0) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kTcSmem));
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        max_blocks = sms;                 // one CTA per SM (its shared memory and all tensor memory)
+      }
+      int blocks = (tiles + kTcWarps - 1) / kTcWarps;
+      if (blocks > max_blocks) blocks = max_blocks;
+      fn<<<blocks, kTcWarps * 32, kTcSmem, s>>>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos,
+                                                static_cast<uint8_t*>(cache), n_pages);
+      return cudaGetLastError();
+    }
+  }
   const int warps = 8;
   int blocks = (tiles + warps - 1) / warps;
   const size_t smem = pf_smem(warps, elem);

@@ -59,7 +59,8 @@ def _t(x, dtype):
 # ----------------------------------------------------------------- quantize
 @pytest.mark.parametrize("bk,bv,dtype,path", [(3, 3, "fp32", "prefill"), (3, 2, "bf16", "append"),
                                               (4, 4, "bf16", "prefill"), (2, 4, "fp16", "append"),
-                                              (4, 2, "bf16", "append"), (2, 3, "bf16", "prefill")])
+                                              (4, 2, "bf16", "append"), (2, 3, "bf16", "prefill"),
+                                              (3, 4, "fp16", "prefill")])
 def test_quantize_matches_oracle(bk, bv, dtype, path):
     seeds = (11 + bk, 22 + bv, 33)
     ctx = _ctx(bk, bv, seeds)
