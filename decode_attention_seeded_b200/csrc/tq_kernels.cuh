@@ -729,28 +729,31 @@ constexpr float kPfInvRootD = 0.08838834764831845f;   // 1 / sqrt(128)
 // the rotated unit domain with |u|^2, and u 2^10 as fp16 high and low parts in
 // the m16n8k16 A-fragment order of z = S u (tokens on the rows): ah[ks][r],
 // r = token half (r & 1), coordinate pair 4ks + 2 (r >> 1).
+// cnk10: the key centroids times 2^10, so that u 2^10 = y 2^10 - c^ 2^10 is one
+// fused operation with a single rounding (the same value as (y - c^) 2^10).
 template <int BK, typename TA>
 __device__ __forceinline__ void pf_key_residual(float (&vv)[2][32], const float (&ss)[2], const TA& thk,
-                                                const TA& cnk, uint32_t (&kw)[2][4], float (&nk)[2],
+                                                const TA& cnk10, uint32_t (&kw)[2][4], float (&nk)[2],
                                                 float (&uu)[2], uint32_t (&ah)[8][4], uint32_t (&al)[8][4]) {
 #pragma unroll
   for (int th = 0; th < 2; ++th) {
     kw[th][0] = kw[th][1] = kw[th][2] = kw[th][3] = 0u;
-    uu[th] = 0.0f;
+    float u2 = 0.0f;
     nk[th] = sqrtf(ss[th]);
     const float inv = nk[th] > 0.0f ? kPfInvRootD / nk[th] : 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float y = vv[th][i] * inv;
-      float chat;
-      const int c = cell_of<BK>(y, thk, cnk, chat);
+      float chat10;
+      const int c = cell_of<BK>(y, thk, cnk10, chat10);
       put_key_code<BK>(kw[th], i, static_cast<uint32_t>(c));
-      const float u = y - chat;
-      uu[th] = fmaf(u, u, uu[th]);
-      vv[th][i] = u * 1024.0f;                  // u 2^10: well inside the fp16 range
+      const float u10 = fmaf(y, 1024.0f, -chat10);  // u 2^10: well inside the fp16 range
+      u2 = fmaf(u10, u10, u2);
+      vv[th][i] = u10;
     }
-    uu[th] += __shfl_xor_sync(kFull, uu[th], 1);
-    uu[th] += __shfl_xor_sync(kFull, uu[th], 2);
+    u2 += __shfl_xor_sync(kFull, u2, 1);
+    u2 += __shfl_xor_sync(kFull, u2, 2);
+    uu[th] = u2 * 9.5367431640625e-07f;               // 2^-20: |u|^2
   }
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks)
@@ -888,10 +891,10 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
     dmk |= (T.signs_k[pf_coord(i, t)] < 0.0f ? 1u : 0u) << i;
     dmv |= (T.signs_v[pf_coord(i, t)] < 0.0f ? 1u : 0u) << i;
   }
-  float thk[16], cnk[16], thv[16], cnv[16];
+  float thk[16], cnk10[16], thv[16], cnv[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    thk[i] = T.thr_k[i]; cnk[i] = T.cen_k[i]; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
+    thk[i] = T.thr_k[i]; cnk10[i] = T.cen_k[i] * 1024.0f; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
   }
   __syncwarp();
   const int first_page = start_pos / kPage;
@@ -1010,7 +1013,7 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
         float nk[2], uu[2];
         uint32_t kw[2][4], sw[2] = {0u, 0u};
         uint32_t ah[8][4], al[8][4];
-        pf_key_residual<BK>(vv, ss, thk, cnk, kw, nk, uu, ah, al);
+        pf_key_residual<BK>(vv, ss, thk, cnk10, kw, nk, uu, ah, al);
 #pragma unroll 1
         for (int nt = 0; nt < 16; nt += 2) {             // two independent accumulator chains
           float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1116,10 +1119,10 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
     mbar_expect_tx(bar_sk, 32768u);
     tma_load_1d(sk, T.sketch_umma, 32768u, bar_sk);
   }
-  float thk[16], cnk[16], thv[16], cnv[16];
+  float thk[16], cnk10[16], thv[16], cnv[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    thk[i] = T.thr_k[i]; cnk[i] = T.cen_k[i]; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
+    thk[i] = T.thr_k[i]; cnk10[i] = T.cen_k[i] * 1024.0f; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
   }
   const bool bf16 = dtype == TQ_BF16;
   const int first_page = start_pos / kPage;
@@ -1199,7 +1202,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
         kpend = true;
       }
       uint32_t ah[8][4], al[8][4];
-      pf_key_residual<BK>(vv, ss, thk, cnk, kw, nk, uu, ah, al);
+      pf_key_residual<BK>(vv, ss, thk, cnk10, kw, nk, uu, ah, al);
       uint32_t ra[32];
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
@@ -1356,12 +1359,11 @@ __device__ __forceinline__ int warp_isum(int v) {
 // ================================================================== decode
 // Warps per decode CTA, one CTA per SM. Uniform split: 16 for one group of 4
 // query heads (the kernel then fits 128 registers), 12 for two groups (168
-// registers: a few spill, and the extra warps hide more latency than the spills
-// cost), 8 for three. The balanced split always takes 8 warps: its loop over
-// segments needs the registers that more warps do not leave.
+// registers), 8 for three. The balanced split, whose loop over segments needs
+// more registers: 12 for one group, 8 for more.
 template <int NH, bool BAL = false>
 struct DecodeWarps {
-  static constexpr int value = BAL ? 8 : NH == 1 ? 16 : NH == 2 ? 12 : 8;
+  static constexpr int value = BAL ? (NH == 1 ? 12 : 8) : NH == 1 ? 16 : NH == 2 ? 12 : 8;
 };
 // TMA stages per warp: six when they fit in 160 KB of shared memory, else four.
 constexpr int kAccPitch = 132;      // floats per accumulator column in the CTA merge
@@ -2276,9 +2278,12 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   };
 
   while (inflight > 0) {
-    // Two pages per iteration while two are in flight: their key work is
-    // independent and interleaves; the softmax reduction is shared.
-    const int npg = inflight >= 2 ? 2 : 1;
+    // Two pages per iteration while two are in flight (one group of 4 query
+    // heads, uniform split): their key work is independent and interleaves, and
+    // the softmax reduction is shared. With more head groups the second page's
+    // registers would spill, and the balanced split spends them on more warps;
+    // one page at a time is faster there.
+    const int npg = (NH == 1 && !LOOP && inflight >= 2) ? 2 : 1;
     const int s2 = s + 1 == S ? 0 : s + 1;
     const unsigned parity2 = s + 1 == S ? parity ^ 1u : parity;
     // warp-uniform outcome: the page body runs warp-wide shuffles and mma.sync
@@ -2487,7 +2492,7 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
 
 // The decode launch.
 // Uniform mode: CTA i serves chunk i / n_pairs of pair i % n_pairs (chunks of ppc pages).
-// Balanced mode (always 8 warps): the pairs' pages are laid end to end, each
+// Balanced mode (12 or 8 warps, see DecodeWarps): the pairs' pages are laid end to end, each
 // non-empty pair preceded by seg_w "virtual" pages standing for its fixed cost
 // (prologue, merge), and the line is cut into G equal shares, one per CTA (share of
 // position y: ceil((y + 1) G / N) - 1). A CTA serves one segment per pair its share
