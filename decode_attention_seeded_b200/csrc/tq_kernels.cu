@@ -163,6 +163,31 @@ cudaError_t launch_logits(const Tables& t, const DecodePlan& plan, const void* q
   return dispatch_bits(t, a, dim3(plan.grid), s, 2);
 }
 
+cudaError_t encode_kv_tensor_map(CUtensorMap* map, const void* base, int dtype, int n_tokens, int n_kv) {
+  using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static const Encode encode = []() -> Encode {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<Encode>(fn);
+  }();
+  if (!encode) return cudaErrorNotSupported;
+  if (n_tokens < 1 || n_kv < 1 || (reinterpret_cast<uintptr_t>(base) & 15u)) return cudaErrorInvalidValue;
+  const cuuint64_t dims[4] = {64, 2, static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(n_tokens)};
+  const cuuint64_t strides[3] = {128, 256, 256ull * static_cast<cuuint64_t>(n_kv)};   // bytes, dims 1..3
+  const cuuint32_t box[4] = {64, 2, 1, 16};
+  const cuuint32_t step[4] = {1, 1, 1, 1};
+  const CUresult r = encode(map, dtype == TQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                            4, const_cast<void*>(base), dims, strides, box, step, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_decode_step(const Tables& t, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, const void* q, int q_dtype, void* cache, int64_t n_pages,
                                const int32_t* block_tables, int max_pages_per_seq, const int32_t* seq_lens,

@@ -7,12 +7,19 @@
 #include "tq.h"
 #include "tq_internal.h"
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstddef>
 #include <cstdint>
 
 namespace tq {
+
+// Tensor map of a run of 16-bit K or V rows [n_tokens][n_kv][128] for the prefill's
+// tile loads: four dimensions (64 coordinates, 2 halves, n_kv heads, n_tokens),
+// box 64 x 2 x 1 x 16 (one 16-token tile of one head), 128-byte swizzle, zero fill
+// outside the run (tq_kernels.cu).
+cudaError_t encode_kv_tensor_map(CUtensorMap* map, const void* base, int dtype, int n_tokens, int n_kv);
 
 struct DecodeArgs {
   const void* q;                 // [batch][n_q][128]
@@ -471,6 +478,17 @@ __device__ __forceinline__ uint64_t umma_desc_noswizzle(uint32_t saddr, uint32_t
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+// Tiled tensor copy of one box into shared memory (this GPU's memory, no
+// multicast); the box's bytes complete the transaction count on `bar`.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ===================================================================== prefill
 // Quantize a contiguous run of one sequence, one warp per (page, KV head) tile.
 //
@@ -849,6 +867,52 @@ __device__ __forceinline__ void pf_values(const float (&vv)[2][32], const float 
   }
 }
 
+// pf_rotate16 on a tile loaded by the tensor map above: 16 tokens x 2 halves of
+// 128-byte lines (line l = 2 token + half), 16-byte chunk c of line l stored at
+// chunk c ^ (l % 8) (the 128-byte swizzle; the tile is 1024-byte aligned). Tokens
+// g and g + 8 are 16 lines apart, so both use the same chunk permutation, and the
+// eight rows a quarter-warp reads fall in distinct chunks.
+__device__ __forceinline__ void pf_rotate16_sw(const uint8_t* tile, bool bf16, int g, int t, const uint4* frag,
+                                               int lane, float (&v)[2][32], float (&ss)[2]) {
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int half = ks >> 2, l0 = 2 * g + half;
+    const int chunk = (2 * (ks & 3) + (t >> 1)) ^ (l0 & 7);
+    const uint8_t* p = tile + l0 * 128 + chunk * 16 + 8 * (t & 1);
+    const uint2 x0 = *reinterpret_cast<const uint2*>(p);
+    const uint2 x1 = *reinterpret_cast<const uint2*>(p + 16 * 128);
+    const uint4 b = frag[ks * 32 + lane];
+    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+    if (bf16) {
+      mma_bf16(z0, x0.x, x1.x, x0.y, x1.y, b.x, b.y);
+      mma_bf16(z1, x0.x, x1.x, x0.y, x1.y, b.z, b.w);
+    } else {
+      mma_f16(z0, x0.x, x1.x, x0.y, x1.y, b.x, b.y);
+      mma_f16(z1, x0.x, x1.x, x0.y, x1.y, b.z, b.w);
+    }
+    v[0][4 * ks + 0] = z0[0]; v[0][4 * ks + 1] = z0[1]; v[1][4 * ks + 0] = z0[2]; v[1][4 * ks + 1] = z0[3];
+    v[0][4 * ks + 2] = z1[0]; v[0][4 * ks + 3] = z1[1]; v[1][4 * ks + 2] = z1[2]; v[1][4 * ks + 3] = z1[3];
+  }
+#pragma unroll
+  for (int th = 0; th < 2; ++th) {
+#pragma unroll
+    for (int bit = 2; bit < 5; ++bit)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (!(i & (1 << bit))) {
+          const float a = v[th][i], b = v[th][i | (1 << bit)];
+          v[th][i] = a + b;
+          v[th][i | (1 << bit)] = a - b;
+        }
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc = fmaf(v[th][i], v[th][i], acc);
+    acc += __shfl_xor_sync(kFull, acc, 1);
+    acc += __shfl_xor_sync(kFull, acc, 2);
+    ss[th] = acc * (1.0f / 128.0f);
+  }
+}
+
 // Shared memory of the prefill kernel, per CTA of W warps: W value-transpose
 // tiles (2 KB), W x 2 half-stages (16 staged K rows, 16 staged V rows, pf_pitch
 // bytes apart), the rotation B fragments of D_K and D_V (8 KB), W x 2 barriers.
@@ -1062,31 +1126,35 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
 // of the mma.sync n-tile nt, whose sign-packing order is kept).
 // S (fp16, 32 KB) is one bulk copy of Tables::sketch_umma: row n = 8 nt + c,
 // coordinate k at byte 2048 (n >> 3) + 128 (k >> 3) + 16 (n & 7) + 2 (k & 7).
+// Each warp's K and V tiles come in by one tensor copy each (encode_kv_tensor_map),
+// into 4 KB 128-byte-swizzled buffers read by pf_rotate16_sw; the next round's
+// tiles are requested as soon as a tile has been read.
 constexpr int kTcWarps = 16;
-constexpr int kTcStageBytes = 32 * pf_pitch(2);
-constexpr size_t kTcOffRot = 32768;
+constexpr int kTcTileBytes = 16 * 256;                      // one 16-token tile of K or V rows
+constexpr size_t kTcOffS = size_t(kTcWarps) * 2 * kTcTileBytes;   // after the (1024-aligned) stages
+constexpr size_t kTcOffRot = kTcOffS + 32768;
 constexpr size_t kTcOffVt = kTcOffRot + kPfRotBytes;
-constexpr size_t kTcOffStage = kTcOffVt + kTcWarps * 2048;
-constexpr size_t kTcOffBar = kTcOffStage + size_t(kTcWarps) * kTcStageBytes;
+constexpr size_t kTcOffBar = kTcOffVt + kTcWarps * 2048;
 constexpr int kTcBars = 2 * kTcWarps + 1 + 2 + 2;          // staging, S copy, A ready x 2, z ready x 2
-constexpr size_t kTcSmem = kTcOffBar + kTcBars * 8 + 16;
+constexpr size_t kTcSmem = 1024 + kTcOffBar + kTcBars * 8 + 16;   // + alignment of the stages
 constexpr uint32_t kTcCols = 512;
 
 template <int BK, int BV>
 __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
-    Tables T, const void* k, const void* v, int dtype, int n_tokens, int n_kv, const int32_t* block_table,
-    int start_pos, uint8_t* cache, int64_t n_pages) {
+    Tables T, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv, int dtype,
+    int n_tokens, int n_kv, const int32_t* block_table, int start_pos, uint8_t* cache, int64_t n_pages) {
   static_assert(BK >= 2 && BK <= 4, "TurboQuant keys only");
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   constexpr int W = kTcWarps;
-  const int pitch = pf_pitch(2), rb = 256;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int grp = warp >> 3, wg = warp & 7;
-  uint8_t* sk = smem;                                            // S, tensor-core B layout
+  // the swizzled tiles need 1024-byte alignment
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stage0 = smem + warp * 2 * kTcTileBytes;              // K tile, then V tile
+  uint8_t* sk = smem + kTcOffS;                                  // S, tensor-core B layout
   uint4* rot = reinterpret_cast<uint4*>(smem + kTcOffRot);       // rotation B fragments [kv][ks][lane]
   uint8_t* vt = smem + kTcOffVt + warp * 2048;
-  uint8_t* stage0 = smem + kTcOffStage + warp * kTcStageBytes;   // K rows, then V rows
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTcOffBar);
   uint64_t* bar = bars + 2 * warp;                               // this warp's K and V rows landed
   uint64_t* bar_sk = bars + 2 * W;                               // S landed
@@ -1130,21 +1198,18 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
   const int bb = T.block_bytes;
   const int gstride = gridDim.x * 2 * 8;                       // tiles per round over the grid
 
+  // Stage the K (kv = 0) or V (kv = 1) tile of `tile`: one tensor copy of the
+  // page's 16 tokens of head h (tokens outside the run read as zeros).
   auto stage_rows = [&](int tile, int kv) {
-    const int lp = first_page + tile / n_kv, h = tile % n_kv;
-    const int phys = block_table[lp];
-    const bool good = phys >= 0 && phys < n_pages;
-    const int tau0 = max(start_pos - lp * kPage, 0), tau1 = min(start_pos + n_tokens - lp * kPage, kPage);
     if (lane == 0) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");    // earlier reads of these rows
-      mbar_expect_tx(bar + kv, good ? static_cast<unsigned>((tau1 - tau0) * rb) : 0u);
+      const int lp = first_page + tile / n_kv, h = tile % n_kv;
+      const int phys = block_table[lp];
+      const bool good = phys >= 0 && phys < n_pages;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");    // earlier reads of this tile
+      mbar_expect_tx(bar + kv, good ? static_cast<unsigned>(kTcTileBytes) : 0u);
+      if (good) tma_load_4d(stage0 + kv * kTcTileBytes, kv ? &tmv : &tmk, 0, 0, h, lp * kPage - start_pos, bar + kv);
     }
     __syncwarp();
-    if (good && lane >= tau0 && lane < tau1) {
-      const int64_t row = static_cast<int64_t>(lp * kPage + lane - start_pos) * n_kv + h;
-      const uint8_t* src = static_cast<const uint8_t*>(kv ? v : k) + row * rb;
-      tma_load_1d(stage0 + (kv * 16 + lane) * pitch, src, rb, bar + kv);
-    }
   };
 
   const uint32_t lanes = static_cast<uint32_t>(32 * (warp & 3) + 16 * ((warp >> 2) & 1)) << 16;
@@ -1195,7 +1260,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
       kpend = false;
       kph ^= 1u;
       float vv[2][32], ss[2];
-      pf_rotate16(stage0, pitch, bf16, g, t, rot, lane, vv, ss);
+      pf_rotate16_sw(stage0, bf16, g, t, rot, lane, vv, ss);
       __syncwarp();                                               // the K rows are read
       if (next < n_tiles) {
         stage_rows(next, 0);
@@ -1248,7 +1313,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
       vpend = false;
       vph ^= 1u;
       float vv[2][32], ss[2];
-      pf_rotate16(stage0 + 16 * pitch, pitch, bf16, g, t, rot + 256, lane, vv, ss);
+      pf_rotate16_sw(stage0 + kTcTileBytes, bf16, g, t, rot + 256, lane, vv, ss);
       __syncwarp();                                               // the V rows are read
       if (next < n_tiles) {
         stage_rows(next, 1);
@@ -2717,7 +2782,11 @@ cudaError_t launch_prefill_t(const Tables& t, const void* k, const void* v, int 
       }
       int blocks = (tiles + kTcWarps - 1) / kTcWarps;
       if (blocks > max_blocks) blocks = max_blocks;
-      fn<<<blocks, kTcWarps * 32, kTcSmem, s>>>(t, k, v, dtype, n_tokens, n_kv, block_table, start_pos,
+      CUtensorMap tmk, tmv;
+      cudaError_t e = encode_kv_tensor_map(&tmk, k, dtype, n_tokens, n_kv);
+      if (e == cudaSuccess) e = encode_kv_tensor_map(&tmv, v, dtype, n_tokens, n_kv);
+      if (e != cudaSuccess) return e;
+      fn<<<blocks, kTcWarps * 32, kTcSmem, s>>>(t, tmk, tmv, dtype, n_tokens, n_kv, block_table, start_pos,
                                                 static_cast<uint8_t*>(cache), n_pages);
       return cudaGetLastError();
     }
