@@ -2401,18 +2401,20 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   if constexpr (LOGITS) return;                   // logits are written; nothing to merge
 
   // ---- merge the warps of this CTA
+  constexpr int kSlots = NH * kGroupHeads;
+  __shared__ float s_mx[W * kSlots];                    // each warp's running maxima (not in the stages)
 #pragma unroll
   for (int h = 0; h < NH; ++h) {                        // each head's denominator over its 8 lanes
     lsum[h] += __shfl_xor_sync(kFull, lsum[h], 4);
     lsum[h] += __shfl_xor_sync(kFull, lsum[h], 8);
     lsum[h] += __shfl_xor_sync(kFull, lsum[h], 16);
+    if (g == 0) s_mx[warp * kSlots + 4 * h + t] = mp2[h];
   }
   __syncthreads();                                      // every warp is out of its page loop: stages free
   // s_acc [W][kSlots][kAccPitch]: each warp's head sums (lanes t < 2 store the even
   // m-tiles, t >= 2 the odd ones: with a pitch of 132 floats one store touches 32
-  // banks); s_m, s_l, s_f [W][kSlots]: running maximum, denominator and the factor
-  // 2^(m_w - M) towards the CTA's maximum M (s_M [kSlots]).
-  constexpr int kSlots = NH * kGroupHeads;
+  // banks); s_l, s_f [W][kSlots]: denominator and the factor 2^(m_w - M) towards
+  // the CTA's maximum M (s_M [kSlots]); the maxima m_w are in s_mx.
   float* s_acc = reinterpret_cast<float*>(smem);
   float* s_m = s_acc + W * kSlots * kAccPitch;
   float* s_l = s_m + W * kSlots;
@@ -2432,18 +2434,14 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
         if ((mt & 1) == (t >> 1)) s_acc[(warp * kSlots + slot) * kAccPitch + coord] = sum;
       }
     }
-    if (g == 0) {
-      s_m[warp * kSlots + 4 * h + t] = mp2[h];
-      s_l[warp * kSlots + 4 * h + t] = lsum[h];
-    }
+    if (g == 0) s_l[warp * kSlots + 4 * h + t] = lsum[h];
   }
-  __syncthreads();
   if (threadIdx.x < W * kSlots) {                       // one thread per (warp, head slot)
     const int w = threadIdx.x / kSlots, slot = threadIdx.x % kSlots;
     float M = kNegBig;
 #pragma unroll
-    for (int v = 0; v < W; ++v) M = fmaxf(M, s_m[v * kSlots + slot]);
-    s_f[w * kSlots + slot] = ex2(s_m[w * kSlots + slot] - M);
+    for (int v = 0; v < W; ++v) M = fmaxf(M, s_mx[v * kSlots + slot]);
+    s_f[w * kSlots + slot] = ex2(s_mx[w * kSlots + slot] - M);
     if (w == 0) s_M[slot] = M;
   }
   __syncthreads();
