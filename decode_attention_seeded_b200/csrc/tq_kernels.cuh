@@ -478,8 +478,8 @@ __device__ __forceinline__ uint64_t umma_desc_noswizzle(uint32_t saddr, uint32_t
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
-// Tiled tensor copy of one box into shared memory (this GPU's memory, no
-// multicast); the box's bytes complete the transaction count on `bar`.
+// Tiled tensor copy of one box of this GPU's memory into this CTA's shared
+// memory; the box's bytes complete the transaction count on `bar`.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
                                             uint64_t* bar) {
   asm volatile(

@@ -92,6 +92,60 @@ def test_quantize_matches_oracle(bk, bv, dtype, path):
         assert rep["excused_k_codes"] + rep["excused_v_codes"] < 0.001 * L * 128
 
 
+@pytest.mark.parametrize("bk,bv,dtype", [(3, 2, "bf16"), (4, 4, "fp16"), (2, 3, "bf16")])
+def test_prefill_short_runs_match_oracle(bk, bv, dtype):
+    """A context built by prefill calls of 1, 3, 12, 1, 33 and 150 tokens: runs that
+    start and end inside a page, single tokens, runs spanning several pages, an odd
+    number of KV heads. Every token is checked against the oracle's quantization."""
+    seeds = (41 + bk, 42 + bv, 43)
+    ctx = _ctx(bk, bv, seeds)
+    tab = oracle_tables(seeds, bk, bv)
+    rng = np.random.default_rng(bk * 11 + bv)
+    runs = [1, 3, 12, 1, 33, 150]
+    L, n_kv = sum(runs), 3
+    k, v = _rand_kv(rng, L, n_kv, dtype)
+    bt, n_pages = _pool([L], 7)
+    cache = torch.zeros(n_pages * ctx.page_bytes(n_kv), dtype=torch.uint8, device=DEV)
+    kt, vt = _t(k, dtype), _t(v, dtype)
+    btt = torch.from_numpy(bt[0]).to(DEV)
+    pos = 0
+    for n in runs:
+        ctx.quantize_prefill(kt[pos:pos + n].contiguous(), vt[pos:pos + n].contiguous(), btt, pos, cache, n_pages)
+        pos += n
+    assert ctx.device_error() == 0
+    host = cache.cpu().numpy().reshape(n_pages, n_kv, -1)
+    for h in range(n_kv):
+        qk, qv = oracle_quantize(k[:, h].astype(np.float64), v[:, h].astype(np.float64), tab)
+        rep = compare_tokens(unpack_tokens(host, bt[0], 0, L, h, bk, bv), qk, qv, tab)
+        assert all(x == 0 for key, x in rep.items() if key.startswith("bad")), (h, rep)
+
+
+def test_prefill_bad_page_sets_device_error_and_spares_the_rest():
+    """A block-table entry outside the pool: that page is skipped with
+    TQ_DEV_BAD_SLOT, every other page is written as usual."""
+    bk, bv, n_kv = 3, 2, 2
+    seeds = (51, 52, 53)
+    ctx = _ctx(bk, bv, seeds)
+    tab = oracle_tables(seeds, bk, bv)
+    rng = np.random.default_rng(9)
+    L = 64                                      # 4 pages
+    k, v = _rand_kv(rng, L, n_kv, "bf16")
+    bt, n_pages = _pool([L], 3)
+    bad = bt[0].copy()
+    bad[2] = n_pages + 5                        # third page out of range
+    cache = torch.zeros(n_pages * ctx.page_bytes(n_kv), dtype=torch.uint8, device=DEV)
+    ctx.quantize_prefill(_t(k, "bf16"), _t(v, "bf16"), torch.from_numpy(bad).to(DEV), 0, cache, n_pages)
+    assert ctx.device_error() & binding.DEV_BAD_SLOT
+    host = cache.cpu().numpy().reshape(n_pages, n_kv, -1)
+    good_tokens = np.r_[0:32, 48:64]
+    for h in range(n_kv):
+        # the oracle quantizes each token on its own: quantize the kept tokens only
+        qk, qv = oracle_quantize(k[good_tokens, h].astype(np.float64), v[good_tokens, h].astype(np.float64), tab)
+        got = unpack_tokens(host, bt[0], 0, L, h, bk, bv)
+        rep = compare_tokens(tuple(np.asarray(x)[good_tokens] for x in got), qk, qv, tab)
+        assert all(x == 0 for key, x in rep.items() if key.startswith("bad")), (h, rep)
+
+
 def test_quantize_bad_slot_sets_device_error():
     ctx = _ctx(3, 2, (1, 2, 3))
     n_pages = 2
