@@ -2255,11 +2255,13 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     for (int h = 0; h < NH; ++h) {
       float pm = fmaxf(pg[0].lp2[h][0], pg[0].lp2[h][1]);
       if (npg == 2) pm = fmaxf(pm, fmaxf(pg[1].lp2[h][0], pg[1].lp2[h][1]));
-      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 4));
-      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 8));
-      pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 16));
-      const bool need = pm > mp2[h] + 8.0f;
-      if (__any_sync(kFull, need)) {
+      // The head's maximum over its 8 lanes is only needed when it moves: when no
+      // lane's own values exceed the margin, no head's maximum does either.
+      if (__any_sync(kFull, pm > mp2[h] + 8.0f)) {
+        pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 4));
+        pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 8));
+        pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 16));
+        const bool need = pm > mp2[h] + 8.0f;
         const float fac = need ? ex2(mp2[h] - pm) : 1.0f;
         if (need) mp2[h] = pm;
         lsum[h] *= fac;
