@@ -1423,12 +1423,14 @@ __device__ __forceinline__ int warp_isum(int v) {
 
 // ================================================================== decode
 // Warps per decode CTA, one CTA per SM. Uniform split: 16 for one group of 4
-// query heads (the kernel then fits 128 registers), 12 for two groups (168
-// registers), 8 for three. The balanced split, whose loop over segments needs
-// more registers: 12 for one group, 8 for more.
+// query heads (the kernel then fits 128 registers), 12 for two or three groups
+// (168 registers; with three groups a few hundred bytes spill, and the extra
+// warps still hide more latency than the spills cost). The balanced split,
+// whose loop over segments needs more registers: 12 for one or three groups, 8
+// for two (12 were slower there).
 template <int NH, bool BAL = false>
 struct DecodeWarps {
-  static constexpr int value = BAL ? (NH == 1 ? 12 : 8) : NH == 1 ? 16 : NH == 2 ? 12 : 8;
+  static constexpr int value = BAL ? (NH == 2 ? 8 : 12) : NH == 1 ? 16 : 12;
 };
 // TMA stages per warp: six when they fit in 160 KB of shared memory, else four.
 constexpr int kAccPitch = 132;      // floats per accumulator column in the CTA merge
