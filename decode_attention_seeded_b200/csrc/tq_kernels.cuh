@@ -507,35 +507,26 @@ __device__ __forceinline__ int pf_coord(int i, int t) { return 16 * (i >> 2) + 4
 
 // Cell of y in a symmetric b-bit codebook: code = #{j : y > t_j} (a value on a
 // threshold may land in either neighbour; such values lie inside the tolerance
-// band) and the centroid c[code]. thr / cen: the 2^b - 1 thresholds and 2^b
-// centroids in ascending order; the middle threshold is 0.
-template <int B, typename TA, typename CA>
-__device__ __forceinline__ int cell_of(float y, const TA& thr, const CA& cen, float& chat) {
+// band). thr: the 2^b - 1 thresholds in ascending order; the middle one is 0, so
+// a binary search over the positive half and the sign give the cell.
+template <int B, typename TA>
+__device__ __forceinline__ int cell_code(float y, const TA& thr) {
   constexpr int H = 1 << (B - 1);
   const float a = fabsf(y);
   int k;
-  float cp;
   if constexpr (B == 2) {
-    const bool p = a > thr[H];
-    k = p;
-    cp = p ? cen[H + 1] : cen[H];
+    k = a > thr[H];
   } else if constexpr (B == 3) {
     const bool p2 = a > thr[H + 1];
     const bool p1 = a > (p2 ? thr[H + 2] : thr[H]);
     k = 2 * p2 + p1;
-    cp = p2 ? (p1 ? cen[H + 3] : cen[H + 2]) : (p1 ? cen[H + 1] : cen[H]);
   } else {
     const bool p4 = a > thr[H + 3];
     const bool p2 = a > (p4 ? thr[H + 5] : thr[H + 1]);
     const bool p1 = a > (p4 ? (p2 ? thr[H + 6] : thr[H + 4]) : (p2 ? thr[H + 2] : thr[H]));
     k = 4 * p4 + 2 * p2 + p1;
-    const float lo = p2 ? (p1 ? cen[H + 3] : cen[H + 2]) : (p1 ? cen[H + 1] : cen[H]);
-    const float hi = p2 ? (p1 ? cen[H + 7] : cen[H + 6]) : (p1 ? cen[H + 5] : cen[H + 4]);
-    cp = p4 ? hi : lo;
   }
-  const bool pos = y > 0.0f;
-  chat = pos ? cp : -cp;
-  return pos ? H + k : H - 1 - k;
+  return y > 0.0f ? H + k : H - 1 - k;
 }
 
 // Add code `c` of lane-local coordinate i (selector i >> 2, nibble i & 3) to the
@@ -747,11 +738,12 @@ constexpr float kPfInvRootD = 0.08838834764831845f;   // 1 / sqrt(128)
 // the rotated unit domain with |u|^2, and u 2^10 as fp16 high and low parts in
 // the m16n8k16 A-fragment order of z = S u (tokens on the rows): ah[ks][r],
 // r = token half (r & 1), coordinate pair 4ks + 2 (r >> 1).
-// cnk10: the key centroids times 2^10, so that u 2^10 = y 2^10 - c^ 2^10 is one
-// fused operation with a single rounding (the same value as (y - c^) 2^10).
+// cnk10: the key centroids times 2^10 (in shared memory, indexed by the code), so
+// that u 2^10 = y 2^10 - c^ 2^10 is one fused operation with a single rounding (the
+// same value as (y - c^) 2^10).
 template <int BK, typename TA>
 __device__ __forceinline__ void pf_key_residual(float (&vv)[2][32], const float (&ss)[2], const TA& thk,
-                                                const TA& cnk10, uint32_t (&kw)[2][4], float (&nk)[2],
+                                                const float* cnk10, uint32_t (&kw)[2][4], float (&nk)[2],
                                                 float (&uu)[2], uint32_t (&ah)[8][4], uint32_t (&al)[8][4]) {
 #pragma unroll
   for (int th = 0; th < 2; ++th) {
@@ -762,8 +754,8 @@ __device__ __forceinline__ void pf_key_residual(float (&vv)[2][32], const float 
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float y = vv[th][i] * inv;
-      float chat10;
-      const int c = cell_of<BK>(y, thk, cnk10, chat10);
+      const int c = cell_code<BK>(y, thk);
+      const float chat10 = cnk10[c];
       put_key_code<BK>(kw[th], i, static_cast<uint32_t>(c));
       const float u10 = fmaf(y, 1024.0f, -chat10);  // u 2^10: well inside the fp16 range
       u2 = fmaf(u10, u10, u2);
@@ -824,7 +816,7 @@ __device__ __forceinline__ void pf_key_store(uint8_t* blk, int lane, int g, bool
 // stored (merged under the token mask at the ends of a run).
 template <int BK, int BV, typename TA>
 __device__ __forceinline__ void pf_values(const float (&vv)[2][32], const float (&ss)[2], const TA& thv,
-                                          const TA& cnv, uint8_t* vt, uint8_t* blk, int lane, int g, int t,
+                                          uint8_t* vt, uint8_t* blk, int lane, int g, int t,
                                           int tau0, int tau1, bool full, bool ok0, bool ok1) {
   float nv[2];
 #pragma unroll
@@ -835,9 +827,8 @@ __device__ __forceinline__ void pf_values(const float (&vv)[2][32], const float 
     __syncwarp();                                            // the tile's previous readers are done
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      float chat;
-      const int c0 = cell_of<BV>(vv[0][i] * inv0, thv, cnv, chat);
-      const int c1 = cell_of<BV>(vv[1][i] * inv1, thv, cnv, chat);
+      const int c0 = cell_code<BV>(vv[0][i] * inv0, thv);
+      const int c1 = cell_code<BV>(vv[1][i] * inv1, thv);
       // tokens g, g + 8 sit at bytes 2g, 2g + 1 of the coordinate's 16-byte row
       *reinterpret_cast<uint16_t*>(vt + pf_coord(i, t) * 16 + 2 * g) = static_cast<uint16_t>(c0 | (c1 << 8));
     }
@@ -955,11 +946,15 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
     dmk |= (T.signs_k[pf_coord(i, t)] < 0.0f ? 1u : 0u) << i;
     dmv |= (T.signs_v[pf_coord(i, t)] < 0.0f ? 1u : 0u) << i;
   }
-  float thk[16], cnk10[16], thv[16], cnv[16];
+  float thk[16], thv[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    thk[i] = T.thr_k[i]; cnk10[i] = T.cen_k[i] * 1024.0f; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
+    thk[i] = T.thr_k[i];
+    thv[i] = T.thr_v[i];
   }
+  __shared__ float cnk10[16];                   // key centroids x 2^10, by code
+  if (threadIdx.x < 16) cnk10[threadIdx.x] = T.cen_k[threadIdx.x] * 1024.0f;
+  __syncthreads();
   __syncwarp();
   const int first_page = start_pos / kPage;
   const int n_tiles = ((start_pos + n_tokens - 1) / kPage - first_page + 1) * n_kv;
@@ -1095,7 +1090,7 @@ __global__ void __launch_bounds__(256, 2) quantize_prefill_kernel(Tables T, cons
         pf_key_store<BK, BV>(blk, lane, g, ok0, ok1, kw, sw, nk, uu);
       }
     } else {
-      pf_values<BK, BV>(vv, ss, thv, cnv, vt, blk, lane, g, t, tau0, tau1, full, ok0, ok1);
+      pf_values<BK, BV>(vv, ss, thv, vt, blk, lane, g, t, tau0, tau1, full, ok0, ok1);
     }
     }
   }
@@ -1187,11 +1182,15 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
     mbar_expect_tx(bar_sk, 32768u);
     tma_load_1d(sk, T.sketch_umma, 32768u, bar_sk);
   }
-  float thk[16], cnk10[16], thv[16], cnv[16];
+  float thk[16], thv[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    thk[i] = T.thr_k[i]; cnk10[i] = T.cen_k[i] * 1024.0f; thv[i] = T.thr_v[i]; cnv[i] = T.cen_v[i];
+    thk[i] = T.thr_k[i];
+    thv[i] = T.thr_v[i];
   }
+  __shared__ float cnk10[16];                   // key centroids x 2^10, by code
+  if (threadIdx.x < 16) cnk10[threadIdx.x] = T.cen_k[threadIdx.x] * 1024.0f;
+  __syncthreads();
   const bool bf16 = dtype == TQ_BF16;
   const int first_page = start_pos / kPage;
   const int n_tiles = ((start_pos + n_tokens - 1) / kPage - first_page + 1) * n_kv;
@@ -1319,7 +1318,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
         stage_rows(next, 1);
         vpend = true;
       }
-      if (good) pf_values<BK, BV>(vv, ss, thv, cnv, vt, blk, lane, g, t, tau0, tau1, full, ok0, ok1);
+      if (good) pf_values<BK, BV>(vv, ss, thv, vt, blk, lane, g, t, tau0, tau1, full, ok0, ok1);
     }
 
     // ---- this warp's rows of z: sign bits, then the key words
