@@ -13,7 +13,10 @@ caches (about 0.86 GB) exceed the 126 MB L2, so every step streams from HBM.
             K steps, CUDA events on the launching stream, max over ranks).
 ``e2e``     the same steps through the C ABI with host buffers: per step the
             new K/V and queries are copied from pinned host memory and the
-            attention outputs copied back, inside the timed region.
+            attention outputs copied back, inside the timed region. The copies
+            run on a second stream and overlap the layers' work (layer 0's
+            inputs first; each layer's outputs as soon as it ends), checked
+            against the same steps with every copy in line.
 ``roofline`` the kernel the timed step launches (decode_kernel via
             tq_decode_step: append, query transform, split-K decode and merge,
             once per layer) against the measured HBM copy bandwidth: algorithmic
@@ -209,20 +212,20 @@ class DecodeBench:
         self.out = torch.zeros((self.n_layers, B, nq, 128), dtype=torch.float32, device=device)
         self.ws_bytes = self.ctx.decode_workspace_bytes(B, nq, n_kv, self.max_len)
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=device)
-        # host-side buffers for the end-to-end arm
-        self.h_newk = torch.empty((self.total_steps, self.n_layers, B, n_kv, 128), dtype=torch.bfloat16,
-                                  pin_memory=True)
-        self.h_newv = torch.empty_like(self.h_newk, pin_memory=True)
-        self.h_q = torch.empty((self.total_steps, self.n_layers, B, nq, 128), dtype=torch.bfloat16,
-                               pin_memory=True)
-        self.h_newk.copy_(self.newk.transpose(0, 1).cpu())
-        self.h_newv.copy_(self.newv.transpose(0, 1).cpu())
-        self.h_q.copy_(self.q.cpu())
+        # host-side buffers for the end-to-end arm: per step and layer the new K, the
+        # new V and the queries back to back, so that one copy moves any run of layers
+        self.n_k, self.n_qe = B * n_kv * 128, B * nq * 128
+        row = 2 * self.n_k + self.n_qe
+        self.h_in = torch.empty((self.total_steps, self.n_layers, row), dtype=torch.bfloat16, pin_memory=True)
+        nk = self.n_k
+        self.h_in[:, :, :nk].copy_(self.newk.transpose(0, 1).reshape(self.total_steps, self.n_layers, nk).cpu())
+        self.h_in[:, :, nk:2 * nk].copy_(self.newv.transpose(0, 1).reshape(self.total_steps, self.n_layers, nk).cpu())
+        self.h_in[:, :, 2 * nk:].copy_(self.q.reshape(self.total_steps, self.n_layers, self.n_qe).cpu())
         self.h_out = torch.empty((self.total_steps, self.n_layers, B, nq, 128), dtype=torch.float32,
                                  pin_memory=True)
-        self.d_stepk = torch.empty((self.n_layers, B, n_kv, 128), dtype=torch.bfloat16, device=device)
-        self.d_stepv = torch.empty_like(self.d_stepk)
-        self.d_stepq = torch.empty((self.n_layers, B, nq, 128), dtype=torch.bfloat16, device=device)
+        self.d_in = torch.empty((self.n_layers, row), dtype=torch.bfloat16, device=device)
+        self.copy_stream = torch.cuda.Stream(device=device)
+        self.ev_in, self.ev_out = torch.cuda.Event(), (torch.cuda.Event(), torch.cuda.Event())
 
     @property
     def cache_tokens(self):
@@ -238,25 +241,55 @@ class DecodeBench:
                                  n_pages, self.btabs[layer], self.lens[s], wl.n_kv_heads, self.max_len,
                                  self.out[layer], self.ws)
 
-    # the same step through host buffers
+    # the same step through host buffers, copies overlapped with the layers' work.
+    # Layer 0's inputs are copied on the launching stream; the other layers'
+    # inputs follow on a copy stream (layer 1 waits for them) while layer 0 runs.
+    # The outputs of all but the last two layers go back on the copy stream while
+    # those two run; the last two layers' outputs end the step.
     def step_e2e(self, s):
-        wl = self.wl
-        self.d_stepk.copy_(self.h_newk[s], non_blocking=True)
-        self.d_stepv.copy_(self.h_newv[s], non_blocking=True)
-        self.d_stepq.copy_(self.h_q[s], non_blocking=True)
+        torch = self.torch
+        main, cs = torch.cuda.current_stream(self.dev), self.copy_stream
+        n = self.n_layers
+        split = max(n - 2, 0)
+        self.d_in[0].copy_(self.h_in[s, 0], non_blocking=True)
+        cs.wait_stream(main)                  # after layer 0's copy and the previous step
+        with torch.cuda.stream(cs):
+            if n > 1:
+                self.d_in[1:].copy_(self.h_in[s, 1:], non_blocking=True)
+            self.ev_in.record(cs)
+        for layer in range(n):
+            if layer == 1:
+                main.wait_event(self.ev_in)
+            self.decode_layer_e2e(layer, s)
+            for a, b, ev in ((0, split, self.ev_out[0]), (split, n, self.ev_out[1])):
+                if layer == b - 1:
+                    ev.record(main)
+                    with torch.cuda.stream(cs):
+                        cs.wait_event(ev)
+                        self.h_out[s, a:b].copy_(self.out[a:b], non_blocking=True)
+        main.wait_stream(cs)
+
+    # the same step through host buffers, every copy in line with the layers (the
+    # order check of the overlapped step compares against it)
+    def step_e2e_serial(self, s):
+        self.d_in.copy_(self.h_in[s], non_blocking=True)
         for layer in range(self.n_layers):
-            cache, n_pages = self.caches[layer]
-            self.ctx.decode_step(self.d_stepk[layer], self.d_stepv[layer], self.d_stepq[layer],
-                                 cache, n_pages, self.btabs[layer], self.lens[s], wl.n_kv_heads, self.max_len,
-                                 self.out[layer], self.ws)
+            self.decode_layer_e2e(layer, s)
         self.h_out[s].copy_(self.out, non_blocking=True)
 
+    def decode_layer_e2e(self, layer, s):
+        wl, nk = self.wl, self.n_k
+        cache, n_pages = self.caches[layer]
+        k = self.d_in[layer, :nk].view(wl.batch, wl.n_kv_heads, 128)
+        v = self.d_in[layer, nk:2 * nk].view(wl.batch, wl.n_kv_heads, 128)
+        q = self.d_in[layer, 2 * nk:].view(wl.batch, wl.n_q_heads, 128)
+        self.ctx.decode_step(k, v, q, cache, n_pages, self.btabs[layer], self.lens[s], wl.n_kv_heads,
+                             self.max_len, self.out[layer], self.ws)
+
     def e2e_bytes(self):
-        e = 2
-        wl = self.wl
-        h2d = self.n_layers * wl.batch * (2 * wl.n_kv_heads * 128 * e + wl.n_q_heads * 128 * e)
-        d2h = self.n_layers * wl.batch * wl.n_q_heads * 128 * 4
-        return h2d, d2h
+        """Bytes the end-to-end step copies in (h_in[s]) and out (h_out[s])."""
+        return (self.h_in[0].numel() * self.h_in.element_size(),
+                self.h_out[0].numel() * self.h_out.element_size())
 
     def capture(self, fn, steps):
         torch = self.torch
@@ -822,8 +855,21 @@ def main():
     # end-to-end arm: same K steps from host buffers (state rewinds: same slots rewritten)
     g_e2e = bench.capture(bench.step_e2e, range(W, W + K))
     g_e2e_w = bench.capture(bench.step_e2e, range(W))
+    # order check of the overlapped copies: the same steps with every copy in line
+    # with the layers give the host the same outputs (up to the summation order of
+    # the split-K merge, which depends on which warp took which page)
+    g_ser = bench.capture(bench.step_e2e_serial, range(W, W + K))
+    g_e2e_w.replay()
+    g_ser.replay()
+    torch.cuda.synchronize(dev)
+    ref_out = bench.h_out[W:W + K].clone()
+    del g_ser
     g_e2e_w.replay()
     g_e2e.replay()                                        # graph upload, untimed (as above)
+    torch.cuda.synchronize(dev)
+    e2e_dev = float((bench.h_out[W:W + K] - ref_out).abs().max() / ref_out.abs().max().clamp_min(1e-30))
+    assert e2e_dev < 1e-4, f"overlapped end-to-end copies disagree with the in-line ones: {e2e_dev}"
+    del ref_out
     barrier()
     t_e2e = max_over_ranks(timed(torch, dev, g_e2e.replay), world, dev)
     barrier()
@@ -863,7 +909,9 @@ def main():
         "dtype": f"int8/fp16 tensor-core, fp32 accumulate ({key_format(wl.key_bits)}, {wl.value_bits}-bit values)",
         "data": "synthetic",
         "config": workload_config(wl, world, K, W, args.sparse_v, args.peaked),
-        "e2e": {"value": job_throughput(K * wl.batch, world, t_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": job_throughput(K * wl.batch, world, t_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "copies": "layer 0's inputs in line, the others' on a copy stream; outputs in two copies, the first overlapping the last two layers",
+                "order_check_max_rel_diff": e2e_dev},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                      "kernel": "decode_kernel via tq_decode_step (append, query transform, split-K decode, "
