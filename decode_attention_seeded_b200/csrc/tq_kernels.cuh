@@ -1489,9 +1489,11 @@ __device__ __forceinline__ void key_limbs(uint32_t sel, const uint32_t (&th)[4],
   }
 }
 
-// Value selectors: 16 selectors s = 2*mt + tg; nibble n = 2*hf + e.
+// Value selectors (2- and 3-bit values; 4-bit values use a byte-indexed table):
+// 16 selectors s = 2*mt + tg; nibble n = 2*hf + e.
 template <int B>
 __device__ __forceinline__ void value_selectors(const uint32_t* w, uint32_t (&sel)[16]) {
+  static_assert(B == 2 || B == 3, "value selectors: 2 or 3 bits");
   if constexpr (B == 2) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -1511,12 +1513,6 @@ __device__ __forceinline__ void value_selectors(const uint32_t* w, uint32_t (&se
       s[0] = a; s[1] = shr<16>(a); s[2] = b; s[3] = shr<16>(b);
       s[4] = c; s[5] = shr<16>(c); s[6] = sp; s[7] = shr<16>(sp);
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      sel[2 * i] = w[i];
-      sel[2 * i + 1] = shr<16>(w[i]);
-    }
   }
 }
 
@@ -1525,14 +1521,7 @@ __device__ __forceinline__ void value_selectors(const uint32_t* w, uint32_t (&se
 template <int B>
 __device__ __forceinline__ void value_regs(uint32_t sel, const uint32_t (&vl)[4], const uint32_t (&vh)[4],
                                            uint32_t& r0, uint32_t& r1) {
-  uint32_t lo, hi;
-  if constexpr (B == 4) {
-    lo = lookup16(sel, vl[0], vl[1], vl[2], vl[3]);
-    hi = lookup16(sel, vh[0], vh[1], vh[2], vh[3]);
-  } else {
-    lo = prmt(vl[0], vl[1], sel);
-    hi = prmt(vh[0], vh[1], sel);
-  }
+  const uint32_t lo = prmt(vl[0], vl[1], sel), hi = prmt(vh[0], vh[1], sel);
   r0 = prmt(lo, hi, 0x5140u);
   r1 = prmt(lo, hi, 0x7362u);
 }
@@ -1724,6 +1713,20 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     P.tab[16 + threadIdx.x] = T.cen_k[threadIdx.x];
     P.tab[32 + threadIdx.x] = T.thr_v[threadIdx.x];
     P.tab[48 + threadIdx.x] = T.cen_v[threadIdx.x];
+  }
+  // 4-bit values: the fp16 A-operand registers of the value product come from a
+  // byte-indexed table in shared memory, entry b = fp16x2 (c(b & 15), c(b >> 4))
+  // with the first code in the low half, one load per two codes instead of the
+  // 16-entry byte-permute lookup (whose bit-3 select costs more than the load).
+  // For 2-bit values the 8-byte entries a byte would need collide on the banks,
+  // and for 4-bit keys the limb pairs need two more byte-permutes per load: both
+  // stay on the byte-permute lookups.
+  __shared__ uint32_t s_vtab[BV == 4 && !LOGITS ? 256 : 1];
+  if constexpr (BV == 4 && !LOGITS) {
+    auto byte_of = [](const uint32_t (&tb)[4], int c) -> uint32_t { return (tb[c >> 2] >> (8 * (c & 3))) & 0xFFu; };
+    for (int e = threadIdx.x; e < 256; e += blockDim.x)
+      s_vtab[e] = byte_of(T.v_lo, e & 15) | (byte_of(T.v_hi, e & 15) << 8) | (byte_of(T.v_lo, e >> 4) << 16) |
+                  (byte_of(T.v_hi, e >> 4) << 24);
   }
   // Everything above reads only the context's own tables, which no kernel writes.
   // Launched as a programmatic dependent of the previous kernel in the stream:
@@ -2318,15 +2321,30 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
 
   // ---- weighted value sum in the rotated domain: fp16 tensor-core products
   auto value_product = [&](const uint32_t (&vw)[2 * BV], const uint32_t (&pbq)[NH][2]) {
-    uint32_t vs[16];
-    value_selectors<BV>(vw, vs);
+    if constexpr (BV == 4) {
+      // m-tile mt: word mt, whose bytes 0 .. 3 give A registers 0 .. 3
+      const uint8_t* vt8 = reinterpret_cast<const uint8_t*>(s_vtab);
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      uint32_t a0, a1, a2, a3;
-      value_regs<BV>(vs[2 * mt], vlo_, vhi_, a0, a1);
-      value_regs<BV>(vs[2 * mt + 1], vlo_, vhi_, a2, a3);
+      for (int mt = 0; mt < 8; ++mt) {
+        const uint32_t w = vw[mt];
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(vt8 + ((w << 2) & 0x3FCu));
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(vt8 + (shr<6>(w) & 0x3FCu));
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vt8 + (shr<14>(w) & 0x3FCu));
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vt8 + (shr<22>(w) & 0x3FCu));
 #pragma unroll
-      for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pbq[h][0], pbq[h][1]);
+        for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pbq[h][0], pbq[h][1]);
+      }
+    } else {
+      uint32_t vs[16];
+      value_selectors<BV>(vw, vs);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        value_regs<BV>(vs[2 * mt], vlo_, vhi_, a0, a1);
+        value_regs<BV>(vs[2 * mt + 1], vlo_, vhi_, a2, a3);
+#pragma unroll
+        for (int h = 0; h < NH; ++h) mma_f16(acc[h][mt], a0, a1, a2, a3, pbq[h][0], pbq[h][1]);
+      }
     }
   };
 
