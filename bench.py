@@ -678,19 +678,35 @@ def bench_parity(bench, layer, pairs=4, near=1e-5, rtol=1e-3):
     rng = np.random.default_rng(0)
     allp = [(b, h) for b in range(wl.batch) for h in range(n_kv)]
     pick = [allp[int(i)] for i in rng.permutation(len(allp))[:pairs]]
-    worst, worst_e = 0.0, 0.0
+    worst, worst_e, nonfinite = 0.0, 0.0, 0
     for b, h in pick:
         want = odec.decode_paged(host[:, h:h + 1], bt[b:b + 1], [int(L[b])], q[b:b + 1, h * g:(h + 1) * g], tab)[0]
-        got = out[b, h * g:(h + 1) * g]
-        ref = np.linalg.norm(want, axis=-1)
-        worst = max(worst, float(np.max(np.linalg.norm(got - want, axis=-1) / ref)))
-        floor = ref[:, None] / np.sqrt(128)
-        worst_e = max(worst_e, float(np.max(np.abs(got - want) / np.maximum(np.abs(want), floor))))
+        w, we, nf = decode_row_errors(out[b, h * g:(h + 1) * g], want)
+        worst, worst_e, nonfinite = max(worst, w), max(worst_e, we), nonfinite + nf
     res.update({"decode_pairs": [list(x) for x in pick], "decode_tokens": [int(L[b]) for b, _ in pick],
-                "worst_rel_err": worst, "worst_elem_err": worst_e, "tolerance": rtol,
-                "ok": bool(worst <= rtol and worst_e <= rtol and all(
+                "worst_rel_err": worst, "worst_elem_err": worst_e, "nonfinite_outputs": nonfinite,
+                "tolerance": rtol,
+                "ok": bool(nonfinite == 0 and worst <= rtol and worst_e <= rtol and all(
                     res[k] == 0 for k in res if isinstance(k, str) and k.startswith("bad")))})
     return res
+
+
+def decode_row_errors(got, want):
+    """(worst per-head relative error, worst element error, count of non-finite
+    outputs) of decode outputs got [heads, 128] against the oracle's want. The
+    element error is relative to the element, floored at the head's rms element
+    size. Non-finite outputs are counted, not folded into the maxima (a NaN would
+    otherwise compare as no error)."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    nonfinite = int(np.sum(~np.isfinite(got)))
+    if nonfinite:
+        return 0.0, 0.0, nonfinite
+    ref = np.linalg.norm(want, axis=-1)
+    worst = float(np.max(np.linalg.norm(got - want, axis=-1) / ref))
+    floor = ref[:, None] / np.sqrt(want.shape[-1])
+    worst_e = float(np.max(np.abs(got - want) / np.maximum(np.abs(want), floor)))
+    return worst, worst_e, 0
 
 
 def reference_arm(wl, args, world):
