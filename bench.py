@@ -303,7 +303,32 @@ class DecodeBench:
         torch.cuda.current_stream(self.dev).wait_stream(s)
         return g
 
-    def quantize_timing(self, reps=5):
+    def graph_seconds(self, calls, reps=1):
+        """Device seconds per call of `calls` (zero-argument callables that launch
+        work on the current stream), each run once eagerly (library set-up, first-use
+        allocations), then `reps` times over captured in one CUDA graph, replayed once
+        untimed and timed on one more replay with CUDA events: the host's launch
+        overhead stays out of the figure, as it does for the decode steps."""
+        torch = self.torch
+        for c in calls:
+            c()
+        torch.cuda.synchronize(self.dev)
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=self.dev)
+        s.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(reps):
+                    for c in calls:
+                        c()
+        torch.cuda.current_stream(self.dev).wait_stream(s)
+        g.replay()
+        torch.cuda.synchronize(self.dev)
+        t = timed(torch, self.dev, g.replay)
+        del g
+        return t / (reps * len(calls))
+
+    def quantize_timing(self, reps=6):
         """Quantize-prefill of one layer's full context (K and V of every KV head).
 
         Algorithmic bytes = the K/V inputs read + the compressed blocks written.
@@ -321,22 +346,14 @@ class DecodeBench:
             bufs.append((k, v))
         cache, n_pages = self.caches[0]
         bt = self.btabs[0][0]
-        self.ctx.quantize_prefill(bufs[0][0], bufs[0][1], bt, 0, cache, n_pages)
-        torch.cuda.synchronize(self.dev)
-        st = torch.cuda.current_stream(self.dev)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        for r in range(reps):
-            k, v = bufs[r % 2]
-            evs[r][0].record(st)
-            self.ctx.quantize_prefill(k, v, bt, 0, cache, n_pages)
-            evs[r][1].record(st)
-        torch.cuda.synchronize(self.dev)
-        secs = statistics.median(a.elapsed_time(b) for a, b in evs) / 1e3
+        calls = [lambda k=k, v=v: self.ctx.quantize_prefill(k, v, bt, 0, cache, n_pages) for k, v in bufs]
+        secs = self.graph_seconds(calls, reps=reps // 2)
         bytes_in = 2 * self.T0 * n_kv * 128 * 2
         bytes_out = self.T0 * n_kv * (self.ctx.block_bytes // 16)
         return {"gbs": (bytes_in + bytes_out) / secs / 1e9, "us_per_call": secs * 1e6,
                 "tokens": self.T0, "kv_heads": n_kv, "bytes_in": bytes_in, "bytes_out": bytes_out,
-                "kernel": "quantize_prefill_kernel via tq_quantize_prefill (bf16 K/V, one layer)"}
+                "timing": f"CUDA graph of {reps} calls on two alternating input buffers",
+                "kernel": "quantize_prefill_tc_kernel via tq_quantize_prefill (bf16 K/V, one layer)"}
 
     def logits_timing(self, reps=10):
         """Logits only (tq_decode_logits) against logits from full-precision fp32 keys.
@@ -351,7 +368,6 @@ class DecodeBench:
         g = nq // n_kv
         last = self.total_steps - 1
         out = torch.empty((B, nq, T), dtype=torch.float32, device=self.dev)
-        st = torch.cuda.current_stream(self.dev)
 
         def run_ours(layer):
             cache, n_pages = self.caches[layer]
@@ -359,20 +375,12 @@ class DecodeBench:
                                    T, out)
 
         def time_it(fn, layers):
-            fn(0)
-            torch.cuda.synchronize(self.dev)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(st)
-            for _ in range(reps):
-                for layer in range(layers):
-                    fn(layer)
-            b.record(st)
-            b.synchronize()
-            return a.elapsed_time(b) / 1e3 / (reps * layers)
+            return self.graph_seconds([lambda layer=layer: fn(layer) for layer in range(layers)], reps=reps)
 
         ours = time_it(run_ours, self.n_layers)
         key_bytes = self.cache_tokens * n_kv * key_bytes_per_token(wl.key_bits)
         res = {"kernel": "decode_kernel (logits mode) via tq_decode_logits", "us_per_layer": ours * 1e6,
+               "timing": f"CUDA graph of {reps} passes over the layer caches (both arms)",
                "key_bytes_per_layer": key_bytes, "gbs": key_bytes / ours / 1e9,
                "logit_bytes_written": nq * int(self.lens[last].sum().item()) * 4}
         try:
@@ -411,11 +419,18 @@ class DecodeBench:
         lens = self.lens[-1]                          # final step's lengths (int32, per sequence)
         ragged = bool((lens != lens[0]).any())
         st = torch.cuda.current_stream(self.dev)
-        results, errors = {}, {}
+        results, errors, timing = {}, {}, {}
 
-        def time_it(fn):
-            fn(0)
-            torch.cuda.synchronize(self.dev)
+        def time_it(fn, name):
+            # a CUDA graph like the compressed path; eager launches if the library
+            # call cannot be captured
+            try:
+                t = self.graph_seconds([lambda layer=layer: fn(layer) for layer in range(layers)], reps=reps)
+                timing[name] = "cuda graph"
+                return t
+            except Exception as e:
+                errors[name + " (graph capture)"] = repr(e)[:200]
+                torch.cuda.synchronize(self.dev)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(st)
             for _ in range(reps):
@@ -423,13 +438,14 @@ class DecodeBench:
                     fn(layer)
             b.record(st)
             b.synchronize()
+            timing[name] = "eager"
             return a.elapsed_time(b) / 1e3 / (reps * layers)
 
         try:
             from flash_attn import __version__ as fav
             from flash_attn import flash_attn_with_kvcache
-            results[f"flash_attn {fav} flash_attn_with_kvcache"] = time_it(
-                lambda l: flash_attn_with_kvcache(q, kc[l], vc[l], cache_seqlens=lens))
+            name = f"flash_attn {fav} flash_attn_with_kvcache"
+            results[name] = time_it(lambda l: flash_attn_with_kvcache(q, kc[l], vc[l], cache_seqlens=lens), name)
         except Exception as e:                       # library kernel unavailable on this build
             errors["flash_attn"] = repr(e)[:200]
         try:
@@ -439,8 +455,8 @@ class DecodeBench:
             qs = q.transpose(1, 2)                   # [B, nq, 1, 128]
             kt = [k.transpose(1, 2) for k in kc]
             vt = [v.transpose(1, 2) for v in vc]
-            results[f"torch {torch.__version__} scaled_dot_product_attention (enable_gqa)"] = time_it(
-                lambda l: F.scaled_dot_product_attention(qs, kt[l], vt[l], enable_gqa=True))
+            name = f"torch {torch.__version__} scaled_dot_product_attention (enable_gqa)"
+            results[name] = time_it(lambda l: F.scaled_dot_product_attention(qs, kt[l], vt[l], enable_gqa=True), name)
         except Exception as e:
             errors["sdpa"] = repr(e)[:200]
         del kc, vc
@@ -451,7 +467,7 @@ class DecodeBench:
         nbytes = 2 * int(lens.sum().item()) * n_kv * 128 * 2
         return {"kernel": name, "us_per_layer": secs * 1e6, "bytes_per_layer": nbytes,
                 "gbs": nbytes / secs / 1e9, "all_us": {k: v * 1e6 for k, v in results.items()},
-                "errors": errors or None}
+                "timing": timing, "errors": errors or None}
 
     def decode_only_graph(self, reps):
         """reps x (32 layers of tq_decode_attention) at the final context length."""
