@@ -1373,7 +1373,10 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
 // tile of codes or sign bits:
 //   n-tile 0: column 2h = Q2 of head h, column 2h + 1 = Q1 of head h,
 //   n-tile 1: column 2h = Q0 of head h, column 2h + 1 = 0,
-// so that lane (g, t) of the accumulator sees all three limbs of head t. In
+// so that lane (g, t) of the accumulator sees all three limbs of head t. With
+// two or more groups (code keys), two groups share n-tile 1: column 2h + 1 then
+// holds Q0 of head h of the second group (put_frag_paired), which saves one
+// product in five per k-step for every second group. In
 // log2 units the logit is l2 = |k| <Q, C> a + gamma (2 <P, s> - sum P) b with
 // a = scale log2(e) 2^(-e_q - k_exp), b = scale log2(e) sqrt(pi/2)/m 2^(-e_p).
 constexpr int kGroupHeads = 4;
@@ -1580,6 +1583,28 @@ __device__ __forceinline__ void put_frag(uint4 (&frag)[4][32], int hj, int w, ui
   odd[sub] = q1;
   even[2 + sub] = q0;
   odd[2 + sub] = 0u;
+}
+
+// The same for group h of NH when groups are paired (two or more groups, code
+// keys): n-tile 1 of the even group of a pair carries the lowest limb of both,
+// column 2 hj for head hj of the even group and column 2 hj + 1 for head hj of
+// the odd one, so that one product serves both and lane (g, t) still finds the
+// lowest limbs of its own heads t and 4 + t in its accumulator. The odd group's
+// own n-tile 1 is never read; an unpaired last group keeps a zero column.
+template <int NH>
+__device__ __forceinline__ void put_frag_paired(uint4 (&frags)[NH][2][4][32], int which, int h, int hj, int w,
+                                                uint32_t q2, uint32_t q1, uint32_t q0) {
+  const int kt = w >> 3, sub = (w >> 2) & 1, tt = w & 3;
+  uint32_t* even = reinterpret_cast<uint32_t*>(&frags[h][which][kt][4 * (2 * hj) + tt]);
+  uint32_t* odd = reinterpret_cast<uint32_t*>(&frags[h][which][kt][4 * (2 * hj + 1) + tt]);
+  even[sub] = q2;
+  odd[sub] = q1;
+  if (h & 1) {
+    reinterpret_cast<uint32_t*>(&frags[h - 1][which][kt][4 * (2 * hj + 1) + tt])[2 + sub] = q0;
+  } else {
+    even[2 + sub] = q0;
+    if (h + 1 >= NH) odd[2 + sub] = 0u;
+  }
 }
 
 // Rotate and code one vector held 4 per lane; returns codes in o, n and (keys) gamma,
@@ -1908,7 +1933,8 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
     }
     const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
     const Limbs lq = split3(x, eq);
-    put_frag(P.qb[j >> 2][0], j & 3, lane, lq.w2, lq.w1, lq.w0);   // lane l: coordinates 4l .. 4l + 3
+    if constexpr (!KQ8 && NH >= 2) put_frag_paired<NH>(P.qb, 0, j >> 2, j & 3, lane, lq.w2, lq.w1, lq.w0);
+    else put_frag(P.qb[j >> 2][0], j & 3, lane, lq.w2, lq.w1, lq.w0);   // lane l: coordinates 4l .. 4l + 3
     if (lane == 0) {
       const bool real = j < A.group;
       P.cst[j][0] = real ? A.scale * kLog2e * pow2i(-eq - (KQ8 ? 0 : T.k_exp)) : 0.0f;
@@ -2018,8 +2044,13 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       ps += __shfl_xor_sync(kFull, ps, 16);
       if ((g & 3) == 0) {
         const int wd = 4 * skw + (g >> 2);
-        put_frag(P.qb[h][1], t, wd, w[2], w[1], w[0]);
-        put_frag(P.qb[h][1], t, wd + 2, w[5], w[4], w[3]);
+        if constexpr (NH >= 2) {
+          put_frag_paired<NH>(P.qb, 1, h, t, wd, w[2], w[1], w[0]);
+          put_frag_paired<NH>(P.qb, 1, h, t, wd + 2, w[5], w[4], w[3]);
+        } else {
+          put_frag(P.qb[h][1], t, wd, w[2], w[1], w[0]);
+          put_frag(P.qb[h][1], t, wd + 2, w[5], w[4], w[3]);
+        }
       }
       if (g == 0) {
         atomicAdd(reinterpret_cast<int*>(&P.cst[j][2]), j < A.group ? ps : 0);
@@ -2202,6 +2233,9 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
           const uint4 fp = P.qb[h][1][kt][lane];
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
+            if constexpr (NH >= 2) {
+              if (nt == 1 && (h & 1)) continue;              // the pair's even group serves n-tile 1
+            }
             const uint32_t q0 = nt ? fq.z : fq.x, q1 = nt ? fq.w : fq.y;
             const uint32_t r0 = nt ? fp.z : fp.x, r1 = nt ? fp.w : fp.y;
             mma_s8(dh[h][nt], ah, q0, q1);
@@ -2229,10 +2263,21 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
         if constexpr (KQ8) {
           l2 = ca[h] * lq8[h][r];
         } else {
-          const int hiw = 256 * dh[h][0][2 * r] + dl[h][0][2 * r] + dh[h][0][2 * r + 1];
-          const int low = 256 * (dl[h][0][2 * r + 1] + dh[h][1][2 * r]);
+          int hiw, low, sj;
+          if constexpr (NH == 1) {
+            hiw = 256 * dh[h][0][2 * r] + dl[h][0][2 * r] + dh[h][0][2 * r + 1];
+            low = 256 * (dl[h][0][2 * r + 1] + dh[h][1][2 * r]);
+            sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + ds[h][1][2 * r];
+          } else {
+            // the lowest limbs: n-tile 1 of this group, or (the odd group of a pair)
+            // column 2t + 1 of the even group's
+            const int q0t = (h & 1) ? dh[h & ~1][1][2 * r + 1] : dh[h][1][2 * r];
+            const int p0t = (h & 1) ? ds[h & ~1][1][2 * r + 1] : ds[h][1][2 * r];
+            hiw = 256 * dh[h][0][2 * r] + dl[h][0][2 * r] + dh[h][0][2 * r + 1];
+            low = 256 * (dl[h][0][2 * r + 1] + q0t);
+            sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + p0t;
+          }
           const float main = fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
-          const int sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + ds[h][1][2 * r];
           const float nk = r ? nK.y : nK.x, gg = r ? gm.y : gm.x;
           l2 = fmaf(nk * ca[h], main, gg * cb[h] * static_cast<float>(2 * sj - csum[h]));
         }
