@@ -1376,7 +1376,11 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) quantize_prefill_tc_kernel(
 // so that lane (g, t) of the accumulator sees all three limbs of head t. With
 // two or more groups (code keys), two groups share n-tile 1: column 2h + 1 then
 // holds Q0 of head h of the second group (put_frag_paired), which saves one
-// product in five per k-step for every second group. In
+// product in five per k-step for every second group. With 4-bit keys and two or
+// more groups the key term instead runs on fp16 tensor cores: the centroids are
+// fp16 values, looked up in pairs from a byte-indexed table, and q~ 2^sig is split
+// into fp16 high and low parts (columns 2h, 2h + 1 of one n-tile), two m16n8k16
+// products per k-tile and group; the sign term keeps its int8 limbs. In
 // log2 units the logit is l2 = |k| <Q, C> a + gamma (2 <P, s> - sum P) b with
 // a = scale log2(e) 2^(-e_q - k_exp), b = scale log2(e) sqrt(pi/2)/m 2^(-e_p).
 constexpr int kGroupHeads = 4;
@@ -1674,6 +1678,7 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   constexpr bool APPEND = MODE == 1;        // append the new token first (decode step)
   constexpr bool LOGITS = MODE == 2;        // write the logits; no softmax, no value sum
   constexpr bool KQ8 = BK == 8;              // q8_0 keys (raw query, block scales, no QJL)
+  constexpr bool KF16 = BK == 4 && NH >= 2;  // 4-bit keys, two or more head groups: fp16 key products
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int W = DecodeWarps<NH, LOOP>::value;
   constexpr int kBlock = block_bytes_of(BK, BV);
@@ -1747,6 +1752,13 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
   // and for 4-bit keys the limb pairs need two more byte-permutes per load: both
   // stay on the byte-permute lookups.
   __shared__ uint32_t s_vtab[BV == 4 && !LOGITS ? 256 : 1];
+  // 4-bit keys: entry b = fp16x2 (c(b & 15), c(b >> 4)) of the key centroids (fp16
+  // values), the A-operand pairs of the fp16 key products
+  __shared__ uint32_t s_ktab[KF16 ? 256 : 1];
+  if constexpr (KF16) {
+    for (int e = threadIdx.x; e < 256; e += blockDim.x)
+      s_ktab[e] = pack_half2(T.cen_k[e & 15], T.cen_k[e >> 4]);
+  }
   if constexpr (BV == 4 && !LOGITS) {
     auto byte_of = [](const uint32_t (&tb)[4], int c) -> uint32_t { return (tb[c >> 2] >> (8 * (c & 3))) & 0xFFu; };
     for (int e = threadIdx.x; e < 256; e += blockDim.x)
@@ -1931,13 +1943,39 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
 #pragma unroll
       for (int e = 0; e < 4; ++e) x[e] *= kInvSqrtD;
     }
-    const int eq = pick_exponent24(warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])))));
-    const Limbs lq = split3(x, eq);
-    if constexpr (!KQ8 && NH >= 2) put_frag_paired<NH>(P.qb, 0, j >> 2, j & 3, lane, lq.w2, lq.w1, lq.w0);
-    else put_frag(P.qb[j >> 2][0], j & 3, lane, lq.w2, lq.w1, lq.w0);   // lane l: coordinates 4l .. 4l + 3
+    const float qmax = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+    int eq;
+    if constexpr (KF16) {
+      // q~ 2^sig as fp16 high and low parts (|q~ 2^sig| < 2^10) in the B order of the
+      // fp16 key products: k-tile kt, half jh = coordinates 32 kt + 16 jh + 4 t' + 0..3
+      // at lane (g', t'), column g' = 2 (head) + part; this lane holds the four
+      // coordinates 4 lane .. 4 lane + 3, i.e. kt = lane >> 3, jh = (lane >> 2) & 1, t' = lane & 3
+      const int E = qmax > 0.0f ? max(exp_above(qmax), -100) : 0;
+      eq = 10 - E;
+      const float sc = pow2i(eq);
+      float hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float v = x[e] * sc;
+        hi[e] = __half2float(__float2half_rn(v));
+        lo[e] = v - hi[e];
+      }
+      const int kt = lane >> 3, jh = (lane >> 2) & 1, tt = lane & 3, hj = j & 3;
+      uint32_t* ph = reinterpret_cast<uint32_t*>(&P.qb[j >> 2][0][kt][4 * (2 * hj) + tt]);
+      uint32_t* pl = reinterpret_cast<uint32_t*>(&P.qb[j >> 2][0][kt][4 * (2 * hj + 1) + tt]);
+      ph[2 * jh] = pack_half2(hi[0], hi[1]);
+      ph[2 * jh + 1] = pack_half2(hi[2], hi[3]);
+      pl[2 * jh] = pack_half2(lo[0], lo[1]);
+      pl[2 * jh + 1] = pack_half2(lo[2], lo[3]);
+    } else {
+      eq = pick_exponent24(qmax);
+      const Limbs lq = split3(x, eq);
+      if constexpr (!KQ8 && NH >= 2) put_frag_paired<NH>(P.qb, 0, j >> 2, j & 3, lane, lq.w2, lq.w1, lq.w0);
+      else put_frag(P.qb[j >> 2][0], j & 3, lane, lq.w2, lq.w1, lq.w0);   // lane l: coordinates 4l .. 4l + 3
+    }
     if (lane == 0) {
       const bool real = j < A.group;
-      P.cst[j][0] = real ? A.scale * kLog2e * pow2i(-eq - (KQ8 ? 0 : T.k_exp)) : 0.0f;
+      P.cst[j][0] = real ? A.scale * kLog2e * pow2i(-eq - (KQ8 || KF16 ? 0 : T.k_exp)) : 0.0f;
       if (KQ8) {
         P.cst[j][1] = 0.0f;
         P.cst[j][2] = __int_as_float(0);
@@ -2173,12 +2211,16 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
 
     // ---- logits: int8 tensor-core products, tokens on the rows
     int dh[NH][2][4], dl[NH][2][4], ds[NH][2][4];
+    float dk[NH][4];                          // 4-bit keys: fp16 products (columns: head t high, low part)
 #pragma unroll
-    for (int h = 0; h < NH; ++h)
+    for (int h = 0; h < NH; ++h) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) dh[h][nt][c] = dl[h][nt][c] = ds[h][nt][c] = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) dk[h][c] = 0.0f;
+    }
     float lq8[NH][2];                        // q8_0: sum over blocks of d_b <Q_b, k8_b>
     if constexpr (KQ8) {
       float dsc[2][4];
@@ -2214,15 +2256,39 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       }
     } else {
       uint32_t sel0[8], sel1[8];
-      key_selectors<BK>(kw, sel0);
-      key_selectors<BK>(kw + BK, sel1);
+      if constexpr (!KF16) {
+        key_selectors<BK>(kw, sel0);
+        key_selectors<BK>(kw + BK, sel1);
+      }
+      const uint8_t* kt8 = reinterpret_cast<const uint8_t*>(s_ktab);
 #pragma unroll
       for (int kt = 0; kt < 4; ++kt) {
         uint32_t ah[4], al[4], as[4];
-        key_limbs<BK>(sel0[2 * kt], kth_, ktl_, ah[0], al[0]);          // token g,     k 4t..
-        key_limbs<BK>(sel1[2 * kt], kth_, ktl_, ah[1], al[1]);          // token g + 8, k 4t..
-        key_limbs<BK>(sel0[2 * kt + 1], kth_, ktl_, ah[2], al[2]);      // token g,     k 16+4t..
-        key_limbs<BK>(sel1[2 * kt + 1], kth_, ktl_, ah[3], al[3]);      // token g + 8, k 16+4t..
+        if constexpr (KF16) {
+          // word kt of token g (g + 8): byte 0 = coordinates 4t, 4t + 1, byte 1 = 4t + 2, 4t + 3,
+          // bytes 2, 3 the same 16 coordinates on: the A pairs of the two k-halves
+          const uint32_t w0 = kw[kt], w1 = kw[4 + kt];
+          uint32_t a[8];
+          a[0] = *reinterpret_cast<const uint32_t*>(kt8 + ((w0 << 2) & 0x3FCu));
+          a[1] = *reinterpret_cast<const uint32_t*>(kt8 + ((w1 << 2) & 0x3FCu));
+          a[2] = *reinterpret_cast<const uint32_t*>(kt8 + (shr<6>(w0) & 0x3FCu));
+          a[3] = *reinterpret_cast<const uint32_t*>(kt8 + (shr<6>(w1) & 0x3FCu));
+          a[4] = *reinterpret_cast<const uint32_t*>(kt8 + (shr<14>(w0) & 0x3FCu));
+          a[5] = *reinterpret_cast<const uint32_t*>(kt8 + (shr<14>(w1) & 0x3FCu));
+          a[6] = *reinterpret_cast<const uint32_t*>(kt8 + (shr<22>(w0) & 0x3FCu));
+          a[7] = *reinterpret_cast<const uint32_t*>(kt8 + (shr<22>(w1) & 0x3FCu));
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            const uint4 fq = P.qb[h][0][kt][lane];
+            mma_f16(dk[h], a[0], a[1], a[2], a[3], fq.x, fq.y);
+            mma_f16(dk[h], a[4], a[5], a[6], a[7], fq.z, fq.w);
+          }
+        } else {
+          key_limbs<BK>(sel0[2 * kt], kth_, ktl_, ah[0], al[0]);          // token g,     k 4t..
+          key_limbs<BK>(sel1[2 * kt], kth_, ktl_, ah[1], al[1]);          // token g + 8, k 4t..
+          key_limbs<BK>(sel0[2 * kt + 1], kth_, ktl_, ah[2], al[2]);      // token g,     k 16+4t..
+          key_limbs<BK>(sel1[2 * kt + 1], kth_, ktl_, ah[3], al[3]);      // token g + 8, k 16+4t..
+        }
         as[0] = (kt == 0 ? sw.x : __umulhi(sw.x, 1u << (32 - 2 * kt))) & 0x01010101u;
         as[1] = (kt == 0 ? sw.y : __umulhi(sw.y, 1u << (32 - 2 * kt))) & 0x01010101u;
         as[2] = __umulhi(sw.x, 1u << (31 - 2 * kt)) & 0x01010101u;
@@ -2238,8 +2304,10 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
             }
             const uint32_t q0 = nt ? fq.z : fq.x, q1 = nt ? fq.w : fq.y;
             const uint32_t r0 = nt ? fp.z : fp.x, r1 = nt ? fp.w : fp.y;
-            mma_s8(dh[h][nt], ah, q0, q1);
-            if (nt == 0) mma_s8(dl[h][nt], al, q0, q1);   // Q0 x C_lo (below 2^-22 of the sum) is left out
+            if constexpr (!KF16) {
+              mma_s8(dh[h][nt], ah, q0, q1);
+              if (nt == 0) mma_s8(dl[h][nt], al, q0, q1);   // Q0 x C_lo (below 2^-22 of the sum) is left out
+            }
             mma_s8(ds[h][nt], as, r0, r1);
           }
         }
@@ -2277,7 +2345,8 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
             low = 256 * (dl[h][0][2 * r + 1] + q0t);
             sj = 65536 * ds[h][0][2 * r] + 256 * ds[h][0][2 * r + 1] + p0t;
           }
-          const float main = fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
+          const float main = KF16 ? dk[h][2 * r] + dk[h][2 * r + 1]
+                                  : fmaf(65536.0f, static_cast<float>(hiw), static_cast<float>(low));
           const float nk = r ? nK.y : nK.x, gg = r ? gm.y : gm.x;
           l2 = fmaf(nk * ca[h], main, gg * cb[h] * static_cast<float>(2 * sj - csum[h]));
         }
