@@ -48,11 +48,13 @@ def _lens(rng, n, hi, zeros):
     return [int(x) for x in lens]
 
 
-@pytest.mark.parametrize("n_seq,n_kv,g,hi,zeros", [(20, 8, 4, 300, 3), (8, 4, 4, 2500, 1), (40, 4, 12, 120, 5),
-                                                   (8, 4, 8, 2500, 1), (20, 8, 8, 300, 3)])
-def test_balanced_decode_matches_oracle(n_seq, n_kv, g, hi, zeros):
+@pytest.mark.parametrize("n_seq,n_kv,g,hi,zeros,bk,bv", [(20, 8, 4, 300, 3, 3, 2), (8, 4, 4, 2500, 1, 3, 2),
+                                                         (40, 4, 12, 120, 5, 3, 2), (8, 4, 8, 2500, 1, 3, 2),
+                                                         (20, 8, 8, 300, 3, 3, 2), (40, 4, 12, 120, 5, 4, 2),
+                                                         (20, 8, 8, 300, 3, 4, 4)])
+def test_balanced_decode_matches_oracle(n_seq, n_kv, g, hi, zeros, bk, bv):
     seq_lens = _lens(np.random.default_rng(n_seq + hi), n_seq, hi, zeros)
-    tab, _, _, cache_np, bt, n_pages, q, ctx = _case(seq_lens, n_kv, g, seed=n_seq)
+    tab, _, _, cache_np, bt, n_pages, q, ctx = _case(seq_lens, n_kv, g, seed=n_seq, bk=bk, bv=bv)
     max_len = max(seq_lens)
     ws = torch.zeros(ctx.decode_workspace_bytes(n_seq, n_kv * g, n_kv, max_len), dtype=torch.uint8, device=DEV)
     out = torch.full((n_seq, n_kv * g, 128), float("nan"), device=DEV)

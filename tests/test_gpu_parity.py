@@ -197,6 +197,15 @@ def test_decode_gqa_groups(g):
     print("worst rel err", assert_outputs_close(got, want))
 
 
+@pytest.mark.parametrize("g,bv", [(8, 2), (12, 4), (8, 3)])
+def test_decode_4bit_keys_head_groups(g, bv):
+    """4-bit keys with two or three groups of 4 query heads: the key term on fp16
+    tensor cores (centroid pairs from the byte table, q~ in fp16 high and low parts),
+    the sign term on the int8 limbs, the lowest sketch limbs of two groups in one n-tile."""
+    got, want = _decode_case(4, bv, [333, 17, 64], n_kv=2, g=g, seed=70 + g + bv)
+    print("worst rel err", assert_outputs_close(got, want))
+
+
 def test_decode_long_context_many_chunks():
     # spans many split-K chunks with a ragged final page
     got, want = _decode_case(3, 2, [4000, 2500], n_kv=1, g=4, seed=7)
