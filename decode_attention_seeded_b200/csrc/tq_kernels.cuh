@@ -1560,7 +1560,8 @@ constexpr int kQrawPitch = 136;     // floats per raw query row: the sketch's B 
 template <int NH>
 struct alignas(16) Prologue {
   alignas(16) float qraw[NH * kGroupHeads][kQrawPitch];   // queries as given (fp32)
-  alignas(16) uint4 qb[NH][2][4][32];              // B fragments [group][q~ / p][k-tile][lane] (see put_frag)
+  alignas(16) uint4 qb[NH][2][4][32];              // B fragments [group][q~ / p][k-tile][lane] (see put_frag;
+                                                   // with fp16 key products, q~ as fp16 pairs for both k-halves)
   alignas(16) float cst[NH * kGroupHeads][4];      // a, b, sum P (int bits)
   alignas(16) float qn[NH * kGroupHeads];          // |q|
   alignas(16) float u[128];                        // appended key: R_K^T u (original domain)
