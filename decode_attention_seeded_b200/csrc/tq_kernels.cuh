@@ -2266,8 +2266,9 @@ __device__ __forceinline__ void decode_segment(const Tables& T, const DecodeArgs
       for (int kt = 0; kt < 4; ++kt) {
         uint32_t ah[4], al[4], as[4];
         if constexpr (KF16) {
-          // word kt of token g (g + 8): byte 0 = coordinates 4t, 4t + 1, byte 1 = 4t + 2, 4t + 3,
-          // bytes 2, 3 the same 16 coordinates on: the A pairs of the two k-halves
+          // word kt of token g (g + 8): byte 0 = coordinates 4t, 4t + 1 and byte 1 = 4t + 2, 4t + 3
+          // (the A pairs of the first k-half), bytes 2, 3 = coordinates 16 + 4t .. 16 + 4t + 3
+          // (the second k-half); the B fragments use the same coordinate order
           const uint32_t w0 = kw[kt], w1 = kw[4 + kt];
           uint32_t a[8];
           a[0] = *reinterpret_cast<const uint32_t*>(kt8 + ((w0 << 2) & 0x3FCu));
